@@ -1,0 +1,258 @@
+"""Test helpers: small paged cases built from contiguous K/V, and the
+independent checks the oracle is pinned to.
+
+Every case starts from contiguous per-sequence K and V and scatters them into
+a NaN-filled pool through a random block table, so that the dense and
+brute-force checks below never look at the paged layout.
+"""
+from __future__ import annotations
+
+from decimal import Decimal, getcontext
+
+import numpy as np
+import scipy.special
+
+from workloads import nan_bits, to_storage_bits
+
+
+def widen_bits(bits: np.ndarray, dtype: str) -> np.ndarray:
+    """uint16 patterns -> float64 via numpy's own fp16 / fp32 conversions."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    if dtype == "f16":
+        return bits.view(np.float16).astype(np.float64)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def paged_case(rng, ctx_list, H, D, bs, num_blocks=None, dtype="f16", scale=None):
+    """Contiguous K/V per sequence, scattered into a pool [NB, H, bs, D]."""
+    ctx_list = [int(c) for c in ctx_list]
+    S = len(ctx_list)
+    nblk = [-(-c // bs) for c in ctx_list]
+    need = sum(nblk)
+    NB = num_blocks if num_blocks is not None else need + 3
+    perm = rng.permutation(NB)
+    nan = nan_bits(dtype)
+    kpool = np.full((NB, H, bs, D), nan, dtype=np.uint16)
+    vpool = np.full((NB, H, bs, D), nan, dtype=np.uint16)
+    MB = max(1, max(nblk, default=1))
+    bt = np.full((S, MB), -1, dtype=np.int32)
+    K, V = [], []
+    nxt = 0
+    for s, c in enumerate(ctx_list):
+        blocks = perm[nxt: nxt + nblk[s]]
+        nxt += nblk[s]
+        bt[s, : nblk[s]] = blocks
+        k = to_storage_bits(rng.standard_normal((c, H, D), dtype=np.float32), dtype)
+        v = to_storage_bits(rng.standard_normal((c, H, D), dtype=np.float32), dtype)
+        if c:
+            j = np.arange(c)
+            kpool[blocks[j // bs], :, j % bs, :] = k
+            vpool[blocks[j // bs], :, j % bs, :] = v
+        K.append(k)
+        V.append(v)
+    q = to_storage_bits(rng.standard_normal((S, H, D), dtype=np.float32), dtype)
+    if scale is None:
+        scale = np.float32(1.0 / np.sqrt(D))
+    return dict(q=q, K=K, V=V, kpool=kpool, vpool=vpool, bt=bt,
+                ctx=np.array(ctx_list, dtype=np.int32), scale=np.float32(scale),
+                dtype=dtype, bs=bs)
+
+
+def dense_attention(q, K, V, scale, dtype="f16"):
+    """softmax(scale q K^T) V on the unpaged copy, through scipy's softmax.
+    q [H, D], K/V [n, H, D] as uint16 patterns; returns float64 [H, D]."""
+    qf = widen_bits(q, dtype)
+    if K.shape[0] == 0:
+        return np.zeros_like(qf)
+    Kf, Vf = widen_bits(K, dtype), widen_bits(V, dtype)
+    scores = float(scale) * np.einsum("hd,nhd->hn", qf, Kf)
+    p = scipy.special.softmax(scores, axis=-1)
+    return np.einsum("hn,nhd->hd", p, Vf)
+
+
+def brute_force(q, K, V, scale, dtype="f16", digits=50):
+    """The same quantity in 50-digit decimal arithmetic, one (head) at a time.
+    Returns float64 [H, D]."""
+    getcontext().prec = digits
+    qf, Kf, Vf = widen_bits(q, dtype), widen_bits(K, dtype), widen_bits(V, dtype)
+    H, D = qf.shape
+    n = Kf.shape[0]
+    sc = Decimal(float(scale))
+    out = np.zeros((H, D))
+    for h in range(H):
+        if n == 0:
+            continue
+        qd = [Decimal(float(x)) for x in qf[h]]
+        s = []
+        for j in range(n):
+            s.append(sc * sum(qd[d] * Decimal(float(Kf[j, h, d])) for d in range(D)))
+        m = max(s)
+        w = [(x - m).exp() for x in s]
+        z = sum(w)
+        for d in range(D):
+            out[h, d] = float(sum(w[j] * Decimal(float(Vf[j, h, d])) for j in range(n)) / z)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Pins. Each takes an oracle.Oracle and raises AssertionError on a mismatch.
+# ---------------------------------------------------------------------------
+
+def _decode_case(orc, c):
+    return orc.decode(c["q"], c["kpool"], c["vpool"], c["bt"], c["ctx"], c["scale"],
+                      c["dtype"])
+
+
+def pin_dense(orc, seed=11):
+    rng = np.random.default_rng(seed)
+    for H, D, bs, ctxs, dtype in [
+        (2, 64, 16, [1, 15, 16, 17, 40], "f16"),
+        (3, 128, 8, [7, 64, 100], "f16"),
+        (2, 128, 32, [31, 33, 200], "f16"),
+        (2, 64, 16, [5, 50], "bf16"),
+    ]:
+        c = paged_case(rng, ctxs, H, D, bs, dtype=dtype)
+        got = _decode_case(orc, c)
+        for s in range(len(ctxs)):
+            ref = dense_attention(c["q"][s], c["K"][s], c["V"][s], c["scale"], dtype)
+            err = np.max(np.abs(got[s] - ref))
+            assert err <= 1e-12, f"dense mismatch {err} (H{H} D{D} bs{bs} s{s})"
+
+
+def pin_bruteforce(orc, seed=12):
+    rng = np.random.default_rng(seed)
+    c = paged_case(rng, [1, 17, 33, 100], 4, 64, 16, scale=0.125)
+    got = _decode_case(orc, c)
+    for s in range(4):
+        ref = brute_force(c["q"][s], c["K"][s], c["V"][s], c["scale"])
+        err = np.max(np.abs(got[s] - ref))
+        assert err <= 1e-12, f"brute-force mismatch {err} (seq {s})"
+
+
+def pin_closed_forms(orc, seed=13):
+    rng = np.random.default_rng(seed)
+    H, D, bs = 2, 64, 16
+    # ctx = 1: the output is the single value row, exactly.
+    c = paged_case(rng, [1, 1], H, D, bs)
+    got = _decode_case(orc, c)
+    for s in range(2):
+        assert np.array_equal(got[s], widen_bits(c["V"][s][0], "f16")), "ctx=1 != v0"
+    # scale = 0: uniform weights, the output is the mean of the value rows.
+    c = paged_case(rng, [37, 5], H, D, bs, scale=0.0)
+    got = _decode_case(orc, c)
+    for s in range(2):
+        ref = widen_bits(c["V"][s], "f16").mean(axis=0)
+        assert np.max(np.abs(got[s] - ref)) <= 1e-13, "scale=0 != mean(V)"
+    # All keys equal: again the mean of the value rows.
+    c = paged_case(rng, [23], H, D, bs)
+    row = c["K"][0][0].copy()
+    c["K"][0][:] = row
+    j = np.arange(23)
+    c["kpool"][c["bt"][0][j // bs], :, j % bs, :] = c["K"][0]
+    got = _decode_case(orc, c)
+    ref = widen_bits(c["V"][0], "f16").mean(axis=0)
+    assert np.max(np.abs(got[0] - ref)) <= 1e-13, "equal keys != mean(V)"
+    # Two tokens: o = (v0 + e^d v1) / (1 + e^d), d = scale (q.k1 - q.k0).
+    c = paged_case(rng, [2], H, D, bs)
+    qf = widen_bits(c["q"][0], "f16")
+    kf, vf = widen_bits(c["K"][0], "f16"), widen_bits(c["V"][0], "f16")
+    got = _decode_case(orc, c)
+    for h in range(H):
+        d = float(c["scale"]) * (qf[h] @ kf[1, h] - qf[h] @ kf[0, h])
+        a = 1.0 / (1.0 + np.exp(d))
+        ref = a * vf[0, h] + (1.0 - a) * vf[1, h]
+        assert np.max(np.abs(got[0, h] - ref)) <= 1e-13, "two-token closed form"
+    # One dominant token with scores in the thousands: the output is that
+    # token's value row (and nothing overflows).
+    c = paged_case(rng, [50], H, D, bs, scale=np.float32(64.0))
+    k = widen_bits(c["K"][0], "f16")
+    qf = widen_bits(c["q"][0], "f16")
+    got = _decode_case(orc, c)
+    checked = 0
+    for h in range(H):
+        sc = k[:, h] @ qf[h]
+        top = np.argsort(sc)[-2:]
+        assert np.all(np.isfinite(got[0, h])), "overflow with large scores"
+        if 64.0 * (sc[top[1]] - sc[top[0]]) > 60:
+            ref = widen_bits(c["V"][0][top[1], h], "f16")
+            assert np.max(np.abs(got[0, h] - ref)) <= 1e-12, "dominant token"
+            checked += 1
+    assert checked >= 1, "no head had a dominant token; change the seed"
+
+
+def pin_permutation(orc, seed=14):
+    """Moving every physical block to another id (and the tables with it)
+    leaves the output bit-identical."""
+    rng = np.random.default_rng(seed)
+    c = paged_case(rng, [3, 16, 41, 90], 3, 64, 16, num_blocks=24)
+    got = _decode_case(orc, c)
+    NB = c["kpool"].shape[0]
+    pi = rng.permutation(NB)
+    k2 = np.empty_like(c["kpool"])
+    v2 = np.empty_like(c["vpool"])
+    k2[pi] = c["kpool"]
+    v2[pi] = c["vpool"]
+    bt2 = np.where(c["bt"] >= 0, pi[np.maximum(c["bt"], 0)], -1).astype(np.int32)
+    got2 = orc.decode(c["q"], k2, v2, bt2, c["ctx"], c["scale"])
+    assert np.array_equal(got, got2), "not invariant under a block permutation"
+
+
+def pin_write_kv(orc, seed=15):
+    """Appending tokens one by one through slots fills a sequence so that the
+    gathered cache equals the tokens written; nothing else changes."""
+    rng = np.random.default_rng(seed)
+    H, D, bs, NB = 2, 64, 8, 12
+    nan = nan_bits("f16")
+    kc = np.full((NB, H, bs, D), nan, dtype=np.uint16)
+    vc = kc.copy()
+    blocks = rng.permutation(NB)[:4]
+    n = 29
+    toks_k = to_storage_bits(rng.standard_normal((n, H, D), dtype=np.float32), "f16")
+    toks_v = to_storage_bits(rng.standard_normal((n, H, D), dtype=np.float32), "f16")
+    for t in range(n):  # one token per decode step, like the engine does
+        slot = np.array([blocks[t // bs] * bs + t % bs], dtype=np.int64)
+        orc.write_kv(toks_k[t:t + 1], toks_v[t:t + 1], slot, kc, vc, bs)
+    for t in range(n):
+        assert np.array_equal(kc[blocks[t // bs], :, t % bs, :], toks_k[t]), "K slot"
+        assert np.array_equal(vc[blocks[t // bs], :, t % bs, :], toks_v[t]), "V slot"
+    written = np.zeros((NB, bs), dtype=bool)
+    for t in range(n):
+        written[blocks[t // bs], t % bs] = True
+    assert np.all(kc.transpose(0, 2, 1, 3)[~written] == nan), "K written elsewhere"
+    assert np.all(vc.transpose(0, 2, 1, 3)[~written] == nan), "V written elsewhere"
+    # A negative slot is padding: nothing is written.
+    before = kc.copy()
+    orc.write_kv(toks_k[:1], toks_v[:1], np.array([-1], dtype=np.int64), kc, vc, bs)
+    assert np.array_equal(before, kc), "padding slot wrote"
+    # The round trip through the oracle's own decode: a sequence whose K/V
+    # went in through write_kv decodes like the dense copy.
+    bt = np.full((1, 4), -1, dtype=np.int32)
+    bt[0] = blocks
+    q = to_storage_bits(rng.standard_normal((1, H, D), dtype=np.float32), "f16")
+    got = orc.decode(q, kc, vc, bt, np.array([n], dtype=np.int32), np.float32(0.125))
+    ref = dense_attention(q[0], toks_k, toks_v, np.float32(0.125))
+    assert np.max(np.abs(got[0] - ref)) <= 1e-12, "write_kv round trip"
+
+
+def pin_copy_blocks(orc, seed=16):
+    rng = np.random.default_rng(seed)
+    L, NB, H, bs, D = 3, 10, 2, 16, 64
+    ks = [rng.integers(0, 1 << 16, size=(NB, H, bs, D), dtype=np.uint16) for _ in range(L)]
+    vs = [rng.integers(0, 1 << 16, size=(NB, H, bs, D), dtype=np.uint16) for _ in range(L)]
+    k0 = [k.copy() for k in ks]
+    v0 = [v.copy() for v in vs]
+    pairs = np.array([[1, 7], [4, 2], [9, 0]], dtype=np.int64)
+    orc.copy_blocks(ks, vs, pairs)
+    dsts = set(pairs[:, 1].tolist())
+    for l in range(L):
+        for src, dst in pairs:
+            assert np.array_equal(ks[l][dst], k0[l][src]), "K dst != src"
+            assert np.array_equal(vs[l][dst], v0[l][src]), "V dst != src"
+        for b in range(NB):
+            if b not in dsts:
+                assert np.array_equal(ks[l][b], k0[l][b]), "K block changed"
+                assert np.array_equal(vs[l][b], v0[l][b]), "V block changed"
+
+
+ALL_PINS = [pin_dense, pin_bruteforce, pin_closed_forms, pin_permutation, pin_write_kv,
+            pin_copy_blocks]
