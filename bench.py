@@ -1,0 +1,465 @@
+"""Benchmark: paged-attention decode query-tokens/s and achieved K/V-read HBM
+bandwidth on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl ours|reference]
+
+A step is one decode step of the whole hot path on one batch: copy-on-write
+block copies (when the workload has any), the K/V write of every sequence's
+new token, and decode attention (plus its reduce when the context is split),
+for every layer of the workload. The default workload is the Llama-7B-shaped
+single layer: 96 sequences, 32 heads, head_dim 128, block size 16, context
+lengths uniform in [128, 2048], an 8192-block pool.
+
+Under torchrun (N > 1) every rank runs an independent replica of the workload
+(the path has no exchange step); the time is the maximum over ranks and the
+value counts the query tokens of all ranks.
+
+--impl reference times the fp64 CPU oracle on this machine's host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged-attn decode query-tokens/s; achieved KV-read HBM GB/s vs B200 peak"
+UNIT = "query-tokens/s"
+NORTH_STAR_PEAK_GBS = 8000.0
+FALLBACK_PEAK_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+WORKLOADS = {
+    "tiny": (lambda seed: wl.tiny(seed=seed),
+             "tiny: 4 seqs, 4 heads, head_dim 64, block_size 16, ctx {1,17,33,100}, "
+             "64-block pool"),
+    "llama7b_layer": (lambda seed: wl.llama_layer(seed=seed),
+                      "llama7b_layer: 96 seqs, 32 heads, head_dim 128, block_size 16, "
+                      "ctx U[128,2048], 8192-block pool, write_kv + decode"),
+    "long_context": (lambda seed: wl.long_context(seed=seed),
+                     "long_context: 8 seqs, 32 heads, head_dim 128, block_size 16, "
+                     "ctx U[16384,32768], 20000-block pool, split decode + reduce"),
+    "prefix_cow": (lambda seed: wl.prefix_cow(seed=seed),
+                   "prefix_cow: 64 seqs sharing a 1024-token prefix, suffix U[1,512], "
+                   "32 heads, head_dim 128, copy_blocks + write_kv + decode"),
+    "full_step_bs8": (lambda seed: wl.full_step(seed=seed, block_size=8),
+                      "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 8"),
+    "full_step_bs16": (lambda seed: wl.full_step(seed=seed, block_size=16),
+                       "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 16"),
+    "full_step_bs32": (lambda seed: wl.full_step(seed=seed, block_size=32),
+                       "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 32"),
+}
+SEEDS = {"tiny": 0, "llama7b_layer": 1, "long_context": 2, "prefix_cow": 3,
+         "full_step_bs8": 4, "full_step_bs16": 4, "full_step_bs32": 4}
+
+
+def algorithmic_bytes(step) -> dict:
+    """Bytes one decode over one layer must move: every context token's K and
+    V row (head_dim x 2 bytes, all heads), the query and output rows and the
+    block-table entries it reads. Over-reads of partly filled blocks are not
+    counted."""
+    H, D = step.num_heads, step.head_dim
+    ctx = step.context_lens.astype(np.int64)
+    kv = int(ctx.sum()) * H * D * 2 * 2
+    qo = step.num_seqs * H * D * 2 * 2
+    table = int(np.sum(-(-ctx // step.block_size))) * 4
+    return {"kv": kv, "total": kv + qo + table}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_417_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_PEAK_GBS, "fallback"
+
+
+def recorded_traffic(config):
+    """DRAM bytes per decode launch from an ncu capture, if one was taken on
+    the current kernel sources (profiles/traffic.json); else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(config)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons while the GPU works."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_uuid):
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if device_uuid:
+            cmd[1:1] = ["-i", device_uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.strip()]
+        os.unlink(self.out.name)
+        sm, smax, reasons = [], [], set()
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def device_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------
+# The oracle on the host cores (cpu_baseline, and the reference arm).
+# ----------------------------------------------------------------------------
+
+def oracle_inputs(sub, layers):
+    """Host pools of a sub-step (input generation, outside any timing)."""
+    return [wl.host_pools(sub, li) for li in layers]
+
+
+def time_oracle(sub, layers, pools):
+    """Seconds the oracle takes for the whole step of ``sub`` on ``layers``:
+    copy-on-write, K/V write, decode."""
+    import oracle
+    t0 = time.perf_counter()
+    for li, (kc, vc) in zip(layers, pools):
+        L = sub.layers[li]
+        oracle.copy_blocks([kc], [vc], sub.copy_pairs)
+        oracle.write_kv(L.new_key, L.new_value, sub.slot_mapping, kc, vc, sub.block_size)
+        oracle.decode(L.query, kc, vc, sub.block_tables, sub.context_lens, float(sub.scale),
+                      sub.dtype)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(step, target_seconds):
+    """A sub-batch of ``step`` whose oracle run on one layer takes about
+    ``target_seconds``."""
+    order = np.random.default_rng(123).permutation(step.num_seqs)
+    probe = wl.subset(step, order[:1])
+    t1 = time_oracle(probe, [0], oracle_inputs(probe, [0]))
+    per_token = t1 / max(1, int(probe.context_lens.sum()))
+    budget = target_seconds / max(per_token, 1e-9)
+    ids, tokens = [], 0
+    for s in order:
+        if ids and tokens + int(step.context_lens[s]) > budget:
+            break
+        ids.append(int(s))
+        tokens += int(step.context_lens[s])
+    return wl.subset(step, sorted(ids))
+
+
+def cpu_baseline(step, target_seconds=15.0):
+    import oracle
+    layers = [0] if step.num_layers == 1 else [0, step.num_layers - 1]
+    sub = oracle_sample(step, target_seconds / len(layers))
+    secs = time_oracle(sub, layers, oracle_inputs(sub, layers))
+    value = sub.num_seqs * len(layers) / (secs * step.num_layers)
+    return {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"{sub.num_seqs} of {step.num_seqs} sequences x {len(layers)} of "
+                       f"{step.num_layers} layers (copy-on-write, K/V write, decode), fp64 C "
+                       f"+ OpenMP, {secs:.1f} s; value scaled to whole decode steps")}
+
+
+def max_over_ranks(x, dist=None, device=None):
+    """The maximum of a per-rank number over all ranks (identity alone)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, seqs_per_rank, steps, max_ms):
+    """Query tokens of all ranks per second of the slowest rank."""
+    return world * seqs_per_rank * steps / (max_ms / 1e3)
+
+
+def run_reference(args, config_desc):
+    step = WORKLOADS[args.config][0](SEEDS[args.config])
+    sub = oracle_sample(step, 2.0)
+    layers = [0]
+    pools = oracle_inputs(sub, layers)
+    for _ in range(args.warmup):
+        time_oracle(sub, layers, pools)
+    secs = 0.0
+    for _ in range(args.steps):
+        secs += time_oracle(sub, layers, pools)
+    value = sub.num_seqs * len(layers) * args.steps / (secs * step.num_layers)
+    import oracle
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": config_desc,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{sub.num_seqs} of {step.num_seqs} sequences, 1 of "
+                                   f"{step.num_layers} layers per step, scaled to whole steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# The CUDA path.
+# ----------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="llama7b_layer", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition", type=int, default=0)
+    ap.add_argument("--soak-seconds", type=float, default=1.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    flush = args.config != "prefix_cow"  # prefix reuse through L2 is part of that workload
+    config_desc = {"workload": WORKLOADS[args.config][1],
+                   "l2": "flushed between steps (256 MiB write)" if flush else
+                         "not flushed (shared-prefix reuse is part of the workload)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "partition": args.partition or "auto"}
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, config_desc)
+        return
+
+    import torch
+    import paged_kv_cache_417_b200 as pk
+    from workloads.device import device_step
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+
+    step = WORKLOADS[args.config][0](SEEDS[args.config] + 1000 * rank)
+    d = device_step(step, dev)
+    L, S = step.num_layers, step.num_seqs
+    stream = torch.cuda.current_stream(dev)
+    outs = [torch.empty_like(q) for q in d["query"]]
+    ws = pk.alloc_workspace(S, step.num_heads, step.head_dim, step.max_context_len,
+                            args.partition, dev)
+    P = pk.decode_partition_size(S, step.num_heads, step.head_dim, step.block_size,
+                                 step.max_context_len, args.partition)
+    split = step.max_context_len > P
+    has_copy = step.copy_pairs.shape[0] > 0
+    launches_per_step = (1 if has_copy else 0) + L * (2 + (1 if split else 0))
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def one_step(dec_events=None, inputs=None):
+        src = inputs or d
+        if has_copy:
+            pk.copy_blocks(d["key_caches"], d["value_caches"], src["copy_pairs"])
+        for li in range(L):
+            kc, vc = d["key_caches"][li], d["value_caches"][li]
+            pk.write_kv(src["new_key"][li], src["new_value"][li], src["slot_mapping"], kc, vc)
+            if dec_events is not None:
+                dec_events[0].append(torch.cuda.Event(enable_timing=True))
+                dec_events[0][-1].record(stream)
+            pk.decode(outs[li], src["query"][li], kc, vc, src["block_tables"],
+                      src["context_lens"], step.max_context_len, float(step.scale),
+                      partition_size=args.partition, workspace=ws)
+            if dec_events is not None:
+                dec_events[1].append(torch.cuda.Event(enable_timing=True))
+                dec_events[1][-1].record(stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # Warm-up, then an untimed soak so clocks settle and get sampled.
+    for _ in range(args.warmup):
+        one_step()
+    sampler = ClockSampler(device_uuid(torch, dev))
+    t_end = time.perf_counter() + args.soak_seconds
+    while time.perf_counter() < t_end:
+        for _ in range(10):
+            if flush:
+                flush_buf.zero_()
+            one_step()
+        torch.cuda.synchronize(dev)
+
+    # Timed region: K steps, L2 flushed between them, each step bracketed by
+    # CUDA events on the launching stream.
+    barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dec_events = ([], [])
+    for k in range(args.steps):
+        if flush:
+            flush_buf.zero_()
+        starts[k].record(stream)
+        one_step(dec_events)
+        ends[k].record(stream)
+    barrier()
+    clocks = sampler.stop()
+    step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    dec_ms = [a.elapsed_time(b) for a, b in zip(*dec_events)]
+    total_ms = max_over_ranks(step_ms, dist, dev)
+    value = job_throughput(world, S, args.steps, total_ms)
+
+    # Roofline of the dominant kernel (the decode call: decode + its reduce).
+    ab = algorithmic_bytes(step)
+    dec_avg_s = statistics.mean(dec_ms) / 1e3
+    achieved = ab["total"] / dec_avg_s / 1e9
+    peak, peak_kind = measured_peak()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(args.config),
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "kernel": "pa_decode (decode kernel + reduce kernel when split)",
+                "algorithmic_bytes_per_launch": ab["total"],
+                "kv_bytes_per_launch": ab["kv"],
+                "decode_us": dec_avg_s * 1e6,
+                "kv_gbs": ab["kv"] / dec_avg_s / 1e9,
+                "frac_of_8tbs": achieved / NORTH_STAR_PEAK_GBS}
+
+    # End to end through the public API with host buffers: pinned host ->
+    # device copies of the step's inputs, the step, device -> host output.
+    e2e = None
+    if not args.no_e2e:
+        host = {k: [t.cpu().pin_memory() for t in d[k]] for k in ("query", "new_key", "new_value")}
+        for k in ("slot_mapping", "block_tables", "context_lens", "copy_pairs"):
+            host[k] = d[k].cpu().pin_memory()
+        dev_in = {k: [torch.empty_like(t) for t in d[k]] for k in ("query", "new_key", "new_value")}
+        for k in ("slot_mapping", "block_tables", "context_lens", "copy_pairs"):
+            dev_in[k] = torch.empty_like(d[k])
+        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        h2d = sum(t.numel() * t.element_size() for k in ("query", "new_key", "new_value")
+                  for t in host[k])
+        h2d += sum(host[k].numel() * host[k].element_size()
+                   for k in ("slot_mapping", "block_tables", "context_lens"))
+        if has_copy:
+            h2d += host["copy_pairs"].numel() * 8
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+
+        def e2e_step():
+            for k in ("query", "new_key", "new_value"):
+                for a, b in zip(dev_in[k], host[k]):
+                    a.copy_(b, non_blocking=True)
+            for k in ("slot_mapping", "block_tables", "context_lens") + (
+                    ("copy_pairs",) if has_copy else ()):
+                dev_in[k].copy_(host[k], non_blocking=True)
+            one_step(inputs=dev_in)
+            for a, b in zip(host_out, outs):
+                a.copy_(b, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for k in range(args.steps):
+            if flush:
+                flush_buf.zero_()
+            es[k].record(stream)
+            e2e_step()
+            ee[k].record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(es, ee)), dist, dev)
+        e2e = {"value": job_throughput(world, S, args.steps, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(step)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": step.dtype,
+            "accumulate": "f32", "data": "synthetic", "config": config_desc,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+            "partition_size": P, "split": split,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

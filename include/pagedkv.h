@@ -1,0 +1,175 @@
+/*
+ * pagedkv.h - C ABI of a B200 (sm_100a) paged-KV-cache decode library.
+ *
+ * The method: PagedAttention keeps the KV cache in fixed-size physical blocks
+ * (16 tokens by default) that may lie anywhere in a pool; each sequence
+ * reaches its blocks through a block table that maps logical block i to a
+ * physical block id ("vLLM基础：架构、推理流程与关键组件", §2.3;
+ * "啃透vLLM源码", §2.2). Decode-step attention reads the caches through
+ * those physical block indices ("VLLM源码解析", core technology,
+ * paged_attention_forward). Shared blocks are copied before a sequence
+ * writes into them (copy-on-write, "vLLM基础", §2.3).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Cache layout: key_cache and value_cache are two separate device arrays
+ *   [num_blocks][num_kv_heads][block_size][head_dim] of 16-bit elements
+ *   (fp16 or bf16), row-major. Token t of a sequence lives in physical block
+ *   block_table[t / block_size] at offset t % block_size; its "slot" is
+ *   block * block_size + offset.
+ * - Supported shapes: head_dim 64 or 128; block_size 8, 16 or 32;
+ *   num_heads == num_kv_heads (one query head per KV head).
+ * - Ownership: the caller owns every buffer, including the decode
+ *   workspace. The library allocates no memory, keeps no per-call state and
+ *   never synchronises; every call only enqueues kernels on `stream` (a
+ *   cudaStream_t passed as void*, NULL = the legacy default stream) on the
+ *   current CUDA device. Calls are safe from several host threads.
+ * - Errors: arguments are checked on the host before anything is launched;
+ *   a failed check returns a status and launches nothing
+ *   (pa_last_error() then describes it). PA_ERR_CUDA means a launch failed.
+ *   Device-side checks (block ids, slots, context lengths, bounded waits)
+ *   cannot return a status; each call takes an optional device int32
+ *   `dev_err` (may be NULL) into which the kernels OR the PA_DEVERR_* bits
+ *   below. The caller zeroes it and reads it after synchronising.
+ * - Alignment: cache, key, value and query pointers must be 16-byte aligned,
+ *   and so must the workspace.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad alignment ... */
+    PA_ERR_UNSUPPORTED = 2, /* valid but not built: head_dim, block_size, GQA ... */
+    PA_ERR_WORKSPACE = 3,   /* decode workspace missing or too small */
+    PA_ERR_CUDA = 4         /* a CUDA launch or attribute call failed */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 } pa_dtype;
+
+/* Shape of one layer's K (and, identically, V) cache. dtype is PA_F16 or
+ * PA_BF16. */
+typedef struct {
+    int32_t num_blocks;
+    int32_t block_size;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+    pa_dtype dtype;
+} pa_cache_desc;
+
+/* Bits the kernels OR into *dev_err. */
+#define PA_DEVERR_BLOCK_ID 1    /* a block table entry outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 2 /* context_len < 0, > max_context_len, or past the table */
+#define PA_DEVERR_SLOT 4        /* a slot >= num_blocks * block_size */
+#define PA_DEVERR_TIMEOUT 8     /* a bounded wait on a shared-memory copy ran out */
+#define PA_DEVERR_COPY_PAIR 16  /* a copy pair id outside [0, num_blocks) */
+
+/* pa_write_kv - store the K and V of new tokens in their cache slots.
+ *
+ * Follows the request lifecycle's allocation and append steps ("vLLM基础",
+ * §2.2 steps 4-6) and the in-order slot fill of a logical block
+ * ("啃透vLLM源码", §2.2, append_tokens): token t's K/V go to
+ * (slot / block_size, head, slot % block_size, :) for every head.
+ *
+ * key, value    device [num_tokens][num_heads][head_dim], cache dtype.
+ * slot_mapping  device int64 [num_tokens]; a negative slot is padding and is
+ *               skipped; a slot >= num_blocks*block_size sets
+ *               PA_DEVERR_SLOT and is skipped.
+ * key_cache, value_cache  device, layout above; written in place.
+ * num_tokens == 0 is a no-op. Two tokens mapped to one slot race.
+ */
+pa_status pa_write_kv(const void *key, const void *value, int32_t num_tokens,
+                      int32_t num_heads, const int64_t *slot_mapping, void *key_cache,
+                      void *value_cache, const pa_cache_desc *cache, int32_t *dev_err,
+                      void *stream);
+
+/* Bytes of workspace pa_decode needs. partition_size as for pa_decode; with
+ * 0 (automatic) the bound covers every partition size the automatic choice
+ * can take. Returns 0 when no workspace is needed and (size_t)-1 on
+ * invalid arguments. */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_size);
+
+/* The partition size pa_decode uses for these arguments (tokens per CTA
+ * work unit); >= max_context_len means a single pass without a reduce.
+ * Returns -1 on invalid arguments. */
+int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                 int32_t block_size, int32_t max_context_len,
+                                 int32_t partition_size);
+
+/* pa_decode - one decode step of paged attention: for every sequence s and
+ * head h, out[s,h,:] = softmax(scale * q K^T) V over the context_lens[s]
+ * tokens that the block table of s reaches ("VLLM源码解析", core technology:
+ * attention over key_cache/value_cache through physical block indices;
+ * "vLLM基础", §2.3 block table).
+ *
+ * out           device [num_seqs][num_heads][head_dim] of out_dtype
+ *               (PA_F16, PA_BF16 or PA_F32).
+ * query         device [num_seqs][num_heads][head_dim], cache dtype.
+ * block_tables  device int32 [num_seqs][max_blocks_per_seq]; only the first
+ *               ceil(context_len / block_size) entries of a row are read.
+ * context_lens  device int32 [num_seqs]; 0 gives a zero output row.
+ * max_context_len  host; >= every context_lens[s] (a larger value is
+ *               allowed; a smaller one sets PA_DEVERR_CONTEXT_LEN).
+ * scale         multiplies q.k before the softmax (1/sqrt(head_dim) usually).
+ * partition_size  0 = automatic; else tokens per work unit, a positive
+ *               multiple of 32 up to 8192. A sequence longer than it is split
+ *               into partitions whose partial results (running max, sum and
+ *               unnormalised output, fp32) go to the workspace and are merged
+ *               by a second kernel with the log-sum-exp rule.
+ * workspace     device, >= pa_decode_workspace_size(...) bytes when that is
+ *               non-zero (may be NULL otherwise). Its contents on entry do
+ *               not matter; two calls sharing one workspace on different
+ *               streams race.
+ * Accumulation is fp32 throughout. A block id outside the pool sets
+ * PA_DEVERR_BLOCK_ID and makes that sequence's output NaN.
+ */
+pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t num_seqs,
+                    int32_t num_heads, const void *key_cache, const void *value_cache,
+                    const pa_cache_desc *cache, const int32_t *block_tables,
+                    int32_t max_blocks_per_seq, const int32_t *context_lens,
+                    int32_t max_context_len, float scale, int32_t partition_size,
+                    void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                    void *stream);
+
+/* pa_copy_blocks - copy-on-write duplication of shared blocks ("vLLM基础",
+ * §2.3): for each pair i and each layer l, the whole block
+ * block_mapping[i][0] of key_caches[l] and value_caches[l] (all heads, all
+ * slots) is copied to block block_mapping[i][1].
+ *
+ * key_caches, value_caches  HOST arrays of num_layers device pointers
+ *               (1 <= num_layers <= PA_MAX_LAYERS), every layer shaped by
+ *               `cache`.
+ * block_mapping device int64 [num_pairs][2] = (src, dst). Destinations must
+ *               be distinct and no destination may also be a source (else
+ *               the copies race). Ids outside the pool set
+ *               PA_DEVERR_COPY_PAIR and that pair is skipped.
+ * num_pairs == 0 is a no-op.
+ */
+#define PA_MAX_LAYERS 256
+pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches,
+                         int32_t num_layers, const int64_t *block_mapping,
+                         int32_t num_pairs, const pa_cache_desc *cache, int32_t *dev_err,
+                         void *stream);
+
+/* Static text for a status. */
+const char *pa_status_string(pa_status status);
+
+/* Details of the last failed call on this host thread ("" if none). */
+const char *pa_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

@@ -1,0 +1,196 @@
+"""Python binding of libpagedkv (include/pagedkv.h): paged decode attention
+and its cache-maintenance calls on B200 (sm_100a).
+
+Argument marshalling only: tensors are passed to the C ABI as raw device
+pointers with the current CUDA stream; every step of the computation runs in
+the library's kernels. There is no fallback: importing this module fails if
+the library has not been built (``python -m paged_kv_cache_417_b200.build``).
+
+Cache tensors are [num_blocks, num_heads, block_size, head_dim] fp16/bf16
+(see the header for the full contract).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_417_b200.build` "
+        "(nvcc, sm_100a). There is no non-CUDA fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = range(5)
+PA_F16, PA_BF16, PA_F32 = 0, 1, 2
+PA_DEVERR_BLOCK_ID = 1
+PA_DEVERR_CONTEXT_LEN = 2
+PA_DEVERR_SLOT = 4
+PA_DEVERR_TIMEOUT = 8
+PA_DEVERR_COPY_PAIR = 16
+PA_MAX_LAYERS = 256
+
+_DTYPE = {torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.float32: PA_F32}
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("dtype", ctypes.c_int)]
+
+
+_P = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_lib.pa_write_kv.restype = ctypes.c_int
+_lib.pa_write_kv.argtypes = [_P, _P, _i32, _i32, _P, _P, _P, ctypes.POINTER(CacheDesc), _P, _P]
+_lib.pa_decode_workspace_size.restype = ctypes.c_size_t
+_lib.pa_decode_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
+_lib.pa_decode_partition_size.restype = _i32
+_lib.pa_decode_partition_size.argtypes = [_i32] * 6
+_lib.pa_decode.restype = ctypes.c_int
+_lib.pa_decode.argtypes = [_P, ctypes.c_int, _P, _i32, _i32, _P, _P, ctypes.POINTER(CacheDesc),
+                           _P, _i32, _P, _i32, ctypes.c_float, _i32, _P, ctypes.c_size_t, _P, _P]
+_lib.pa_copy_blocks.restype = ctypes.c_int
+_lib.pa_copy_blocks.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_P), _i32, _P, _i32,
+                                ctypes.POINTER(CacheDesc), _P, _P]
+_lib.pa_status_string.restype = ctypes.c_char_p
+_lib.pa_status_string.argtypes = [ctypes.c_int]
+_lib.pa_last_error.restype = ctypes.c_char_p
+_lib.pa_last_error.argtypes = []
+_lib.pa_version.restype = _i32
+_lib.pa_version.argtypes = []
+
+SIZE_MAX = ctypes.c_size_t(-1).value
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{_lib.pa_status_string(status).decode()}: {detail}")
+
+
+def _check(status: int) -> None:
+    if status != PA_OK:
+        raise PagedKVError(status, _lib.pa_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def cache_desc(key_cache: torch.Tensor) -> CacheDesc:
+    if key_cache.dim() != 4:
+        raise ValueError("cache must be [num_blocks, num_heads, block_size, head_dim]")
+    nb, h, bs, d = key_cache.shape
+    if key_cache.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("cache dtype must be float16 or bfloat16")
+    return CacheDesc(nb, bs, h, d, _DTYPE[key_cache.dtype])
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def version() -> int:
+    return int(_lib.pa_version())
+
+
+def write_kv(key, value, slot_mapping, key_cache, value_cache, dev_err=None):
+    """Store new tokens' K/V ([T, H, D]) at ``slot_mapping`` (int64 [T]) in
+    the caches; negative slots are skipped."""
+    for t, n in ((key, "key"), (value, "value"), (key_cache, "key_cache"),
+                 (value_cache, "value_cache")):
+        _need(t, n, key_cache.dtype)
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    if value_cache.shape != key_cache.shape or key.shape != value.shape:
+        raise ValueError("shape mismatch")
+    desc = cache_desc(key_cache)
+    _check(_lib.pa_write_kv(_ptr(key), _ptr(value), key.shape[0], key.shape[1],
+                            _ptr(slot_mapping), _ptr(key_cache), _ptr(value_cache),
+                            ctypes.byref(desc), _ptr(dev_err), _stream(key_cache)))
+
+
+def decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len, partition_size=0):
+    n = _lib.pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len,
+                                      partition_size)
+    if n == SIZE_MAX:
+        raise ValueError("invalid arguments to decode_workspace_size")
+    return int(n)
+
+
+def decode_partition_size(num_seqs, num_heads, head_dim, block_size, max_context_len,
+                          partition_size=0):
+    n = _lib.pa_decode_partition_size(num_seqs, num_heads, head_dim, block_size,
+                                      max_context_len, partition_size)
+    if n < 0:
+        raise ValueError("invalid arguments to decode_partition_size")
+    return int(n)
+
+
+def alloc_workspace(num_seqs, num_heads, head_dim, max_context_len, partition_size=0,
+                    device="cuda"):
+    n = decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len, partition_size)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def decode(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len,
+           scale, partition_size=0, workspace=None, dev_err=None):
+    """out[s,h,:] = softmax(scale * q K^T) V over each sequence's cached
+    tokens. ``out`` may be fp16, bf16 or fp32; ``workspace`` is allocated
+    here when not given."""
+    _need(query, "query", key_cache.dtype)
+    _need(key_cache, "key_cache")
+    _need(value_cache, "value_cache", key_cache.dtype)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    _need(out, "out")
+    if out.dtype not in _DTYPE:
+        raise ValueError("out dtype must be float16, bfloat16 or float32")
+    if out.shape != query.shape or value_cache.shape != key_cache.shape:
+        raise ValueError("shape mismatch")
+    desc = cache_desc(key_cache)
+    S, H, D = query.shape
+    if workspace is None:
+        workspace = alloc_workspace(S, H, D, int(max_context_len), partition_size,
+                                    query.device)
+    mb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    _check(_lib.pa_decode(_ptr(out), _DTYPE[out.dtype], _ptr(query), S, H, _ptr(key_cache),
+                          _ptr(value_cache), ctypes.byref(desc), _ptr(block_tables), mb,
+                          _ptr(context_lens), int(max_context_len), float(scale),
+                          int(partition_size), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _ptr(dev_err),
+                          _stream(query)))
+    return out
+
+
+def copy_blocks(key_caches, value_caches, block_mapping, dev_err=None):
+    """Copy whole blocks (src, dst) = block_mapping[i] in every layer's K
+    and V cache (copy-on-write)."""
+    if len(key_caches) != len(value_caches) or not key_caches:
+        raise ValueError("need the same, non-zero number of K and V caches")
+    _need(block_mapping, "block_mapping", torch.int64)
+    for c in list(key_caches) + list(value_caches):
+        _need(c, "cache", key_caches[0].dtype)
+        if c.shape != key_caches[0].shape:
+            raise ValueError("all caches must have one shape")
+    desc = cache_desc(key_caches[0])
+    L = len(key_caches)
+    kp = (_P * L)(*[c.data_ptr() for c in key_caches])
+    vp = (_P * L)(*[c.data_ptr() for c in value_caches])
+    n = block_mapping.shape[0] if block_mapping.numel() else 0
+    _check(_lib.pa_copy_blocks(kp, vp, L, _ptr(block_mapping), n, ctypes.byref(desc),
+                               _ptr(dev_err), _stream(key_caches[0])))

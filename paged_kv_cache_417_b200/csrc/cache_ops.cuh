@@ -1,0 +1,95 @@
+// cache_ops.cuh - the two cache-maintenance kernels of a decode step.
+//
+// write_kv_kernel: store each new token's K and V in the slot its block table
+// gives it ("vLLM基础", §2.2 steps 4-6; the in-order slot fill of
+// "啃透vLLM源码", §2.2 append_tokens). One CTA per token; every head's row
+// is head_dim * 2 bytes, moved as 16-byte vectors.
+//
+// copy_blocks_kernel: copy-on-write duplication of whole shared blocks
+// ("vLLM基础", §2.3). One CTA per (pair, layer, K-or-V) copies one
+// num_heads * block_size * head_dim block with 16-byte vectors, four loads in
+// flight per thread before the stores.
+#pragma once
+
+#include <cstdint>
+
+#include "pagedkv.h"
+#include "ptx.cuh"
+
+
+namespace pagedkv {
+
+
+struct WriteParams {
+    const uint4 *key;   // [T][H][D] as 16-byte vectors
+    const uint4 *value;
+    const int64_t *slot_mapping;
+    uint4 *key_cache;   // [NB][H][BS][D]
+    uint4 *value_cache;
+    int32_t *dev_err;
+    int64_t num_slots;  // num_blocks * block_size
+    int32_t num_heads, vecs_per_row, block_size;
+};
+
+__global__ void __launch_bounds__(128) write_kv_kernel(const __grid_constant__ WriteParams p)
+{
+    pdl_launch_dependents();
+    const int t = blockIdx.x;
+    const int64_t slot = p.slot_mapping[t];
+    if (slot < 0)
+        return; // padding
+    if (slot >= p.num_slots) {
+        if (threadIdx.x == 0)
+            report(p.dev_err, PA_DEVERR_SLOT);
+        return;
+    }
+    const int64_t blk = slot / p.block_size, off = slot % p.block_size;
+    const int per_token = p.num_heads * p.vecs_per_row;
+    const uint4 *k = p.key + (size_t)t * per_token;
+    const uint4 *v = p.value + (size_t)t * per_token;
+    for (int i = threadIdx.x; i < per_token; i += blockDim.x) {
+        const int h = i / p.vecs_per_row, e = i - h * p.vecs_per_row;
+        const size_t dst = (((size_t)blk * p.num_heads + h) * p.block_size + off) * p.vecs_per_row + e;
+        p.key_cache[dst] = k[i];
+        p.value_cache[dst] = v[i];
+    }
+}
+
+struct CopyParams {
+    uint4 *key_caches[PA_MAX_LAYERS];
+    uint4 *value_caches[PA_MAX_LAYERS];
+    const int64_t *block_mapping; // [N][2] = (src, dst)
+    int32_t *dev_err;
+    int64_t block_vecs;           // 16-byte vectors per block
+    int64_t num_blocks;
+};
+
+__global__ void __launch_bounds__(256) copy_blocks_kernel(const __grid_constant__ CopyParams p)
+{
+    const int pair = blockIdx.x, layer = blockIdx.y, which = blockIdx.z;
+    const int64_t src = p.block_mapping[2 * pair], dst = p.block_mapping[2 * pair + 1];
+    if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
+        if (threadIdx.x == 0 && layer == 0 && which == 0)
+            report(p.dev_err, PA_DEVERR_COPY_PAIR);
+        return;
+    }
+    uint4 *base = which ? p.value_caches[layer] : p.key_caches[layer];
+    const uint4 *from = base + src * p.block_vecs;
+    uint4 *to = base + dst * p.block_vecs;
+    constexpr int U = 4;
+    const int64_t stride = (int64_t)blockDim.x * U;
+    int64_t i = threadIdx.x;
+    for (; i + (U - 1) * blockDim.x < p.block_vecs; i += stride) {
+        uint4 r[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            r[u] = from[i + u * blockDim.x];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            to[i + u * blockDim.x] = r[u];
+    }
+    for (; i < p.block_vecs; i += blockDim.x)
+        to[i] = from[i];
+}
+
+} // namespace pagedkv

@@ -1,0 +1,426 @@
+// decode.cuh - paged decode attention for sm_100a.
+//
+// out[s,h,:] = softmax(scale * q K^T) V over the context_len tokens that the
+// block table of sequence s reaches. Paging changes where K/V bytes live, not
+// the arithmetic ("VLLM源码解析", core technology: attention over key_cache /
+// value_cache through physical block indices; "vLLM基础", §2.3 block table).
+//
+// Work unit (one CTA): (head h, sequence s, partition p) = tokens
+// [p*P, min((p+1)*P, ctx)) of one (sequence, head). A sequence that fits one
+// partition is finished in place; a longer one leaves (running max, running
+// sum, unnormalised output) per partition in the workspace and
+// reduce_kernel merges them with the log-sum-exp rule.
+//
+// Inside a CTA, each of NW warps owns every NW-th chunk of 4 KiB of K rows
+// (16 tokens at head_dim 128, 32 at 64) plus the matching V rows, and keeps
+// its own NS-stage ring in shared memory: lane 0 issues 1-D bulk copies
+// (cp.async.bulk, the TMA unit's non-tensor path) of the chunk's K and V rows
+// straight out of the scattered physical blocks, each stage completing on its
+// own mbarrier, NS chunks ahead of the math. No CTA-wide barrier is taken
+// until the final merge of the NW warps' partial softmax states.
+//
+// Math per chunk (fp32): each row (token) is covered by D/32 lanes holding
+// 32 of its dims; q.k is 4 x 16-byte shared loads + 32 FMAs per lane and a
+// shuffle reduction over the row's lanes. Online softmax in base 2 (q is
+// pre-scaled by scale*log2(e)): running max m, running sum l, rescale of the
+// accumulator when m grows. Rows past the context are excluded (score -inf,
+// V row skipped), never multiplied by zero, so stale or NaN bytes in the
+// tail of a block cannot leak in.
+//
+// Bank conflicts: a 16-byte shared load is served per quarter-warp (8 lanes,
+// 128 bytes). The 16-byte sub-chunk a lane reads in register slot j is
+// XOR-swizzled with its row so that the quarter-warp's 8 loads hit 8
+// distinct 4-bank groups; the slots are put back in order before the
+// cross-row reduction.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "pagedkv.h"
+#include "ptx.cuh"
+
+namespace pagedkv {
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull; // 1 s: far above any copy latency
+constexpr int kMaxPartition = 8192;              // tokens per work unit, upper bound
+
+struct DecodeParams {
+    void *out;
+    const void *query;
+    const void *key_cache;
+    const void *value_cache;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    float *ws_acc; // [S][H][num_parts][D]
+    float *ws_ml;  // [S][H][num_parts][2] = (max, sum), base-2 domain
+    int32_t *dev_err;
+    int32_t num_seqs, num_heads, num_blocks, max_blocks_per_seq, max_context_len;
+    int32_t partition_size, num_parts;
+    int32_t out_dtype; // 0 f16, 1 bf16, 2 f32
+    float qk_scale_log2;
+};
+
+template <typename T> struct Elem;
+template <> struct Elem<__half> {
+    static __device__ __forceinline__ float2 pair(uint32_t u)
+    {
+        __half2 h;
+        memcpy(&h, &u, 4);
+        return __half22float2(h);
+    }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float2 pair(uint32_t u)
+    {
+        __nv_bfloat162 h;
+        memcpy(&h, &u, 4);
+        return __bfloat1622float2(h);
+    }
+};
+
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4 &raw, float (&f)[8])
+{
+    float2 a = Elem<T>::pair(raw.x), b = Elem<T>::pair(raw.y);
+    float2 c = Elem<T>::pair(raw.z), d = Elem<T>::pair(raw.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+__device__ __forceinline__ void store_out(void *out, int dtype, size_t idx, float v)
+{
+    if (dtype == 2)
+        static_cast<float *>(out)[idx] = v;
+    else if (dtype == 0)
+        static_cast<__half *>(out)[idx] = __float2half_rn(v);
+    else
+        static_cast<__nv_bfloat16 *>(out)[idx] = __float2bfloat16_rn(v);
+}
+
+// Clamp a sequence's context length to what the grid and its table cover.
+__device__ __forceinline__ int checked_context(const DecodeParams &p, int s, int bs,
+                                               bool report_it)
+{
+    int ctx = p.context_lens[s];
+    const int cap = min(p.max_context_len, p.max_blocks_per_seq * bs);
+    if (ctx < 0 || ctx > cap) {
+        if (report_it)
+            report(p.dev_err, PA_DEVERR_CONTEXT_LEN);
+        ctx = ctx < 0 ? 0 : cap;
+    }
+    return ctx;
+}
+
+template <typename T, int D, int BS, int NW, int NS> struct DecodeCfg {
+    static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
+    static constexpr int kLPR = D / 32;                  // lanes per row
+    static constexpr int kRPS = 32 / kLPR;               // rows per warp step
+    static constexpr int kQR = 8 / kLPR;                 // rows per quarter-warp
+    static constexpr int kChunk = 4096 / (D * 2);        // tokens per stage (4 KiB of K)
+    static constexpr int kSteps = kChunk / kRPS;
+    static constexpr int kSeg = BS < kChunk ? BS : kChunk; // rows per bulk copy
+    static constexpr int kTile = kChunk * D;             // elements of K (or V) per stage
+    static constexpr int kStageBytes = NW * NS * 2 * kTile * 2;
+    static constexpr int kBarBytes = NW * NS * 8;
+    static constexpr int kMergeBytes = NW * (D + 2) * 4;
+    static constexpr int kFixedBytes = kStageBytes + kBarBytes + kMergeBytes;
+    static_assert(kSteps >= 1 && kChunk % kRPS == 0, "chunk geometry");
+    static_assert(kStageBytes % 128 == 0, "stage alignment");
+
+    static size_t smem_bytes(int partition)
+    {
+        return kFixedBytes + ((partition / BS) * 4 + 15) / 16 * 16;
+    }
+};
+
+template <typename T, int D, int BS, int NW, int NS>
+__global__ void __launch_bounds__(NW * 32)
+    decode_kernel(const __grid_constant__ DecodeParams p)
+{
+    using C = DecodeCfg<T, D, BS, NW, NS>;
+    constexpr int LPR = C::kLPR, RPS = C::kRPS, QR = C::kQR, CHUNK = C::kChunk;
+    constexpr int STEPS = C::kSteps, TILE = C::kTile;
+    constexpr unsigned FULL = 0xffffffffu;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    T *stages = reinterpret_cast<T *>(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kStageBytes);
+    float *merge = reinterpret_cast<float *>(smem + C::kStageBytes + C::kBarBytes);
+    int32_t *table = reinterpret_cast<int32_t *>(smem + C::kFixedBytes);
+    __shared__ int cta_flags;
+
+    // The reduce kernel (if any) may be scheduled once every CTA has started.
+    pdl_launch_dependents();
+
+    const int h = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.num_heads;
+    const int P = p.partition_size;
+
+    const int ctx = checked_context(p, s, BS, tid == 0 && h == 0 && part == 0);
+    const int num_parts = ctx > 0 ? (ctx + P - 1) / P : 1;
+    if (part >= num_parts)
+        return; // uniform across the CTA, before any barrier
+    const int start = part * P;
+    const int n_tok = min(P, ctx - start); // 0 only when ctx == 0
+    const int n_blk = (n_tok + BS - 1) / BS;
+    const int32_t *bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + start / BS;
+
+    if (tid == 0)
+        cta_flags = 0;
+    if (lane == 0)
+        for (int k = 0; k < NS; ++k)
+            mbar_init(smem_addr(&bars[warp * NS + k]), 1);
+    fence_mbar_init();
+    __syncthreads();
+    for (int i = tid; i < n_blk; i += NW * 32) {
+        int b = bt[i];
+        if (b < 0 || b >= p.num_blocks) {
+            atomicOr(&cta_flags, 1);
+            b = 0;
+        }
+        table[i] = b;
+    }
+    __syncthreads();
+    const bool bad = cta_flags != 0;
+    if (bad && tid == 0)
+        report(p.dev_err, PA_DEVERR_BLOCK_ID);
+
+    const int n_chunks = (n_tok + CHUNK - 1) / CHUNK;
+    const int my_chunks = (bad || n_chunks <= warp) ? 0 : (n_chunks - warp + NW - 1) / NW;
+    T *wstage = stages + (size_t)warp * NS * 2 * TILE;
+    const uint32_t wbar = smem_addr(&bars[warp * NS]);
+    const T *kc = static_cast<const T *>(p.key_cache);
+    const T *vc = static_cast<const T *>(p.value_cache);
+    const size_t head_off = (size_t)h * BS * D;
+    const size_t block_elems = (size_t)H * BS * D;
+
+    // Lane 0: stage local chunk i of this warp (its K rows, then its V rows).
+    auto issue = [&](int i) {
+        const int tok0 = (warp + i * NW) * CHUNK;
+        const int rows = min(CHUNK, n_tok - tok0);
+        const int st = i % NS;
+        T *dk = wstage + st * 2 * TILE;
+        T *dv = dk + TILE;
+        const uint32_t bar = wbar + st * 8;
+        mbar_arrive_expect_tx(bar, 2u * rows * D * sizeof(T));
+        for (int r0 = 0; r0 < rows; r0 += C::kSeg) {
+            const int tok = tok0 + r0;
+            const size_t src =
+                (size_t)table[tok / BS] * block_elems + head_off + (size_t)(tok % BS) * D;
+            const uint32_t bytes = (uint32_t)(min(C::kSeg, rows - r0) * D * sizeof(T));
+            bulk_g2s(smem_addr(dk + r0 * D), kc + src, bytes, bar);
+            bulk_g2s(smem_addr(dv + r0 * D), vc + src, bytes, bar);
+        }
+    };
+
+    const int qd = lane % LPR;     // which interleaved quarter of a row
+    const int r = lane / LPR;      // row within a step
+    const int rx = r & (QR - 1);   // swizzle key
+    float qf[4][8];
+    {
+        const T *qp = static_cast<const T *>(p.query) + ((size_t)s * H + h) * D;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int u = qd + LPR * (j ^ rx);
+            unpack8<T>(*reinterpret_cast<const uint4 *>(qp + u * 8), qf[j]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                qf[j][e] *= p.qk_scale_log2;
+        }
+    }
+    float acc[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            acc[j][e] = 0.f;
+    float m = -INFINITY, l = 0.f;
+
+    if (lane == 0)
+        for (int i = 0; i < min(NS, my_chunks); ++i)
+            issue(i);
+    int issued = min(NS, my_chunks);
+    bool timed_out = false;
+    int i = 0;
+    for (; i < my_chunks; ++i) {
+        const int st = i % NS;
+        const bool ok = mbar_wait_bounded(wbar + st * 8, (i / NS) & 1, kWaitLimitNs);
+        if (__any_sync(FULL, !ok)) {
+            timed_out = true;
+            break;
+        }
+        const int rows = min(CHUNK, n_tok - (warp + i * NW) * CHUNK);
+        const T *sk = wstage + st * 2 * TILE;
+        const T *sv = sk + TILE;
+
+        float sc[STEPS];
+#pragma unroll
+        for (int t = 0; t < STEPS; ++t) {
+            const int row = t * RPS + r;
+            const T *kr = sk + row * D;
+            float dot = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float kf[8];
+                unpack8<T>(*reinterpret_cast<const uint4 *>(kr + (qd + LPR * (j ^ rx)) * 8), kf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    dot = fmaf(qf[j][e], kf[e], dot);
+            }
+#pragma unroll
+            for (int o = 1; o < LPR; o <<= 1)
+                dot += __shfl_xor_sync(FULL, dot, o);
+            sc[t] = row < rows ? dot : -INFINITY;
+        }
+        float cm = sc[0];
+#pragma unroll
+        for (int t = 1; t < STEPS; ++t)
+            cm = fmaxf(cm, sc[t]);
+#pragma unroll
+        for (int o = LPR; o < 32; o <<= 1)
+            cm = fmaxf(cm, __shfl_xor_sync(FULL, cm, o));
+        const float m_new = fmaxf(m, cm); // finite: row 0 of a chunk is always valid
+        const float corr = exp2f(m - m_new);
+        m = m_new;
+        l *= corr;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                acc[j][e] *= corr;
+#pragma unroll
+        for (int t = 0; t < STEPS; ++t) {
+            const int row = t * RPS + r;
+            const float pt = exp2f(sc[t] - m_new);
+            l += pt;
+            if (row < rows) {
+                const T *vr = sv + row * D;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float vf[8];
+                    unpack8<T>(*reinterpret_cast<const uint4 *>(vr + (qd + LPR * (j ^ rx)) * 8),
+                               vf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        acc[j][e] = fmaf(pt, vf[e], acc[j][e]);
+                }
+            }
+        }
+        __syncwarp();
+        if (i + NS < my_chunks) {
+            if (lane == 0)
+                issue(i + NS);
+            issued = i + NS + 1;
+        }
+    }
+    if (timed_out) {
+        if (lane == 0)
+            report(p.dev_err, PA_DEVERR_TIMEOUT);
+        // Let the copies still in flight land before shared memory is reused.
+        for (int k = i; k < issued; ++k)
+            mbar_wait_bounded(wbar + (k % NS) * 8, (k / NS) & 1, kWaitLimitNs);
+        if (lane == 0)
+            atomicOr(&cta_flags, 2);
+    }
+
+    // Put the swizzled slots back in order: slot j <- sub-chunk qd + LPR*j.
+    if (rx & 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float t0 = acc[0][e]; acc[0][e] = acc[1][e]; acc[1][e] = t0;
+            float t2 = acc[2][e]; acc[2][e] = acc[3][e]; acc[3][e] = t2;
+        }
+    }
+    if (rx & 2) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float t0 = acc[0][e]; acc[0][e] = acc[2][e]; acc[2][e] = t0;
+            float t1 = acc[1][e]; acc[1][e] = acc[3][e]; acc[3][e] = t1;
+        }
+    }
+    // Sum over the rows this warp's lanes covered (lanes with equal qd).
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) {
+        l += __shfl_xor_sync(FULL, l, o);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                acc[j][e] += __shfl_xor_sync(FULL, acc[j][e], o);
+    }
+    float *mw = merge + warp * (D + 2);
+    if (lane < LPR) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                mw[(qd + LPR * j) * 8 + e] = acc[j][e];
+    }
+    if (lane == 0) {
+        mw[D] = m;
+        mw[D + 1] = l;
+    }
+    __syncthreads();
+
+    const bool failed = cta_flags != 0;
+    for (int d = tid; d < D; d += NW * 32) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+            M = fmaxf(M, merge[w * (D + 2) + D]);
+        float L = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float f = exp2f(merge[w * (D + 2) + D] - M);
+                L = fmaf(merge[w * (D + 2) + D + 1], f, L);
+                O = fmaf(merge[w * (D + 2) + d], f, O);
+            }
+        }
+        if (failed)
+            O = NAN;
+        if (num_parts == 1) {
+            store_out(p.out, p.out_dtype, ((size_t)s * H + h) * D + d, L > 0.f ? O / L : O);
+        } else {
+            const size_t unit = ((size_t)s * H + h) * p.num_parts + part;
+            p.ws_acc[unit * D + d] = O;
+            if (d == 0) {
+                p.ws_ml[unit * 2] = failed ? 0.f : M;
+                p.ws_ml[unit * 2 + 1] = failed ? 1.f : L;
+            }
+        }
+    }
+}
+
+// Merge the partitions of every split sequence:
+// M = max_p m_p, L = sum_p l_p 2^(m_p - M), out = sum_p o_p 2^(m_p - M) / L.
+template <int D>
+__global__ void __launch_bounds__(D) reduce_kernel(const __grid_constant__ DecodeParams p,
+                                                   int block_size)
+{
+    pdl_wait_prior_grid();
+    const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+    const int ctx = checked_context(p, s, block_size, false);
+    const int P = p.partition_size;
+    const int num_parts = ctx > 0 ? (ctx + P - 1) / P : 1;
+    if (num_parts <= 1)
+        return;
+    const size_t unit0 = ((size_t)s * p.num_heads + h) * p.num_parts;
+    float M = -INFINITY;
+    for (int i = 0; i < num_parts; ++i)
+        M = fmaxf(M, p.ws_ml[(unit0 + i) * 2]);
+    float L = 0.f, O = 0.f;
+    for (int i = 0; i < num_parts; ++i) {
+        const float f = exp2f(p.ws_ml[(unit0 + i) * 2] - M);
+        L = fmaf(p.ws_ml[(unit0 + i) * 2 + 1], f, L);
+        O = fmaf(p.ws_acc[(unit0 + i) * D + d], f, O);
+    }
+    store_out(p.out, p.out_dtype, ((size_t)s * p.num_heads + h) * D + d, O / L);
+}
+
+} // namespace pagedkv

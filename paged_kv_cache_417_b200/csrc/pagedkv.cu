@@ -1,0 +1,385 @@
+// pagedkv.cu - the C ABI (include/pagedkv.h): host-side argument checks,
+// launch-shape choices and kernel launches. Nothing here allocates memory or
+// synchronises.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "pagedkv.h"
+
+#include "cache_ops.cuh"
+#include "decode.cuh"
+
+using namespace pagedkv;
+
+namespace {
+
+constexpr int kNumWarps = 4;   // warps per decode CTA
+constexpr int kNumStages = 3;  // bulk-copy stages per warp
+constexpr int kMinAutoPartition = 128;
+constexpr int kAutoPartition = 512;
+constexpr int kPartitionQuantum = 32;
+constexpr int kMaxDevices = 64;
+
+thread_local char g_last_error[512] = "";
+
+pa_status fail(pa_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+pa_status ok()
+{
+    g_last_error[0] = '\0';
+    return PA_OK;
+}
+
+pa_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count_of_current_device()
+{
+    static std::atomic<int> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 148;
+    }
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0)
+        return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+pa_status check_cache(const pa_cache_desc *c)
+{
+    if (!c)
+        return fail(PA_ERR_INVALID_ARG, "cache descriptor is NULL");
+    if (c->num_blocks < 0 || c->block_size <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0)
+        return fail(PA_ERR_INVALID_ARG, "cache descriptor has a non-positive size");
+    if (c->dtype != PA_F16 && c->dtype != PA_BF16)
+        return fail(PA_ERR_UNSUPPORTED, "cache dtype %d (need PA_F16 or PA_BF16)", (int)c->dtype);
+    if (c->head_dim != 64 && c->head_dim != 128)
+        return fail(PA_ERR_UNSUPPORTED, "head_dim %d (built: 64, 128)", c->head_dim);
+    if (c->block_size != 8 && c->block_size != 16 && c->block_size != 32)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d (built: 8, 16, 32)", c->block_size);
+    return PA_OK;
+}
+
+// Partition (tokens per work unit) for a decode; >= max_context_len means a
+// single pass. Automatic choice: 512 tokens, halved (down to 128) while the
+// grid would give fewer than two work units per SM.
+int choose_partition(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, int32_t requested,
+                     int sm_count)
+{
+    int P = requested;
+    if (P == 0) {
+        P = kAutoPartition;
+        const int64_t units = (int64_t)num_seqs * num_heads;
+        while (P > kMinAutoPartition && units * ((max_ctx + P - 1) / P) < 2LL * sm_count)
+            P /= 2;
+    }
+    if (max_ctx <= P) {
+        const int single = ((max_ctx > 0 ? max_ctx : 1) + kPartitionQuantum - 1) /
+                           kPartitionQuantum * kPartitionQuantum;
+        return single;
+    }
+    return P;
+}
+
+pa_status check_partition_request(int32_t partition_size)
+{
+    if (partition_size < 0 || partition_size % kPartitionQuantum != 0 ||
+        partition_size > kMaxPartition)
+        return fail(PA_ERR_INVALID_ARG,
+                    "partition_size %d: need 0 or a multiple of %d up to %d", partition_size,
+                    kPartitionQuantum, kMaxPartition);
+    return PA_OK;
+}
+
+size_t workspace_bytes_for(int64_t units, int64_t num_parts, int head_dim)
+{
+    const size_t acc = (size_t)(units * num_parts * head_dim) * sizeof(float);
+    const size_t acc_padded = (acc + 255) / 256 * 256;
+    return acc_padded + (size_t)(units * num_parts * 2) * sizeof(float);
+}
+
+template <typename Kernel> cudaError_t allow_smem(Kernel k, size_t bytes)
+{
+    // Per device: the attribute belongs to the function in the current context.
+    static std::atomic<size_t> done[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_relaxed) >= bytes)
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return e;
+    if (dev >= 0 && dev < kMaxDevices)
+        done[dev].store(bytes, std::memory_order_relaxed);
+    return cudaSuccess;
+}
+
+template <typename T, int D, int BS>
+pa_status launch_decode(const DecodeParams &p, cudaStream_t stream)
+{
+    using C = DecodeCfg<T, D, BS, kNumWarps, kNumStages>;
+    auto kernel = decode_kernel<T, D, BS, kNumWarps, kNumStages>;
+    const size_t smem = C::smem_bytes(p.partition_size);
+    cudaError_t e = allow_smem(kernel, C::smem_bytes(kMaxPartition));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    dim3 grid(p.num_heads, p.num_seqs, p.num_parts);
+    kernel<<<grid, kNumWarps * 32, smem, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "decode launch");
+    if (p.num_parts > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.num_heads, p.num_seqs, 1);
+        cfg.blockDim = dim3(D, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, reduce_kernel<D>, p, (int)BS);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "reduce launch");
+    }
+    return ok();
+}
+
+template <typename T, int D> pa_status dispatch_bs(const DecodeParams &p, int bs, cudaStream_t st)
+{
+    switch (bs) {
+    case 8: return launch_decode<T, D, 8>(p, st);
+    case 16: return launch_decode<T, D, 16>(p, st);
+    case 32: return launch_decode<T, D, 32>(p, st);
+    }
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d", bs);
+}
+
+template <typename T> pa_status dispatch_d(const DecodeParams &p, int d, int bs, cudaStream_t st)
+{
+    if (d == 64)
+        return dispatch_bs<T, 64>(p, bs, st);
+    return dispatch_bs<T, 128>(p, bs, st);
+}
+
+} // namespace
+
+extern "C" {
+
+const char *pa_status_string(pa_status s)
+{
+    switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PA_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char *pa_last_error(void) { return g_last_error; }
+
+int32_t pa_version(void) { return 100; }
+
+pa_status pa_write_kv(const void *key, const void *value, int32_t num_tokens, int32_t num_heads,
+                      const int64_t *slot_mapping, void *key_cache, void *value_cache,
+                      const pa_cache_desc *cache, int32_t *dev_err, void *stream)
+{
+    pa_status s = check_cache(cache);
+    if (s != PA_OK)
+        return s;
+    if (num_tokens < 0)
+        return fail(PA_ERR_INVALID_ARG, "num_tokens %d < 0", num_tokens);
+    if (num_heads != cache->num_kv_heads)
+        return fail(PA_ERR_UNSUPPORTED, "num_heads %d != num_kv_heads %d", num_heads,
+                    cache->num_kv_heads);
+    if (num_tokens == 0)
+        return ok();
+    if (!key || !value || !slot_mapping || !key_cache || !value_cache)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+        return fail(PA_ERR_INVALID_ARG, "key, value and caches must be 16-byte aligned");
+    WriteParams p;
+    p.key = static_cast<const uint4 *>(key);
+    p.value = static_cast<const uint4 *>(value);
+    p.slot_mapping = slot_mapping;
+    p.key_cache = static_cast<uint4 *>(key_cache);
+    p.value_cache = static_cast<uint4 *>(value_cache);
+    p.dev_err = dev_err;
+    p.num_slots = (int64_t)cache->num_blocks * cache->block_size;
+    p.num_heads = num_heads;
+    p.vecs_per_row = cache->head_dim * 2 / 16;
+    p.block_size = cache->block_size;
+    write_kv_kernel<<<num_tokens, 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "write_kv launch");
+    return ok();
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_size)
+{
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+        check_partition_request(partition_size) != PA_OK)
+        return (size_t)-1;
+    const int P = partition_size == 0 ? kMinAutoPartition : partition_size;
+    if (max_context_len <= P)
+        return 0;
+    const int64_t parts = (max_context_len + P - 1) / P;
+    return workspace_bytes_for((int64_t)num_seqs * num_heads, parts, head_dim);
+}
+
+int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                 int32_t block_size, int32_t max_context_len,
+                                 int32_t partition_size)
+{
+    (void)head_dim;
+    (void)block_size;
+    if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0 ||
+        check_partition_request(partition_size) != PA_OK)
+        return -1;
+    return choose_partition(num_seqs, num_heads, max_context_len, partition_size,
+                            partition_size == 0 ? sm_count_of_current_device() : 148);
+}
+
+pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t num_seqs,
+                    int32_t num_heads, const void *key_cache, const void *value_cache,
+                    const pa_cache_desc *cache, const int32_t *block_tables,
+                    int32_t max_blocks_per_seq, const int32_t *context_lens,
+                    int32_t max_context_len, float scale, int32_t partition_size,
+                    void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream)
+{
+    pa_status s = check_cache(cache);
+    if (s != PA_OK)
+        return s;
+    if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq < 0 || max_context_len < 0)
+        return fail(PA_ERR_INVALID_ARG, "negative size argument");
+    if (num_heads != cache->num_kv_heads)
+        return fail(PA_ERR_UNSUPPORTED, "num_heads %d != num_kv_heads %d (grouped heads not built)",
+                    num_heads, cache->num_kv_heads);
+    if (out_dtype != PA_F16 && out_dtype != PA_BF16 && out_dtype != PA_F32)
+        return fail(PA_ERR_INVALID_ARG, "out_dtype %d", (int)out_dtype);
+    if ((s = check_partition_request(partition_size)) != PA_OK)
+        return s;
+    if (num_seqs == 0)
+        return ok();
+    if (num_seqs > 65535)
+        return fail(PA_ERR_UNSUPPORTED, "num_seqs %d > 65535", num_seqs);
+    if (!out || !query || !key_cache || !value_cache || !context_lens ||
+        (max_blocks_per_seq > 0 && !block_tables))
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+        return fail(PA_ERR_INVALID_ARG, "query and caches must be 16-byte aligned");
+    if (!(scale == scale))
+        return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+
+    const int P = choose_partition(num_seqs, num_heads, max_context_len, partition_size,
+                                   sm_count_of_current_device());
+    const int64_t parts = max_context_len > P ? (max_context_len + P - 1) / P : 1;
+    if (parts > 65535)
+        return fail(PA_ERR_UNSUPPORTED, "too many partitions (%lld)", (long long)parts);
+    DecodeParams p = {};
+    p.out = out;
+    p.query = query;
+    p.key_cache = key_cache;
+    p.value_cache = value_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.dev_err = dev_err;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_blocks = cache->num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.partition_size = P;
+    p.num_parts = (int32_t)parts;
+    p.out_dtype = (int32_t)out_dtype;
+    p.qk_scale_log2 = scale * 1.4426950408889634f;
+    if (parts > 1) {
+        const int64_t units = (int64_t)num_seqs * num_heads;
+        const size_t need = workspace_bytes_for(units, parts, cache->head_dim);
+        if (!workspace || workspace_bytes < need)
+            return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes, need %zu", workspace_bytes,
+                        need);
+        if (!aligned16(workspace))
+            return fail(PA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+        const size_t acc = (size_t)(units * parts * cache->head_dim) * sizeof(float);
+        p.ws_acc = static_cast<float *>(workspace);
+        p.ws_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) + (acc + 255) / 256 * 256);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cache->dtype == PA_F16)
+        return dispatch_d<__half>(p, cache->head_dim, cache->block_size, st);
+    return dispatch_d<__nv_bfloat16>(p, cache->head_dim, cache->block_size, st);
+}
+
+pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches, int32_t num_layers,
+                         const int64_t *block_mapping, int32_t num_pairs,
+                         const pa_cache_desc *cache, int32_t *dev_err, void *stream)
+{
+    pa_status s = check_cache(cache);
+    if (s != PA_OK)
+        return s;
+    if (num_pairs < 0)
+        return fail(PA_ERR_INVALID_ARG, "num_pairs %d < 0", num_pairs);
+    if (num_layers < 1 || num_layers > PA_MAX_LAYERS)
+        return fail(PA_ERR_INVALID_ARG, "num_layers %d outside [1, %d]", num_layers, PA_MAX_LAYERS);
+    if (num_pairs == 0)
+        return ok();
+    if (!block_mapping || !key_caches || !value_caches)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
+    CopyParams p;
+    for (int l = 0; l < num_layers; ++l) {
+        if (!key_caches[l] || !value_caches[l])
+            return fail(PA_ERR_INVALID_ARG, "NULL cache pointer for layer %d", l);
+        if (!aligned16(key_caches[l]) || !aligned16(value_caches[l]))
+            return fail(PA_ERR_INVALID_ARG, "cache of layer %d not 16-byte aligned", l);
+        p.key_caches[l] = static_cast<uint4 *>(key_caches[l]);
+        p.value_caches[l] = static_cast<uint4 *>(value_caches[l]);
+    }
+    for (int l = num_layers; l < PA_MAX_LAYERS; ++l)
+        p.key_caches[l] = p.value_caches[l] = nullptr;
+    p.block_mapping = block_mapping;
+    p.dev_err = dev_err;
+    p.block_vecs = (int64_t)cache->num_kv_heads * cache->block_size * cache->head_dim * 2 / 16;
+    p.num_blocks = cache->num_blocks;
+    dim3 grid(num_pairs, num_layers, 2);
+    copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "copy_blocks launch");
+    return ok();
+}
+
+} // extern "C"

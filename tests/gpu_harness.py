@@ -1,0 +1,68 @@
+"""Run decode steps through the CUDA library for the parity tests."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import paged_kv_cache_417_b200 as pk
+from workloads.device import device_step
+
+TOL = 2e-3  # max |gpu - oracle| for fp16 output, fp32 accumulation
+
+
+def to_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def run_step(step, layers=None, partition_size=0, out_dtype=None, keep_pre=False):
+    """copy_blocks (all layers) -> per layer write_kv, decode. Returns
+    (outs list, device dict, dev_err int)."""
+    layers = list(range(step.num_layers)) if layers is None else list(layers)
+    d = device_step(step, "cuda", layers)
+    if keep_pre:
+        d["pre_key"] = [k.clone() for k in d["key_caches"]]
+        d["pre_value"] = [v.clone() for v in d["value_caches"]]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if step.copy_pairs.shape[0]:
+        pk.copy_blocks(d["key_caches"], d["value_caches"], d["copy_pairs"], dev_err=err)
+    outs = []
+    for i, _ in enumerate(layers):
+        kc, vc = d["key_caches"][i], d["value_caches"][i]
+        pk.write_kv(d["new_key"][i], d["new_value"][i], d["slot_mapping"], kc, vc, dev_err=err)
+        q = d["query"][i]
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device="cuda")
+        pk.decode(out, q, kc, vc, d["block_tables"], d["context_lens"], step.max_context_len,
+                  float(step.scale), partition_size=partition_size, dev_err=err)
+        outs.append(out)
+    torch.cuda.synchronize()
+    return outs, d, int(err.item())
+
+
+def max_err(gpu_out: torch.Tensor, ref: np.ndarray) -> float:
+    got = to_f64(gpu_out)
+    assert got.shape == ref.shape
+    assert np.all(np.isfinite(got)), "non-finite output"
+    return float(np.max(np.abs(got - ref))) if ref.size else 0.0
+
+
+def decode_case(c, partition_size=0, out_dtype=None, max_context_len=None):
+    """Decode a tests.paged_cases case on the GPU."""
+    dt = torch.float16 if c["dtype"] == "f16" else torch.bfloat16
+
+    def up(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).cuda()
+
+    q, kc, vc = up(c["q"]), up(c["kpool"]), up(c["vpool"])
+    bt = torch.from_numpy(c["bt"]).cuda()
+    ctx = torch.from_numpy(c["ctx"]).cuda()
+    out = torch.empty(q.shape, dtype=out_dtype or dt, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mcl = int(c["ctx"].max()) if max_context_len is None else max_context_len
+    pk.decode(out, q, kc, vc, bt, ctx, mcl, float(c["scale"]), partition_size=partition_size,
+              dev_err=err)
+    torch.cuda.synchronize()
+    return out, int(err.item())

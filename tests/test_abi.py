@@ -1,0 +1,129 @@
+"""The C-ABI library without a GPU: it loads, exports every function the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_417_b200 import build
+    build.build()
+    import paged_kv_cache_417_b200 as pk
+    return pk
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \t\*]*?\b(pa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["pa_write_kv", "pa_decode", "pa_copy_blocks", "pa_decode_workspace_size",
+              "pa_status_string", "pa_last_error", "pa_version"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(so, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib._lib.pa_status_string(s)
+    assert lib.version() >= 100
+
+
+def _desc(lib, nb=16, bs=16, h=2, d=64, dt=0):
+    return lib.CacheDesc(nb, bs, h, d, dt)
+
+
+def test_decode_rejects_bad_arguments_on_host(lib):
+    L = lib._lib
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: checks fail first
+    cases = [
+        (_desc(lib, d=96), lib.PA_ERR_UNSUPPORTED),        # head_dim
+        (_desc(lib, bs=64), lib.PA_ERR_UNSUPPORTED),       # block_size
+        (_desc(lib, dt=2), lib.PA_ERR_UNSUPPORTED),        # fp32 cache
+        (_desc(lib, h=3), lib.PA_ERR_UNSUPPORTED),         # num_heads != kv heads
+    ]
+    for desc, want in cases:
+        st = L.pa_decode(fake, 0, fake, 1, 2, fake, fake, ctypes.byref(desc), fake, 1, fake,
+                         16, 0.125, 0, None, 0, None, None)
+        assert st == want, (desc.head_dim, desc.block_size, st)
+        assert L.pa_last_error()
+    desc = _desc(lib)
+    # unaligned query
+    st = L.pa_decode(fake, 0, ctypes.c_void_p(0x1002), 1, 2, fake, fake, ctypes.byref(desc),
+                     fake, 1, fake, 16, 0.125, 0, None, 0, None, None)
+    assert st == lib.PA_ERR_INVALID_ARG
+    # bad partition size
+    st = L.pa_decode(fake, 0, fake, 1, 2, fake, fake, ctypes.byref(desc), fake, 1, fake, 16,
+                     0.125, 48, None, 0, None, None)
+    assert st == lib.PA_ERR_INVALID_ARG
+    # null pointers
+    st = L.pa_decode(None, 0, fake, 1, 2, fake, fake, ctypes.byref(desc), fake, 1, fake, 16,
+                     0.125, 0, None, 0, None, None)
+    assert st == lib.PA_ERR_INVALID_ARG
+    # zero sequences: nothing to do, no launch
+    st = L.pa_decode(None, 0, None, 0, 2, None, None, ctypes.byref(desc), None, 0, None, 0,
+                     0.125, 0, None, 0, None, None)
+    assert st == lib.PA_OK
+    # split needed but no workspace (32 partitions of 32 tokens)
+    st = L.pa_decode(fake, 0, fake, 1, 2, fake, fake, ctypes.byref(desc), fake, 64, fake,
+                     1024, 0.125, 32, None, 0, None, None)
+    assert st == lib.PA_ERR_WORKSPACE
+
+
+def test_write_and_copy_reject_bad_arguments(lib):
+    L = lib._lib
+    fake = ctypes.c_void_p(0x1000)
+    desc = _desc(lib)
+    assert L.pa_write_kv(fake, fake, -1, 2, fake, fake, fake, ctypes.byref(desc), None,
+                         None) == lib.PA_ERR_INVALID_ARG
+    assert L.pa_write_kv(fake, fake, 0, 2, fake, fake, fake, ctypes.byref(desc), None,
+                         None) == lib.PA_OK
+    assert L.pa_write_kv(None, fake, 3, 2, fake, fake, fake, ctypes.byref(desc), None,
+                         None) == lib.PA_ERR_INVALID_ARG
+    assert L.pa_write_kv(fake, fake, 3, 2, fake, fake, fake, None, None,
+                         None) == lib.PA_ERR_INVALID_ARG
+    arr = (ctypes.c_void_p * 1)(0x1000)
+    assert L.pa_copy_blocks(arr, arr, 0, fake, 1, ctypes.byref(desc), None,
+                            None) == lib.PA_ERR_INVALID_ARG
+    assert L.pa_copy_blocks(arr, arr, 1, fake, 0, ctypes.byref(desc), None, None) == lib.PA_OK
+    bad = (ctypes.c_void_p * 1)(0x1004)
+    assert L.pa_copy_blocks(bad, bad, 1, fake, 1, ctypes.byref(desc), None,
+                            None) == lib.PA_ERR_INVALID_ARG
+
+
+def test_workspace_and_partition_sizes(lib):
+    # single pass: no workspace
+    assert lib.decode_workspace_size(4, 4, 64, 100, 0) == 0
+    assert lib.decode_workspace_size(4, 4, 64, 512, 512) == 0
+    # explicit partitions: acc [S,H,P,D] fp32 padded to 256 B, then (m, l) pairs
+    S, H, D, ctx, P = 3, 5, 128, 1000, 256
+    parts = -(-ctx // P)
+    acc = S * H * parts * D * 4
+    want = -(-acc // 256) * 256 + S * H * parts * 2 * 4
+    assert lib.decode_workspace_size(S, H, D, ctx, P) == want
+    # automatic: a bound that covers the smallest automatic partition (128)
+    assert lib.decode_workspace_size(S, H, D, ctx, 0) >= lib.decode_workspace_size(S, H, D, ctx,
+                                                                                   128)
+    with pytest.raises(ValueError):
+        lib.decode_workspace_size(S, H, D, ctx, 40)
+    assert lib.decode_partition_size(S, H, D, 16, 100, 0) == 128  # single pass, rounded to 32
+    assert lib.decode_partition_size(96, 32, 128, 16, 2048, 0) == 512
+    assert lib.decode_partition_size(96, 32, 128, 16, 2048, 1024) == 1024
+    assert lib.decode_partition_size(1, 1, 128, 16, 30000, 0) == 128
