@@ -120,10 +120,12 @@ size_t workspace_bytes_for(int64_t units, int64_t num_parts, int head_dim)
     return acc_padded + (size_t)(units * num_parts * 2) * sizeof(float);
 }
 
-template <typename Kernel> cudaError_t allow_smem(Kernel k, size_t bytes)
+// Raise a kernel's dynamic shared-memory limit once per device. `done` must
+// be distinct for every kernel (one static per template instantiation of the
+// caller), since the attribute belongs to the function.
+template <typename Kernel>
+cudaError_t allow_smem(Kernel k, size_t bytes, std::atomic<size_t> (&done)[kMaxDevices])
 {
-    // Per device: the attribute belongs to the function in the current context.
-    static std::atomic<size_t> done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
@@ -148,7 +150,8 @@ pa_status launch_decode(const DecodeParams &p, cudaStream_t stream)
     using C = DecodeCfg<T, D, BS, kNumWarps, kNumStages>;
     auto kernel = decode_kernel<T, D, BS, kNumWarps, kNumStages>;
     const size_t smem = C::smem_bytes(p.partition_size);
-    cudaError_t e = allow_smem(kernel, C::smem_bytes(kMaxPartition));
+    static std::atomic<size_t> smem_set[kMaxDevices];
+    cudaError_t e = allow_smem(kernel, C::smem_bytes(kMaxPartition), smem_set);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute(decode)");
     dim3 grid(p.num_heads, p.num_seqs, p.num_parts);
