@@ -139,6 +139,42 @@ pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t nu
                     void *workspace, size_t workspace_bytes, int32_t *dev_err,
                     void *stream);
 
+/* pa_decode_noalloc - pa_decode without a caller-provided workspace, for
+ * callers that cannot allocate device memory when they decode.
+ *
+ * The pages have no counterpart to this call; it exists for library users.
+ * Some programs cannot call cudaMalloc on the path that runs decode: a
+ * serving engine that reserved almost all device memory for its KV block
+ * pool at start-up (a later allocation fails, or could only succeed by
+ * giving up cache blocks), or a runtime that forbids allocation after
+ * initialisation because cudaMalloc/cudaFree can synchronise the device and
+ * stall every stream. This call takes the same arguments as pa_decode except
+ * the workspace, and allocates nothing: split partitions are merged through
+ * a fixed PA_NOALLOC_SCRATCH_BYTES array of device memory compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.
+ *
+ * - Limit: if the partial results need more than PA_NOALLOC_SCRATCH_BYTES
+ *   (see pa_decode_workspace_size with the partition size actually used,
+ *   pa_decode_partition_size), the call returns PA_ERR_WORKSPACE and
+ *   launches nothing; a larger partition_size needs less scratch.
+ * - Set-up: the first call on each device looks up that device's address of
+ *   the array (with the device current); make that first call before any
+ *   stream capture.
+ * - Sharing: every call in the process on a device uses the same array and
+ *   leaves its contents behind. Nothing in it has to start at zero (each call
+ *   writes every value it reads), but calls whose kernels overlap on the GPU
+ *   (different streams or host threads) race on it: serialise them.
+ * Everything else (arguments, errors, dev_err) is as for pa_decode.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (32u << 20)
+pa_status pa_decode_noalloc(void *out, pa_dtype out_dtype, const void *query, int32_t num_seqs,
+                            int32_t num_heads, const void *key_cache, const void *value_cache,
+                            const pa_cache_desc *cache, const int32_t *block_tables,
+                            int32_t max_blocks_per_seq, const int32_t *context_lens,
+                            int32_t max_context_len, float scale, int32_t partition_size,
+                            int32_t *dev_err, void *stream);
+
 /* pa_copy_blocks - copy-on-write duplication of shared blocks ("vLLM基础",
  * §2.3): for each pair i and each layer l, the whole block
  * block_mapping[i][0] of key_caches[l] and value_caches[l] (all heads, all

@@ -55,6 +55,10 @@ _lib.pa_decode_partition_size.argtypes = [_i32] * 6
 _lib.pa_decode.restype = ctypes.c_int
 _lib.pa_decode.argtypes = [_P, ctypes.c_int, _P, _i32, _i32, _P, _P, ctypes.POINTER(CacheDesc),
                            _P, _i32, _P, _i32, ctypes.c_float, _i32, _P, ctypes.c_size_t, _P, _P]
+_lib.pa_decode_noalloc.restype = ctypes.c_int
+_lib.pa_decode_noalloc.argtypes = [_P, ctypes.c_int, _P, _i32, _i32, _P, _P,
+                                   ctypes.POINTER(CacheDesc), _P, _i32, _P, _i32,
+                                   ctypes.c_float, _i32, _P, _P]
 _lib.pa_copy_blocks.restype = ctypes.c_int
 _lib.pa_copy_blocks.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_P), _i32, _P, _i32,
                                 ctypes.POINTER(CacheDesc), _P, _P]
@@ -174,6 +178,38 @@ def decode(out, query, key_cache, value_cache, block_tables, context_lens, max_c
                           int(partition_size), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _ptr(dev_err),
                           _stream(query)))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def decode_noalloc(out, query, key_cache, value_cache, block_tables, context_lens,
+                   max_context_len, scale, partition_size=0, dev_err=None):
+    """Like :func:`decode`, for callers that must not allocate device memory
+    while decoding (for example an engine that has handed almost all device
+    memory to its KV block pool): partial results of split contexts go to a
+    fixed 32 MiB array inside the library instead of a workspace. Calls that
+    overlap on the GPU share that array and race; the first call on a device
+    looks up its address and should come before any stream capture."""
+    _need(query, "query", key_cache.dtype)
+    _need(key_cache, "key_cache")
+    _need(value_cache, "value_cache", key_cache.dtype)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    _need(out, "out")
+    if out.dtype not in _DTYPE:
+        raise ValueError("out dtype must be float16, bfloat16 or float32")
+    if out.shape != query.shape or value_cache.shape != key_cache.shape:
+        raise ValueError("shape mismatch")
+    desc = cache_desc(key_cache)
+    S, H, D = query.shape
+    mb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    _check(_lib.pa_decode_noalloc(_ptr(out), _DTYPE[out.dtype], _ptr(query), S, H,
+                                  _ptr(key_cache), _ptr(value_cache), ctypes.byref(desc),
+                                  _ptr(block_tables), mb, _ptr(context_lens),
+                                  int(max_context_len), float(scale), int(partition_size),
+                                  _ptr(dev_err), _stream(query)))
     return out
 
 

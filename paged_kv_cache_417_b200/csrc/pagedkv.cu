@@ -386,3 +386,73 @@ pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches, int
 }
 
 } // extern "C"
+
+// ---------------------------------------------------------------------------
+// pa_decode_noalloc: pa_decode with the workspace taken from a fixed array of
+// device memory compiled into the library, for callers that cannot allocate.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+// In host code g_noalloc_scratch names a host-side stand-in, not device
+// memory: its device address must be looked up, once per device, with that
+// device current.
+pa_status noalloc_scratch(void **out)
+{
+    static std::atomic<void *> addr[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(PA_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+    void *p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        addr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return PA_OK;
+}
+
+} // namespace
+
+extern "C" pa_status pa_decode_noalloc(void *out, pa_dtype out_dtype, const void *query,
+                                       int32_t num_seqs, int32_t num_heads,
+                                       const void *key_cache, const void *value_cache,
+                                       const pa_cache_desc *cache, const int32_t *block_tables,
+                                       int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                       int32_t max_context_len, float scale,
+                                       int32_t partition_size, int32_t *dev_err, void *stream)
+{
+    pa_status s = check_cache(cache);
+    if (s != PA_OK)
+        return s;
+    if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0)
+        return fail(PA_ERR_INVALID_ARG, "negative size argument");
+    if ((s = check_partition_request(partition_size)) != PA_OK)
+        return s;
+    if (num_seqs == 0)
+        return ok();
+    const int P = choose_partition(num_seqs, num_heads, max_context_len, partition_size,
+                                   sm_count_of_current_device());
+    const int64_t parts = max_context_len > P ? (max_context_len + P - 1) / P : 1;
+    if (parts > 1) {
+        const size_t need =
+            workspace_bytes_for((int64_t)num_seqs * num_heads, parts, cache->head_dim);
+        if (need > PA_NOALLOC_SCRATCH_BYTES)
+            return fail(PA_ERR_WORKSPACE,
+                        "split decode needs %zu bytes of scratch (partition %d); the built-in "
+                        "scratch holds %u: use a larger partition_size or pa_decode",
+                        need, P, (unsigned)PA_NOALLOC_SCRATCH_BYTES);
+    }
+    void *scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != PA_OK)
+        return s;
+    return pa_decode(out, out_dtype, query, num_seqs, num_heads, key_cache, value_cache, cache,
+                     block_tables, max_blocks_per_seq, context_lens, max_context_len, scale,
+                     partition_size, scratch, PA_NOALLOC_SCRATCH_BYTES, dev_err, stream);
+}
