@@ -283,6 +283,9 @@ def main():
     ap.add_argument("--config", default="llama7b_layer", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=0)
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="llama7b_layer only: this many sequences (pool scaled to match), "
+                         "for profiler captures on a smaller case of the same kernel")
     ap.add_argument("--soak-seconds", type=float, default=1.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -317,7 +320,14 @@ def main():
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
 
-    step = WORKLOADS[args.config][0](SEEDS[args.config] + 1000 * rank)
+    if args.seqs:
+        if args.config != "llama7b_layer":
+            ap.error("--seqs applies to llama7b_layer only")
+        step = wl.llama_layer(seed=SEEDS[args.config] + 1000 * rank, num_seqs=args.seqs,
+                              num_blocks=max(256, 8192 * args.seqs // 96))
+        config_desc["workload"] += f" (reduced to {args.seqs} seqs)"
+    else:
+        step = WORKLOADS[args.config][0](SEEDS[args.config] + 1000 * rank)
     d = device_step(step, dev)
     L, S = step.num_layers, step.num_seqs
     stream = torch.cuda.current_stream(dev)

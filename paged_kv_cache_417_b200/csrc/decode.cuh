@@ -5,19 +5,23 @@
 // the arithmetic ("VLLM源码解析", core technology: attention over key_cache /
 // value_cache through physical block indices; "vLLM基础", §2.3 block table).
 //
-// Work unit (one CTA): (head h, sequence s, partition p) = tokens
+// A work unit is (sequence s, head h, partition p) = tokens
 // [p*P, min((p+1)*P, ctx)) of one (sequence, head). A sequence that fits one
 // partition is finished in place; a longer one leaves (running max, running
 // sum, unnormalised output) per partition in the workspace and
 // reduce_kernel merges them with the log-sum-exp rule.
 //
-// Inside a CTA, each of NW warps owns every NW-th chunk of 4 KiB of K rows
-// (16 tokens at head_dim 128, 32 at 64) plus the matching V rows, and keeps
-// its own NS-stage ring in shared memory: lane 0 issues 1-D bulk copies
-// (cp.async.bulk, the TMA unit's non-tensor path) of the chunk's K and V rows
-// straight out of the scattered physical blocks, each stage completing on its
-// own mbarrier, NS chunks ahead of the math. No CTA-wide barrier is taken
-// until the final merge of the NW warps' partial softmax states.
+// The K/V of a unit stream through shared memory in chunks of 4 KiB of K
+// rows (16 tokens at head_dim 128, 32 at 64) plus the matching V rows. Each
+// warp keeps its own NS-stage ring: lane 0 issues 1-D bulk copies
+// (cp.async.bulk, the TMA unit's non-tensor path) of a chunk's K and V rows
+// straight out of the scattered physical blocks, each stage completing on
+// its own mbarrier, NS chunks ahead of the math.
+//
+// decode_split_kernel: a CTA takes one unit and its NW warps share it, every
+// NW-th chunk each, merging their softmax states in shared memory at the
+// end. (A mapping with one warp per head and NW heads of a sequence per CTA
+// was measured slower on every workload here and is not built.)
 //
 // Math per chunk (fp32): each row (token) is covered by D/32 lanes holding
 // 32 of its dims; q.k is 4 x 16-byte shared loads + 32 FMAs per lane and a
@@ -101,36 +105,249 @@ __device__ __forceinline__ void store_out(void *out, int dtype, size_t idx, floa
 }
 
 // Clamp a sequence's context length to what the grid and its table cover.
-__device__ __forceinline__ int checked_context(const DecodeParams &p, int s, int bs,
+__device__ __forceinline__ int checked_context(const DecodeParams &p, int raw, int bs,
                                                bool report_it)
 {
-    int ctx = p.context_lens[s];
     const int cap = min(p.max_context_len, p.max_blocks_per_seq * bs);
-    if (ctx < 0 || ctx > cap) {
+    if (raw < 0 || raw > cap) {
         if (report_it)
             report(p.dev_err, PA_DEVERR_CONTEXT_LEN);
-        ctx = ctx < 0 ? 0 : cap;
+        return raw < 0 ? 0 : cap;
     }
-    return ctx;
+    return raw;
 }
 
-template <typename T, int D, int BS, int NW, int NS> struct DecodeCfg {
+template <typename T, int D, int BS, int NS> struct ChunkCfg {
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
-    static constexpr int kLPR = D / 32;                  // lanes per row
-    static constexpr int kRPS = 32 / kLPR;               // rows per warp step
-    static constexpr int kQR = 8 / kLPR;                 // rows per quarter-warp
-    static constexpr int kChunk = 4096 / (D * 2);        // tokens per stage (4 KiB of K)
+    static constexpr int kLPR = D / 32;                    // lanes per row
+    static constexpr int kRPS = 32 / kLPR;                 // rows per warp step
+    static constexpr int kQR = 8 / kLPR;                   // rows per quarter-warp
+    static constexpr int kChunk = 4096 / (D * 2);          // tokens per stage (4 KiB of K)
     static constexpr int kSteps = kChunk / kRPS;
     static constexpr int kSeg = BS < kChunk ? BS : kChunk; // rows per bulk copy
-    static constexpr int kTile = kChunk * D;             // elements of K (or V) per stage
-    static constexpr int kStageBytes = NW * NS * 2 * kTile * 2;
+    static constexpr int kTile = kChunk * D;               // elements of K (or V) per stage
+    static constexpr int kRingBytes = NS * 2 * kTile * 2;  // one warp's stages
+    static_assert(kSteps >= 1 && kChunk % kRPS == 0, "chunk geometry");
+};
+
+// One warp's online-softmax state over the chunks it streamed. After
+// finish(), the lanes with r == 0 (lane < D/32) hold the warp's sums for
+// dims (qd + LPR*j)*8 + e, j < 4, e < 8; every lane holds m and l.
+template <typename T, int D, int BS, int NS> struct WarpStream {
+    using C = ChunkCfg<T, D, BS, NS>;
+    static constexpr int LPR = C::kLPR, RPS = C::kRPS, QR = C::kQR, CHUNK = C::kChunk;
+    static constexpr int STEPS = C::kSteps, TILE = C::kTile;
+    static constexpr unsigned FULL = 0xffffffffu;
+
+    float qf[4][8];
+    float acc[4][8];
+    float m, l;
+    int qd, r, rx, lane;
+    int bad_id; // lane 0: a block id outside the pool was met
+
+    __device__ __forceinline__ void init(const T *q, float qk_scale_log2, int lane_)
+    {
+        lane = lane_;
+        qd = lane % LPR;
+        r = lane / LPR;
+        rx = r & (QR - 1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int u = qd + LPR * (j ^ rx);
+            unpack8<T>(*reinterpret_cast<const uint4 *>(q + u * 8), qf[j]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                qf[j][e] *= qk_scale_log2;
+                acc[j][e] = 0.f;
+            }
+        }
+        m = -INFINITY;
+        l = 0.f;
+        bad_id = 0;
+    }
+
+    // Stream chunks c0, c0 + cstride, ... (count of them) of a unit with
+    // n_tok tokens whose block ids are table[0..]. Lane 0 issues the copies;
+    // an id outside [0, num_blocks) is replaced by block 0 and sets bad_id.
+    // Returns false if a wait ran out of time (the copies in flight have been
+    // waited for, boundedly, before returning).
+    __device__ __forceinline__ bool run(const T *kc, const T *vc, size_t head_off,
+                                        size_t block_elems, int num_blocks,
+                                        const int32_t *table, int n_tok, int c0, int cstride,
+                                        int count, T *ring, uint32_t bar0)
+    {
+        auto issue = [&](int i) {
+            const int tok0 = (c0 + i * cstride) * CHUNK;
+            const int rows = min(CHUNK, n_tok - tok0);
+            const int st = i % NS;
+            T *dk = ring + st * 2 * TILE;
+            T *dv = dk + TILE;
+            const uint32_t bar = bar0 + st * 8;
+            mbar_arrive_expect_tx(bar, 2u * rows * D * sizeof(T));
+            for (int r0 = 0; r0 < rows; r0 += C::kSeg) {
+                const int tok = tok0 + r0;
+                int b = table[tok / BS];
+                if (b < 0 || b >= num_blocks) {
+                    bad_id = 1;
+                    b = 0;
+                }
+                const size_t src = (size_t)b * block_elems + head_off + (size_t)(tok % BS) * D;
+                const uint32_t bytes = (uint32_t)(min(C::kSeg, rows - r0) * D * sizeof(T));
+                bulk_g2s(smem_addr(dk + r0 * D), kc + src, bytes, bar);
+                bulk_g2s(smem_addr(dv + r0 * D), vc + src, bytes, bar);
+            }
+        };
+
+        if (lane == 0)
+            for (int i = 0; i < min(NS, count); ++i)
+                issue(i);
+        int issued = min(NS, count);
+        int i = 0;
+        for (; i < count; ++i) {
+            const int st = i % NS;
+            const bool ok = mbar_wait_bounded(bar0 + st * 8, (i / NS) & 1, kWaitLimitNs);
+            if (__any_sync(FULL, !ok))
+                break;
+            const int rows = min(CHUNK, n_tok - (c0 + i * cstride) * CHUNK);
+            const T *sk = ring + st * 2 * TILE;
+            const T *sv = sk + TILE;
+
+            float sc[STEPS];
+#pragma unroll
+            for (int t = 0; t < STEPS; ++t) {
+                const int row = t * RPS + r;
+                const T *kr = sk + row * D;
+                float dot = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float kf[8];
+                    unpack8<T>(*reinterpret_cast<const uint4 *>(kr + (qd + LPR * (j ^ rx)) * 8),
+                               kf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dot = fmaf(qf[j][e], kf[e], dot);
+                }
+#pragma unroll
+                for (int o = 1; o < LPR; o <<= 1)
+                    dot += __shfl_xor_sync(FULL, dot, o);
+                sc[t] = row < rows ? dot : -INFINITY;
+            }
+            float cm = sc[0];
+#pragma unroll
+            for (int t = 1; t < STEPS; ++t)
+                cm = fmaxf(cm, sc[t]);
+#pragma unroll
+            for (int o = LPR; o < 32; o <<= 1)
+                cm = fmaxf(cm, __shfl_xor_sync(FULL, cm, o));
+            const float m_new = fmaxf(m, cm); // finite: row 0 of a chunk is always valid
+            const float corr = exp2f(m - m_new);
+            m = m_new;
+            l *= corr;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc[j][e] *= corr;
+#pragma unroll
+            for (int t = 0; t < STEPS; ++t) {
+                const int row = t * RPS + r;
+                const float pt = exp2f(sc[t] - m_new);
+                l += pt;
+                if (row < rows) {
+                    const T *vr = sv + row * D;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float vf[8];
+                        unpack8<T>(
+                            *reinterpret_cast<const uint4 *>(vr + (qd + LPR * (j ^ rx)) * 8), vf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            acc[j][e] = fmaf(pt, vf[e], acc[j][e]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (i + NS < count) {
+                if (lane == 0)
+                    issue(i + NS);
+                issued = i + NS + 1;
+            }
+        }
+        if (i < count) {
+            // Timed out: let the copies still in flight land before the
+            // shared memory is reused or the CTA exits.
+            for (int k = i; k < issued; ++k)
+                mbar_wait_bounded(bar0 + (k % NS) * 8, (k / NS) & 1, kWaitLimitNs);
+            return false;
+        }
+        return true;
+    }
+
+    // Put the swizzled slots back in order (slot j <- sub-chunk qd + LPR*j)
+    // and sum acc and l over the rows the warp's lanes covered.
+    __device__ __forceinline__ void finish()
+    {
+        if (rx & 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float t0 = acc[0][e]; acc[0][e] = acc[1][e]; acc[1][e] = t0;
+                float t2 = acc[2][e]; acc[2][e] = acc[3][e]; acc[3][e] = t2;
+            }
+        }
+        if (rx & 2) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float t0 = acc[0][e]; acc[0][e] = acc[2][e]; acc[2][e] = t0;
+                float t1 = acc[1][e]; acc[1][e] = acc[3][e]; acc[3][e] = t1;
+            }
+        }
+#pragma unroll
+        for (int o = LPR; o < 32; o <<= 1) {
+            l += __shfl_xor_sync(FULL, l, o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc[j][e] += __shfl_xor_sync(FULL, acc[j][e], o);
+        }
+    }
+};
+
+// Shared prologue: read the context length and the partition's slice of the
+// block table at the same time (one global latency). Returns false when the
+// partition is past the sequence (the whole CTA returns).
+struct UnitInfo {
+    int ctx, num_parts, start, n_tok;
+};
+
+template <int BS>
+__device__ __forceinline__ bool load_unit(const DecodeParams &p, int s, int part, int tid,
+                                          int nthreads, bool report_ctx, int32_t *table,
+                                          UnitInfo &u)
+{
+    const int P = p.partition_size;
+    const int raw = p.context_lens[s];
+    const int start_blk = part * (P / BS);
+    const int n_load = min(P / BS, p.max_blocks_per_seq - start_blk);
+    const int32_t *bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + start_blk;
+    for (int i = tid; i < n_load; i += nthreads)
+        table[i] = bt[i];
+    u.ctx = checked_context(p, raw, BS, report_ctx);
+    u.num_parts = u.ctx > 0 ? (u.ctx + P - 1) / P : 1;
+    u.start = part * P;
+    u.n_tok = min(P, u.ctx - u.start); // 0 only when ctx == 0
+    return part < u.num_parts;
+}
+
+// NW warps share one unit: CTA = (head blockIdx.x, sequence blockIdx.y,
+// partition blockIdx.z).
+template <typename T, int D, int BS, int NW, int NS> struct SplitCfg {
+    using C = ChunkCfg<T, D, BS, NS>;
+    static constexpr int kRingsBytes = NW * C::kRingBytes;
     static constexpr int kBarBytes = NW * NS * 8;
     static constexpr int kMergeBytes = NW * (D + 2) * 4;
-    static constexpr int kFixedBytes = kStageBytes + kBarBytes + kMergeBytes;
-    static_assert(kSteps >= 1 && kChunk % kRPS == 0, "chunk geometry");
-    static_assert(kStageBytes % 128 == 0, "stage alignment");
-
+    static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kMergeBytes;
     static size_t smem_bytes(int partition)
     {
         return kFixedBytes + ((partition / BS) * 4 + 15) / 16 * 16;
@@ -139,36 +356,22 @@ template <typename T, int D, int BS, int NW, int NS> struct DecodeCfg {
 
 template <typename T, int D, int BS, int NW, int NS>
 __global__ void __launch_bounds__(NW * 32)
-    decode_kernel(const __grid_constant__ DecodeParams p)
+    decode_split_kernel(const __grid_constant__ DecodeParams p)
 {
-    using C = DecodeCfg<T, D, BS, NW, NS>;
-    constexpr int LPR = C::kLPR, RPS = C::kRPS, QR = C::kQR, CHUNK = C::kChunk;
-    constexpr int STEPS = C::kSteps, TILE = C::kTile;
-    constexpr unsigned FULL = 0xffffffffu;
-
+    using W = WarpStream<T, D, BS, NS>;
+    using Cfg = SplitCfg<T, D, BS, NW, NS>;
+    constexpr int LPR = W::LPR;
     extern __shared__ __align__(128) unsigned char smem[];
-    T *stages = reinterpret_cast<T *>(smem);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kStageBytes);
-    float *merge = reinterpret_cast<float *>(smem + C::kStageBytes + C::kBarBytes);
-    int32_t *table = reinterpret_cast<int32_t *>(smem + C::kFixedBytes);
+    T *rings = reinterpret_cast<T *>(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kRingsBytes);
+    float *merge = reinterpret_cast<float *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes);
+    int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
     __shared__ int cta_flags;
 
-    // The reduce kernel (if any) may be scheduled once every CTA has started.
     pdl_launch_dependents();
-
     const int h = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads;
-    const int P = p.partition_size;
-
-    const int ctx = checked_context(p, s, BS, tid == 0 && h == 0 && part == 0);
-    const int num_parts = ctx > 0 ? (ctx + P - 1) / P : 1;
-    if (part >= num_parts)
-        return; // uniform across the CTA, before any barrier
-    const int start = part * P;
-    const int n_tok = min(P, ctx - start); // 0 only when ctx == 0
-    const int n_blk = (n_tok + BS - 1) / BS;
-    const int32_t *bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + start / BS;
 
     if (tid == 0)
         cta_flags = 0;
@@ -176,198 +379,48 @@ __global__ void __launch_bounds__(NW * 32)
         for (int k = 0; k < NS; ++k)
             mbar_init(smem_addr(&bars[warp * NS + k]), 1);
     fence_mbar_init();
+    UnitInfo u;
+    const bool live = load_unit<BS>(p, s, part, tid, NW * 32, tid == 0 && h == 0 && part == 0,
+                                    table, u);
+    if (!live)
+        return; // uniform across the CTA
     __syncthreads();
-    for (int i = tid; i < n_blk; i += NW * 32) {
-        int b = bt[i];
-        if (b < 0 || b >= p.num_blocks) {
-            atomicOr(&cta_flags, 1);
-            b = 0;
-        }
-        table[i] = b;
-    }
-    __syncthreads();
-    const bool bad = cta_flags != 0;
-    if (bad && tid == 0)
-        report(p.dev_err, PA_DEVERR_BLOCK_ID);
 
-    const int n_chunks = (n_tok + CHUNK - 1) / CHUNK;
-    const int my_chunks = (bad || n_chunks <= warp) ? 0 : (n_chunks - warp + NW - 1) / NW;
-    T *wstage = stages + (size_t)warp * NS * 2 * TILE;
-    const uint32_t wbar = smem_addr(&bars[warp * NS]);
-    const T *kc = static_cast<const T *>(p.key_cache);
-    const T *vc = static_cast<const T *>(p.value_cache);
-    const size_t head_off = (size_t)h * BS * D;
-    const size_t block_elems = (size_t)H * BS * D;
-
-    // Lane 0: stage local chunk i of this warp (its K rows, then its V rows).
-    auto issue = [&](int i) {
-        const int tok0 = (warp + i * NW) * CHUNK;
-        const int rows = min(CHUNK, n_tok - tok0);
-        const int st = i % NS;
-        T *dk = wstage + st * 2 * TILE;
-        T *dv = dk + TILE;
-        const uint32_t bar = wbar + st * 8;
-        mbar_arrive_expect_tx(bar, 2u * rows * D * sizeof(T));
-        for (int r0 = 0; r0 < rows; r0 += C::kSeg) {
-            const int tok = tok0 + r0;
-            const size_t src =
-                (size_t)table[tok / BS] * block_elems + head_off + (size_t)(tok % BS) * D;
-            const uint32_t bytes = (uint32_t)(min(C::kSeg, rows - r0) * D * sizeof(T));
-            bulk_g2s(smem_addr(dk + r0 * D), kc + src, bytes, bar);
-            bulk_g2s(smem_addr(dv + r0 * D), vc + src, bytes, bar);
-        }
-    };
-
-    const int qd = lane % LPR;     // which interleaved quarter of a row
-    const int r = lane / LPR;      // row within a step
-    const int rx = r & (QR - 1);   // swizzle key
-    float qf[4][8];
-    {
-        const T *qp = static_cast<const T *>(p.query) + ((size_t)s * H + h) * D;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int u = qd + LPR * (j ^ rx);
-            unpack8<T>(*reinterpret_cast<const uint4 *>(qp + u * 8), qf[j]);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                qf[j][e] *= p.qk_scale_log2;
-        }
-    }
-    float acc[4][8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            acc[j][e] = 0.f;
-    float m = -INFINITY, l = 0.f;
-
-    if (lane == 0)
-        for (int i = 0; i < min(NS, my_chunks); ++i)
-            issue(i);
-    int issued = min(NS, my_chunks);
-    bool timed_out = false;
-    int i = 0;
-    for (; i < my_chunks; ++i) {
-        const int st = i % NS;
-        const bool ok = mbar_wait_bounded(wbar + st * 8, (i / NS) & 1, kWaitLimitNs);
-        if (__any_sync(FULL, !ok)) {
-            timed_out = true;
-            break;
-        }
-        const int rows = min(CHUNK, n_tok - (warp + i * NW) * CHUNK);
-        const T *sk = wstage + st * 2 * TILE;
-        const T *sv = sk + TILE;
-
-        float sc[STEPS];
-#pragma unroll
-        for (int t = 0; t < STEPS; ++t) {
-            const int row = t * RPS + r;
-            const T *kr = sk + row * D;
-            float dot = 0.f;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float kf[8];
-                unpack8<T>(*reinterpret_cast<const uint4 *>(kr + (qd + LPR * (j ^ rx)) * 8), kf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    dot = fmaf(qf[j][e], kf[e], dot);
-            }
-#pragma unroll
-            for (int o = 1; o < LPR; o <<= 1)
-                dot += __shfl_xor_sync(FULL, dot, o);
-            sc[t] = row < rows ? dot : -INFINITY;
-        }
-        float cm = sc[0];
-#pragma unroll
-        for (int t = 1; t < STEPS; ++t)
-            cm = fmaxf(cm, sc[t]);
-#pragma unroll
-        for (int o = LPR; o < 32; o <<= 1)
-            cm = fmaxf(cm, __shfl_xor_sync(FULL, cm, o));
-        const float m_new = fmaxf(m, cm); // finite: row 0 of a chunk is always valid
-        const float corr = exp2f(m - m_new);
-        m = m_new;
-        l *= corr;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                acc[j][e] *= corr;
-#pragma unroll
-        for (int t = 0; t < STEPS; ++t) {
-            const int row = t * RPS + r;
-            const float pt = exp2f(sc[t] - m_new);
-            l += pt;
-            if (row < rows) {
-                const T *vr = sv + row * D;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float vf[8];
-                    unpack8<T>(*reinterpret_cast<const uint4 *>(vr + (qd + LPR * (j ^ rx)) * 8),
-                               vf);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        acc[j][e] = fmaf(pt, vf[e], acc[j][e]);
-                }
-            }
-        }
-        __syncwarp();
-        if (i + NS < my_chunks) {
-            if (lane == 0)
-                issue(i + NS);
-            issued = i + NS + 1;
-        }
-    }
-    if (timed_out) {
-        if (lane == 0)
+    W ws;
+    ws.init(static_cast<const T *>(p.query) + ((size_t)s * H + h) * D, p.qk_scale_log2, lane);
+    const int n_chunks = (u.n_tok + W::CHUNK - 1) / W::CHUNK;
+    const int my_chunks = n_chunks <= warp ? 0 : (n_chunks - warp + NW - 1) / NW;
+    const bool ok = ws.run(static_cast<const T *>(p.key_cache),
+                           static_cast<const T *>(p.value_cache), (size_t)h * BS * D,
+                           (size_t)H * BS * D, p.num_blocks, table, u.n_tok, warp, NW,
+                           my_chunks, rings + (size_t)warp * NS * 2 * W::TILE,
+                           smem_addr(&bars[warp * NS]));
+    if (lane == 0) {
+        if (!ok) {
             report(p.dev_err, PA_DEVERR_TIMEOUT);
-        // Let the copies still in flight land before shared memory is reused.
-        for (int k = i; k < issued; ++k)
-            mbar_wait_bounded(wbar + (k % NS) * 8, (k / NS) & 1, kWaitLimitNs);
-        if (lane == 0)
             atomicOr(&cta_flags, 2);
-    }
-
-    // Put the swizzled slots back in order: slot j <- sub-chunk qd + LPR*j.
-    if (rx & 1) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            float t0 = acc[0][e]; acc[0][e] = acc[1][e]; acc[1][e] = t0;
-            float t2 = acc[2][e]; acc[2][e] = acc[3][e]; acc[3][e] = t2;
         }
+        if (ws.bad_id)
+            atomicOr(&cta_flags, 1);
     }
-    if (rx & 2) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            float t0 = acc[0][e]; acc[0][e] = acc[2][e]; acc[2][e] = t0;
-            float t1 = acc[1][e]; acc[1][e] = acc[3][e]; acc[3][e] = t1;
-        }
-    }
-    // Sum over the rows this warp's lanes covered (lanes with equal qd).
-#pragma unroll
-    for (int o = LPR; o < 32; o <<= 1) {
-        l += __shfl_xor_sync(FULL, l, o);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                acc[j][e] += __shfl_xor_sync(FULL, acc[j][e], o);
-    }
+    ws.finish();
     float *mw = merge + warp * (D + 2);
     if (lane < LPR) {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                mw[(qd + LPR * j) * 8 + e] = acc[j][e];
+                mw[(ws.qd + LPR * j) * 8 + e] = ws.acc[j][e];
     }
     if (lane == 0) {
-        mw[D] = m;
-        mw[D + 1] = l;
+        mw[D] = ws.m;
+        mw[D + 1] = ws.l;
     }
     __syncthreads();
 
     const bool failed = cta_flags != 0;
+    if (tid == 0 && (cta_flags & 1))
+        report(p.dev_err, PA_DEVERR_BLOCK_ID);
     for (int d = tid; d < D; d += NW * 32) {
         float M = -INFINITY;
 #pragma unroll
@@ -384,7 +437,7 @@ __global__ void __launch_bounds__(NW * 32)
         }
         if (failed)
             O = NAN;
-        if (num_parts == 1) {
+        if (u.num_parts == 1) {
             store_out(p.out, p.out_dtype, ((size_t)s * H + h) * D + d, L > 0.f ? O / L : O);
         } else {
             const size_t unit = ((size_t)s * H + h) * p.num_parts + part;
@@ -405,7 +458,7 @@ __global__ void __launch_bounds__(D) reduce_kernel(const __grid_constant__ Decod
 {
     pdl_wait_prior_grid();
     const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
-    const int ctx = checked_context(p, s, block_size, false);
+    const int ctx = checked_context(p, p.context_lens[s], block_size, false);
     const int P = p.partition_size;
     const int num_parts = ctx > 0 ? (ctx + P - 1) / P : 1;
     if (num_parts <= 1)

@@ -17,10 +17,20 @@ using namespace pagedkv;
 
 namespace {
 
-constexpr int kNumWarps = 4;   // warps per decode CTA
-constexpr int kNumStages = 3;  // bulk-copy stages per warp
+// Decode launch shape: 4 warps x 2 bulk-copy stages of 8 KiB per warp =
+// 64 KiB of rings per CTA, 3 CTAs per SM. The macros only exist so that
+// tuning sweeps can build variants.
+#ifndef PA_SPLIT_WARPS
+#define PA_SPLIT_WARPS 4
+#endif
+#ifndef PA_SPLIT_STAGES
+#define PA_SPLIT_STAGES 2
+#endif
+constexpr int kSplitWarps = PA_SPLIT_WARPS;
+constexpr int kSplitStages = PA_SPLIT_STAGES;
+constexpr int kTargetCtasPerSm = 12; // ~4 waves of 3 resident CTAs
 constexpr int kMinAutoPartition = 128;
-constexpr int kAutoPartition = 512;
+constexpr int kAutoPartition = 2048;
 constexpr int kPartitionQuantum = 32;
 constexpr int kMaxDevices = 64;
 
@@ -83,8 +93,8 @@ pa_status check_cache(const pa_cache_desc *c)
 }
 
 // Partition (tokens per work unit) for a decode; >= max_context_len means a
-// single pass. Automatic choice: 512 tokens, halved (down to 128) while the
-// grid would give fewer than two work units per SM.
+// single pass. Automatic choice: 2048 tokens, halved (down to 128) while the
+// grid would give fewer than about four waves of resident CTAs.
 int choose_partition(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, int32_t requested,
                      int sm_count)
 {
@@ -92,7 +102,8 @@ int choose_partition(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, int32
     if (P == 0) {
         P = kAutoPartition;
         const int64_t units = (int64_t)num_seqs * num_heads;
-        while (P > kMinAutoPartition && units * ((max_ctx + P - 1) / P) < 2LL * sm_count)
+        while (P > kMinAutoPartition &&
+               units * ((max_ctx + P - 1) / P) < (int64_t)kTargetCtasPerSm * sm_count)
             P /= 2;
     }
     if (max_ctx <= P) {
@@ -147,15 +158,14 @@ cudaError_t allow_smem(Kernel k, size_t bytes, std::atomic<size_t> (&done)[kMaxD
 template <typename T, int D, int BS>
 pa_status launch_decode(const DecodeParams &p, cudaStream_t stream)
 {
-    using C = DecodeCfg<T, D, BS, kNumWarps, kNumStages>;
-    auto kernel = decode_kernel<T, D, BS, kNumWarps, kNumStages>;
-    const size_t smem = C::smem_bytes(p.partition_size);
+    using Cfg = SplitCfg<T, D, BS, kSplitWarps, kSplitStages>;
+    auto kernel = decode_split_kernel<T, D, BS, kSplitWarps, kSplitStages>;
     static std::atomic<size_t> smem_set[kMaxDevices];
-    cudaError_t e = allow_smem(kernel, C::smem_bytes(kMaxPartition), smem_set);
+    cudaError_t e = allow_smem(kernel, Cfg::smem_bytes(kMaxPartition), smem_set);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute(decode)");
     dim3 grid(p.num_heads, p.num_seqs, p.num_parts);
-    kernel<<<grid, kNumWarps * 32, smem, stream>>>(p);
+    kernel<<<grid, kSplitWarps * 32, Cfg::smem_bytes(p.partition_size), stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return cuda_fail(e, "decode launch");

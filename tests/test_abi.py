@@ -124,6 +124,8 @@ def test_workspace_and_partition_sizes(lib):
     with pytest.raises(ValueError):
         lib.decode_workspace_size(S, H, D, ctx, 40)
     assert lib.decode_partition_size(S, H, D, 16, 100, 0) == 128  # single pass, rounded to 32
-    assert lib.decode_partition_size(96, 32, 128, 16, 2048, 0) == 512
+    assert lib.decode_partition_size(96, 32, 128, 16, 2048, 0) == 2048  # single pass
+    assert lib.decode_partition_size(8, 32, 128, 16, 32768, 0) == 2048
+    assert lib.decode_partition_size(1, 32, 128, 16, 32768, 0) == 512
     assert lib.decode_partition_size(96, 32, 128, 16, 2048, 1024) == 1024
     assert lib.decode_partition_size(1, 1, 128, 16, 30000, 0) == 128
