@@ -34,6 +34,7 @@ struct WriteParams {
 __global__ void __launch_bounds__(128) write_kv_kernel(const __grid_constant__ WriteParams p)
 {
     pdl_launch_dependents();
+    pdl_wait_prior_grid(); // inputs may come from the previous kernel
     const int t = blockIdx.x;
     const int64_t slot = p.slot_mapping[t];
     if (slot < 0)
@@ -47,11 +48,30 @@ __global__ void __launch_bounds__(128) write_kv_kernel(const __grid_constant__ W
     const int per_token = p.num_heads * p.vecs_per_row;
     const uint4 *k = p.key + (size_t)t * per_token;
     const uint4 *v = p.value + (size_t)t * per_token;
-    for (int i = threadIdx.x; i < per_token; i += blockDim.x) {
-        const int h = i / p.vecs_per_row, e = i - h * p.vecs_per_row;
-        const size_t dst = (((size_t)blk * p.num_heads + h) * p.block_size + off) * p.vecs_per_row + e;
-        p.key_cache[dst] = k[i];
-        p.value_cache[dst] = v[i];
+    // All loads of a round before its stores: the stores may alias nothing
+    // the loads read, but the compiler cannot know that.
+    constexpr int U = 4;
+    for (int base = threadIdx.x; base < per_token; base += blockDim.x * U) {
+        uint4 kr[U], vr[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * blockDim.x;
+            if (i < per_token) {
+                kr[u] = k[i];
+                vr[u] = v[i];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * blockDim.x;
+            if (i < per_token) {
+                const int h = i / p.vecs_per_row, e = i - h * p.vecs_per_row;
+                const size_t dst =
+                    (((size_t)blk * p.num_heads + h) * p.block_size + off) * p.vecs_per_row + e;
+                p.key_cache[dst] = kr[u];
+                p.value_cache[dst] = vr[u];
+            }
+        }
     }
 }
 
@@ -66,6 +86,8 @@ struct CopyParams {
 
 __global__ void __launch_bounds__(256) copy_blocks_kernel(const __grid_constant__ CopyParams p)
 {
+    pdl_launch_dependents();
+    pdl_wait_prior_grid();
     const int pair = blockIdx.x, layer = blockIdx.y, which = blockIdx.z;
     const int64_t src = p.block_mapping[2 * pair], dst = p.block_mapping[2 * pair + 1];
     if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {

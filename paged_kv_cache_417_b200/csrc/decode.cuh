@@ -368,6 +368,8 @@ __global__ void __launch_bounds__(NW * 32)
     int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
     __shared__ int cta_flags;
 
+    // Dependent kernels (the reduce, the next layer's write) may launch now;
+    // each of them waits for this grid before it touches data.
     pdl_launch_dependents();
     const int h = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -379,6 +381,7 @@ __global__ void __launch_bounds__(NW * 32)
         for (int k = 0; k < NS; ++k)
             mbar_init(smem_addr(&bars[warp * NS + k]), 1);
     fence_mbar_init();
+    pdl_wait_prior_grid(); // every input may come from the previous kernel
     UnitInfo u;
     const bool live = load_unit<BS>(p, s, part, tid, NW * 32, tid == 0 && h == 0 && part == 0,
                                     table, u);

@@ -155,6 +155,27 @@ cudaError_t allow_smem(Kernel k, size_t bytes, std::atomic<size_t> (&done)[kMaxD
     return cudaSuccess;
 }
 
+// Every kernel of the library is launched with programmatic stream
+// serialisation: it may be scheduled while the previous kernel of the stream
+// drains, and it waits (griddepcontrol.wait) for that kernel before reading
+// or writing anything, in every CTA, so stream order holds for all data.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <typename T, int D, int BS>
 pa_status launch_decode(const DecodeParams &p, cudaStream_t stream)
 {
@@ -164,23 +185,13 @@ pa_status launch_decode(const DecodeParams &p, cudaStream_t stream)
     cudaError_t e = allow_smem(kernel, Cfg::smem_bytes(kMaxPartition), smem_set);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute(decode)");
-    dim3 grid(p.num_heads, p.num_seqs, p.num_parts);
-    kernel<<<grid, kSplitWarps * 32, Cfg::smem_bytes(p.partition_size), stream>>>(p);
-    e = cudaGetLastError();
+    e = launch_pdl(kernel, dim3(p.num_heads, p.num_seqs, p.num_parts), dim3(kSplitWarps * 32),
+                   Cfg::smem_bytes(p.partition_size), stream, p);
     if (e != cudaSuccess)
         return cuda_fail(e, "decode launch");
     if (p.num_parts > 1) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(p.num_heads, p.num_seqs, 1);
-        cfg.blockDim = dim3(D, 1, 1);
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, reduce_kernel<D>, p, (int)BS);
+        e = launch_pdl(reduce_kernel<D>, dim3(p.num_heads, p.num_seqs, 1), dim3(D), 0, stream, p,
+                       (int)BS);
         if (e != cudaSuccess)
             return cuda_fail(e, "reduce launch");
     }
@@ -253,8 +264,8 @@ pa_status pa_write_kv(const void *key, const void *value, int32_t num_tokens, in
     p.num_heads = num_heads;
     p.vecs_per_row = cache->head_dim * 2 / 16;
     p.block_size = cache->block_size;
-    write_kv_kernel<<<num_tokens, 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(write_kv_kernel, dim3(num_tokens), dim3(128), 0,
+                               static_cast<cudaStream_t>(stream), p);
     if (e != cudaSuccess)
         return cuda_fail(e, "write_kv launch");
     return ok();
@@ -387,9 +398,8 @@ pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches, int
     p.dev_err = dev_err;
     p.block_vecs = (int64_t)cache->num_kv_heads * cache->block_size * cache->head_dim * 2 / 16;
     p.num_blocks = cache->num_blocks;
-    dim3 grid(num_pairs, num_layers, 2);
-    copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(copy_blocks_kernel, dim3(num_pairs, num_layers, 2), dim3(256), 0,
+                               static_cast<cudaStream_t>(stream), p);
     if (e != cudaSuccess)
         return cuda_fail(e, "copy_blocks launch");
     return ok();
