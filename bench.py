@@ -11,6 +11,10 @@ for every layer of the workload. The default workload is the Llama-7B-shaped
 single layer: 96 sequences, 32 heads, head_dim 128, block size 16, context
 lengths uniform in [128, 2048], an 8192-block pool.
 
+By default each layer's K/V write and decode run as one launch
+(pa_write_kv_decode) and the whole step is replayed from a CUDA graph;
+--separate uses pa_write_kv + pa_decode, --no-graph launches from the host.
+
 Under torchrun (N > 1) every rank runs an independent replica of the workload
 (the path has no exchange step); the time is the maximum over ranks and the
 value counts the query tokens of all ranks.
@@ -62,9 +66,12 @@ WORKLOADS = {
                        "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 16"),
     "full_step_bs32": (lambda seed: wl.full_step(seed=seed, block_size=32),
                        "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 32"),
+    "small_batch_step": (lambda seed: wl.full_step(seed=seed, block_size=16, num_seqs=8),
+                         "small_batch_step: 32 layers, 8 seqs, ctx min(Geom(1/300),4096), "
+                         "bs 16 (launch-bound)"),
 }
 SEEDS = {"tiny": 0, "llama7b_layer": 1, "long_context": 2, "prefix_cow": 3,
-         "full_step_bs8": 4, "full_step_bs16": 4, "full_step_bs32": 4}
+         "full_step_bs8": 4, "full_step_bs16": 4, "full_step_bs32": 4, "small_batch_step": 5}
 
 
 def algorithmic_bytes(step) -> dict:
@@ -229,6 +236,41 @@ def cpu_baseline(step, target_seconds=12.0):
                        f"to whole decode steps")}
 
 
+def block_manager_timing(step, reps=200):
+    """Host cost of producing one decode step's integer inputs (append one
+    token per sequence: tables, context lengths, slots, copy-on-write pairs)
+    with the library's C++ block manager and with the Python allocator of
+    workloads/, on the workload's sequence lengths."""
+    from paged_kv_cache_417_b200.block_manager import BlockManager
+    S, bs = step.num_seqs, step.block_size
+    pre = (step.context_lens - 1).astype(np.int64)
+    nb = int(np.sum(-(-(pre + reps + 1) // bs))) + S + 16
+    order = np.random.default_rng(7).permutation(nb)
+    mb = int(np.max(-(-(pre + reps + 1) // bs)))
+    cc = BlockManager(nb, bs, order)
+    for i in range(S):
+        cc.add_sequence(i)
+        cc.allocate_tokens(i, int(pre[i]))
+    ids = np.arange(S, dtype=np.int64)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        cc.prepare_decode(ids, mb)
+    cpp = (time.perf_counter() - t0) / reps
+    alloc = wl.BlockAllocator(nb, bs, order)
+    seqs = [wl.Sequence() for _ in range(S)]
+    for i in range(S):
+        wl.allocate_tokens(alloc, seqs[i], int(pre[i]))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        bt = np.full((S, mb), -1, dtype=np.int32)
+        for i, sq in enumerate(seqs):
+            wl.append_token(alloc, sq)
+            bt[i, :len(sq.block_table)] = sq.block_table
+    py = (time.perf_counter() - t0) / reps
+    return {"seqs": S, "cpp_us_per_step": cpp * 1e6, "python_us_per_step": py * 1e6,
+            "reps": reps}
+
+
 def max_over_ranks(x, dist=None, device=None):
     """The maximum of a per-rank number over all ranks (identity alone)."""
     if dist is None:
@@ -287,9 +329,15 @@ def main():
                     help="llama7b_layer only: this many sequences (pool scaled to match), "
                          "for profiler captures on a smaller case of the same kernel")
     ap.add_argument("--soak-seconds", type=float, default=1.0)
+    ap.add_argument("--separate", action="store_true",
+                    help="pa_write_kv then pa_decode instead of the fused pa_write_kv_decode")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every step from the host instead of replaying a CUDA graph")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    args.fused = not args.separate
+    args.graph = not args.no_graph
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
@@ -301,7 +349,9 @@ def main():
                    "l2": "flushed between steps (256 MiB read)" if flush else
                          "not flushed (shared-prefix reuse is part of the workload)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "partition": args.partition or "auto"}
+                   "partition": args.partition or "auto",
+                   "launch": ("fused write+decode" if args.fused else "write_kv, decode") +
+                             (", CUDA graph" if args.graph else "")}
 
     if args.impl == "reference":
         if rank == 0:
@@ -338,7 +388,8 @@ def main():
                                  step.max_context_len, args.partition)
     split = step.max_context_len > P
     has_copy = step.copy_pairs.shape[0] > 0
-    launches_per_step = (1 if has_copy else 0) + L * (2 + (1 if split else 0))
+    launches_per_step = (1 if has_copy else 0) + L * ((1 if args.fused else 2) +
+                                                       (1 if split else 0))
     # L2 flush by reading 256 MiB: the previous step's lines are evicted and
     # L2 is left holding clean lines, so no write-back lands on the next step.
     flush_buf = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
@@ -347,19 +398,29 @@ def main():
         if flush:
             flush_buf.sum()
 
-    def one_step(dec_events=None, inputs=None):
+    def one_step(dec_events=None, inputs=None, out_list=None):
         src = inputs or d
+        dst = out_list or outs
         if has_copy:
             pk.copy_blocks(d["key_caches"], d["value_caches"], src["copy_pairs"])
         for li in range(L):
             kc, vc = d["key_caches"][li], d["value_caches"][li]
-            pk.write_kv(src["new_key"][li], src["new_value"][li], src["slot_mapping"], kc, vc)
+            if not args.fused:
+                pk.write_kv(src["new_key"][li], src["new_value"][li], src["slot_mapping"], kc,
+                            vc)
             if dec_events is not None:
                 dec_events[0].append(torch.cuda.Event(enable_timing=True))
                 dec_events[0][-1].record(stream)
-            pk.decode(outs[li], src["query"][li], kc, vc, src["block_tables"],
-                      src["context_lens"], step.max_context_len, float(step.scale),
-                      partition_size=args.partition, workspace=ws)
+            if args.fused:
+                pk.write_kv_decode(dst[li], src["query"][li], src["new_key"][li],
+                                   src["new_value"][li], kc, vc, src["block_tables"],
+                                   src["context_lens"], step.max_context_len,
+                                   float(step.scale), partition_size=args.partition,
+                                   workspace=ws)
+            else:
+                pk.decode(dst[li], src["query"][li], kc, vc, src["block_tables"],
+                          src["context_lens"], step.max_context_len, float(step.scale),
+                          partition_size=args.partition, workspace=ws)
             if dec_events is not None:
                 dec_events[1].append(torch.cuda.Event(enable_timing=True))
                 dec_events[1][-1].record(stream)
@@ -393,6 +454,40 @@ def main():
         secs = min(1.0, 1.5 * args.steps * host_step_s + 0.002)
         torch.cuda._sleep(int(secs * 2.0e9))
 
+    def capture(inputs=None, out_list=None):
+        """The whole step recorded once as a CUDA graph (the library only
+        enqueues kernels on the current stream, allocates nothing and never
+        synchronises, so it can be captured)."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one_step(inputs=inputs, out_list=out_list)
+        torch.cuda.synchronize(dev)
+        return g
+
+    run_step = one_step
+    if args.graph:
+        graph_main = capture()
+        run_step = lambda dec_events=None, inputs=None: graph_main.replay()  # noqa: E731
+        for _ in range(args.warmup):
+            flush_l2()
+            run_step()
+        torch.cuda.synchronize(dev)
+
+    def host_paced(n):
+        """Steps per second when the host launches each step as it goes (no
+        head start): host launch cost shows here when it exceeds GPU time."""
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            run_step()
+        b.record(stream)
+        barrier()
+        return job_throughput(world, S, n, max_over_ranks(a.elapsed_time(b), dist, dev))
+
+    paced = host_paced(args.steps)
+
     # Timed region: K steps, L2 flushed between them, each step bracketed by
     # CUDA events on the launching stream.
     barrier()
@@ -403,9 +498,17 @@ def main():
     for k in range(args.steps):
         flush_l2()
         starts[k].record(stream)
-        one_step(dec_events)
+        run_step(dec_events)
         ends[k].record(stream)
     barrier()
+    if args.graph:
+        # Decode events cannot sit inside a replayed graph: time the decode
+        # calls on the eager path, same steps, for the roofline.
+        head_start()
+        for k in range(args.steps):
+            flush_l2()
+            one_step(dec_events)
+        barrier()
     clocks = sampler.stop()
     step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     dec_ms = [a.elapsed_time(b) for a, b in zip(*dec_events)]
@@ -428,55 +531,110 @@ def main():
                 "kv_gbs": ab["kv"] / dec_avg_s / 1e9,
                 "frac_of_8tbs": achieved / NORTH_STAR_PEAK_GBS}
 
-    # End to end through the public API with host buffers: pinned host ->
-    # device copies of the step's inputs, the step, device -> host output.
+    # End to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory to the device and its outputs back,
+    # as one packed DMA each way. Two input/output buffer sets and a copy
+    # stream pipeline the steps, so a step's copies overlap its neighbours'
+    # compute on the copy engines. No L2 flush here: every step reads more
+    # K/V than L2 holds.
     e2e = None
     if not args.no_e2e:
-        host = {k: [t.cpu().pin_memory() for t in d[k]] for k in ("query", "new_key", "new_value")}
-        for k in ("slot_mapping", "block_tables", "context_lens", "copy_pairs"):
-            host[k] = d[k].cpu().pin_memory()
-        dev_in = {k: [torch.empty_like(t) for t in d[k]] for k in ("query", "new_key", "new_value")}
-        for k in ("slot_mapping", "block_tables", "context_lens", "copy_pairs"):
-            dev_in[k] = torch.empty_like(d[k])
-        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-        h2d = sum(t.numel() * t.element_size() for k in ("query", "new_key", "new_value")
-                  for t in host[k])
-        h2d += sum(host[k].numel() * host[k].element_size()
-                   for k in ("slot_mapping", "block_tables", "context_lens"))
+        names = [(k, i) for k in ("query", "new_key", "new_value") for i in range(L)]
+        names += [(k, None) for k in ("slot_mapping", "block_tables", "context_lens")]
         if has_copy:
-            h2d += host["copy_pairs"].numel() * 8
-        d2h = sum(o.numel() * o.element_size() for o in outs)
+            names.append(("copy_pairs", None))
 
-        def e2e_step():
-            for k in ("query", "new_key", "new_value"):
-                for a, b in zip(dev_in[k], host[k]):
-                    a.copy_(b, non_blocking=True)
-            for k in ("slot_mapping", "block_tables", "context_lens") + (
-                    ("copy_pairs",) if has_copy else ()):
-                dev_in[k].copy_(host[k], non_blocking=True)
-            one_step(inputs=dev_in)
-            for a, b in zip(host_out, outs):
-                a.copy_(b, non_blocking=True)
+        def tensor_of(name):
+            k, i = name
+            return d[k][i] if i is not None else d[k]
 
-        for _ in range(args.warmup):
-            e2e_step()
+        layout, off = [], 0
+        for nm in names:
+            t = tensor_of(nm)
+            nbytes = t.numel() * t.element_size()
+            layout.append((nm, off, nbytes, t.dtype, t.shape))
+            off = (off + nbytes + 255) // 256 * 256
+        h2d = off
+        host_in = torch.empty(h2d, dtype=torch.uint8, pin_memory=True)
+        for nm, o, nbytes, _, _ in layout:
+            host_in[o:o + nbytes].copy_(tensor_of(nm).reshape(-1).view(torch.uint8).cpu())
+        out_bytes = [o.numel() * o.element_size() for o in outs]
+        d2h = sum(out_bytes)
+
+        def views(buf):
+            v = {"query": [None] * L, "new_key": [None] * L, "new_value": [None] * L,
+                 "copy_pairs": d["copy_pairs"]}
+            for (k, i), o, nbytes, dt, shape in layout:
+                t = buf[o:o + nbytes].view(dt).view(shape)
+                if i is None:
+                    v[k] = t
+                else:
+                    v[k][i] = t
+            return v
+
+        bufs = []
+        for _ in range(2):
+            dev_in = torch.empty(h2d, dtype=torch.uint8, device=dev)
+            dev_out = torch.empty(d2h, dtype=torch.uint8, device=dev)
+            out_list, o = [], 0
+            for ref, nb in zip(outs, out_bytes):
+                out_list.append(dev_out[o:o + nb].view(ref.dtype).view(ref.shape))
+                o += nb
+            bf = {"dev_in": dev_in, "in": views(dev_in), "dev_out": dev_out, "out": out_list,
+                  "host_out": torch.empty(d2h, dtype=torch.uint8, pin_memory=True)}
+            if args.graph:
+                bf["graph"] = capture(inputs=bf["in"], out_list=bf["out"])
+            bufs.append(bf)
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)  # H2D and D2H copy streams
+        ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("h2d", "step", "d2h")}
+
+        def e2e_run(n, sleep_s=0.0):
+            with torch.cuda.stream(up):
+                if sleep_s:
+                    torch.cuda._sleep(int(sleep_s * 2.0e9))
+                t0 = torch.cuda.Event(enable_timing=True)
+                t0.record(up)
+            for k in range(n):
+                b = k % 2
+                bf = bufs[b]
+                with torch.cuda.stream(up):
+                    if k >= 2:
+                        up.wait_event(ev["step"][b])  # step k-2 has read these inputs
+                    bf["dev_in"].copy_(host_in, non_blocking=True)
+                    ev["h2d"][b].record(up)
+                stream.wait_event(ev["h2d"][b])
+                if k >= 2:
+                    stream.wait_event(ev["d2h"][b])  # outputs of step k-2 copied out
+                if args.graph:
+                    bf["graph"].replay()
+                else:
+                    one_step(inputs=bf["in"], out_list=bf["out"])
+                ev["step"][b].record(stream)
+                with torch.cuda.stream(down):
+                    down.wait_event(ev["step"][b])
+                    bf["host_out"].copy_(bf["dev_out"], non_blocking=True)
+                    ev["d2h"][b].record(down)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t1.record(down)
+            return t0, t1
+
         barrier()
-        es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        head_start()
-        for k in range(args.steps):
-            flush_l2()
-            es[k].record(stream)
-            e2e_step()
-            ee[k].record(stream)
+        h0 = time.perf_counter()
+        e2e_run(args.warmup)
+        host_e2e_s = (time.perf_counter() - h0) / args.warmup
         barrier()
-        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(es, ee)), dist, dev)
+        t0, t1 = e2e_run(args.steps, min(1.0, 1.5 * args.steps * host_e2e_s + 0.002))
+        barrier()
+        e2e_ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
         e2e = {"value": job_throughput(world, S, args.steps, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "how": "one packed pinned-host DMA each way per step, 2 buffer sets, "
+                      "separate upload and download streams overlapping compute"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(step)
+    bm_timing = block_manager_timing(step) if rank == 0 else None
 
     if rank == 0:
         line = {
@@ -487,6 +645,7 @@ def main():
             "accumulate": "f32", "data": "synthetic", "config": config_desc,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+            "host_paced_value": paced, "host_block_manager": bm_timing,
             "partition_size": P, "split": split,
         }
         print(json.dumps(line), flush=True)

@@ -139,6 +139,30 @@ pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t nu
                     void *workspace, size_t workspace_bytes, int32_t *dev_err,
                     void *stream);
 
+/* pa_write_kv_decode - pa_write_kv followed by pa_decode for a batch in
+ * which every sequence appends exactly one token, in one launch.
+ *
+ * The request lifecycle appends each sequence's new token and runs attention
+ * over all its tokens ("vLLM基础", §2.2 steps 4-6); here the new token of
+ * sequence s is its last context token, position context_lens[s] - 1, and
+ * its slot is the one the block table gives that position (the in-order
+ * fill of "啃透vLLM源码", §2.2 append_tokens). key/value (device
+ * [num_seqs][num_heads][head_dim], cache dtype, 16-byte aligned) hold the
+ * new rows. The result equals pa_write_kv with that slot mapping followed by
+ * pa_decode; the kernel that reads the sequence's last chunk puts the new
+ * row into its staged copy and into the cache, so no other launch is needed.
+ * Preconditions: the block that receives the new token is read by no other
+ * sequence of the call (copy-on-write has already run); context_lens[s] = 0
+ * appends nothing. All other arguments and errors are as for pa_decode.
+ */
+pa_status pa_write_kv_decode(void *out, pa_dtype out_dtype, const void *query, const void *key,
+                             const void *value, int32_t num_seqs, int32_t num_heads,
+                             void *key_cache, void *value_cache, const pa_cache_desc *cache,
+                             const int32_t *block_tables, int32_t max_blocks_per_seq,
+                             const int32_t *context_lens, int32_t max_context_len, float scale,
+                             int32_t partition_size, void *workspace, size_t workspace_bytes,
+                             int32_t *dev_err, void *stream);
+
 /* pa_decode_noalloc - pa_decode without a caller-provided workspace, for
  * callers that cannot allocate device memory when they decode.
  *

@@ -4,7 +4,7 @@ and its cache-maintenance calls on B200 (sm_100a).
 Argument marshalling only: tensors are passed to the C ABI as raw device
 pointers with the current CUDA stream; every step of the computation runs in
 the library's kernels. There is no fallback: importing this module fails if
-the library has not been built (``python -m paged_kv_cache_417_b200.build``).
+the library has not been built (``python paged_kv_cache_417_b200/build.py``).
 
 Cache tensors are [num_blocks, num_heads, block_size, head_dim] fp16/bf16
 (see the header for the full contract).
@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_417_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python paged_kv_cache_417_b200/build.py` "
         "(nvcc, sm_100a). There is no non-CUDA fallback.")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -55,6 +55,10 @@ _lib.pa_decode_partition_size.argtypes = [_i32] * 6
 _lib.pa_decode.restype = ctypes.c_int
 _lib.pa_decode.argtypes = [_P, ctypes.c_int, _P, _i32, _i32, _P, _P, ctypes.POINTER(CacheDesc),
                            _P, _i32, _P, _i32, ctypes.c_float, _i32, _P, ctypes.c_size_t, _P, _P]
+_lib.pa_write_kv_decode.restype = ctypes.c_int
+_lib.pa_write_kv_decode.argtypes = [_P, ctypes.c_int, _P, _P, _P, _i32, _i32, _P, _P,
+                                    ctypes.POINTER(CacheDesc), _P, _i32, _P, _i32,
+                                    ctypes.c_float, _i32, _P, ctypes.c_size_t, _P, _P]
 _lib.pa_decode_noalloc.restype = ctypes.c_int
 _lib.pa_decode_noalloc.argtypes = [_P, ctypes.c_int, _P, _i32, _i32, _P, _P,
                                    ctypes.POINTER(CacheDesc), _P, _i32, _P, _i32,
@@ -178,6 +182,43 @@ def decode(out, query, key_cache, value_cache, block_tables, context_lens, max_c
                           int(partition_size), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _ptr(dev_err),
                           _stream(query)))
+    return out
+
+
+def write_kv_decode(out, query, key, value, key_cache, value_cache, block_tables,
+                    context_lens, max_context_len, scale, partition_size=0, workspace=None,
+                    dev_err=None):
+    """:func:`write_kv` + :func:`decode` in one launch for a batch where
+    every sequence appends one token: ``key``/``value`` [S, H, D] are the new
+    rows, stored at position ``context_lens[s] - 1`` of each sequence (the
+    slot its block table gives), and attention covers every token including
+    them."""
+    _need(query, "query", key_cache.dtype)
+    _need(key, "key", key_cache.dtype)
+    _need(value, "value", key_cache.dtype)
+    _need(key_cache, "key_cache")
+    _need(value_cache, "value_cache", key_cache.dtype)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    _need(out, "out")
+    if out.dtype not in _DTYPE:
+        raise ValueError("out dtype must be float16, bfloat16 or float32")
+    if not (out.shape == query.shape == key.shape == value.shape) or \
+            value_cache.shape != key_cache.shape:
+        raise ValueError("shape mismatch")
+    desc = cache_desc(key_cache)
+    S, H, D = query.shape
+    if workspace is None:
+        workspace = alloc_workspace(S, H, D, int(max_context_len), partition_size,
+                                    query.device)
+    mb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    _check(_lib.pa_write_kv_decode(_ptr(out), _DTYPE[out.dtype], _ptr(query), _ptr(key),
+                                   _ptr(value), S, H, _ptr(key_cache), _ptr(value_cache),
+                                   ctypes.byref(desc), _ptr(block_tables), mb,
+                                   _ptr(context_lens), int(max_context_len), float(scale),
+                                   int(partition_size), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(),
+                                   _ptr(dev_err), _stream(query)))
     return out
 
 

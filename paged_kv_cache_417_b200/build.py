@@ -1,6 +1,9 @@
 """Build libpagedkv.so in-tree with nvcc for sm_100a.
 
-    python -m paged_kv_cache_417_b200.build [--force] [--verbose]
+    python paged_kv_cache_417_b200/build.py [--force] [--ptxas-verbose]
+
+Run it by path (or through __graft_entry__.build()): importing the package
+loads the library this script builds.
 """
 from __future__ import annotations
 
@@ -26,11 +29,12 @@ NVCC_FLAGS = [
 
 
 def sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def deps():
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + \
+        sorted(glob.glob(os.path.join(CSRC, "*.h"))) + \
         sorted(glob.glob(os.path.join(INCLUDE, "*.h"))) + [os.path.abspath(__file__)]
 
 

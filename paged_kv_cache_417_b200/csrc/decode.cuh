@@ -65,6 +65,11 @@ struct DecodeParams {
     int32_t partition_size, num_parts;
     int32_t out_dtype; // 0 f16, 1 bf16, 2 f32
     float qk_scale_log2;
+    // Fused append (pa_write_kv_decode): the new token of sequence s, at
+    // position context_lens[s] - 1, has K/V rows new_key/new_value[s][h][:];
+    // NULL for a plain decode.
+    const void *new_key;
+    const void *new_value;
 };
 
 template <typename T> struct Elem;
@@ -145,6 +150,13 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
     float m, l;
     int qd, r, rx, lane;
     int bad_id; // lane 0: a block id outside the pool was met
+    // Fused append: local chunk patch_i holds the new token at row
+    // patch_row. Lanes < 2*D/8 carry 16 bytes of its K (then V) row in
+    // patch_val, which replace that row in shared memory once the chunk has
+    // landed and go to the cache at patch_dst (NULL: the block id was bad).
+    int patch_i, patch_row;
+    uint4 patch_val;
+    uint4 *patch_dst;
 
     __device__ __forceinline__ void init(const T *q, float qk_scale_log2, int lane_)
     {
@@ -165,6 +177,9 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
         m = -INFINITY;
         l = 0.f;
         bad_id = 0;
+        patch_i = -1;
+        patch_row = 0;
+        patch_dst = nullptr;
     }
 
     // Stream chunks c0, c0 + cstride, ... (count of them) of a unit with
@@ -210,8 +225,19 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
             if (__any_sync(FULL, !ok))
                 break;
             const int rows = min(CHUNK, n_tok - (c0 + i * cstride) * CHUNK);
-            const T *sk = ring + st * 2 * TILE;
-            const T *sv = sk + TILE;
+            T *sk = ring + st * 2 * TILE;
+            T *sv = sk + TILE;
+            if (i == patch_i) { // warp-uniform
+                constexpr int RV = D * 2 / 16;
+                if (lane < 2 * RV) {
+                    T *srow = (lane >= RV ? sv : sk) + patch_row * D;
+                    reinterpret_cast<uint4 *>(srow)[lane % RV] = patch_val;
+                    if (patch_dst)
+                        *patch_dst = patch_val;
+                    fence_proxy_async_smem(); // before the stage is refilled by a bulk copy
+                }
+                __syncwarp();
+            }
 
             float sc[STEPS];
 #pragma unroll
@@ -393,6 +419,31 @@ __global__ void __launch_bounds__(NW * 32)
     ws.init(static_cast<const T *>(p.query) + ((size_t)s * H + h) * D, p.qk_scale_log2, lane);
     const int n_chunks = (u.n_tok + W::CHUNK - 1) / W::CHUNK;
     const int my_chunks = n_chunks <= warp ? 0 : (n_chunks - warp + NW - 1) / NW;
+    if (p.new_key != nullptr && part == u.num_parts - 1 && u.n_tok > 0) {
+        // This CTA holds the sequence's last token: the warp owning its
+        // chunk puts the new K/V row in place (shared memory and cache).
+        const int c_last = (u.n_tok - 1) / W::CHUNK;
+        if (c_last % NW == warp) {
+            constexpr int RV = D * 2 / 16;
+            ws.patch_i = c_last / NW;
+            ws.patch_row = (u.n_tok - 1) - c_last * W::CHUNK;
+            if (lane < 2 * RV) {
+                const bool isv = lane >= RV;
+                const int e = lane % RV;
+                ws.patch_val = reinterpret_cast<const uint4 *>(isv ? p.new_value : p.new_key)
+                    [((size_t)s * H + h) * RV + e];
+                const int b = table[(u.n_tok - 1) / BS];
+                if (b >= 0 && b < p.num_blocks) {
+                    T *cache = const_cast<T *>(
+                        static_cast<const T *>(isv ? p.value_cache : p.key_cache));
+                    ws.patch_dst = reinterpret_cast<uint4 *>(
+                                       cache + (size_t)b * H * BS * D + (size_t)h * BS * D +
+                                       (size_t)((u.n_tok - 1) % BS) * D) +
+                                   e;
+                }
+            }
+        }
+    }
     const bool ok = ws.run(static_cast<const T *>(p.key_cache),
                            static_cast<const T *>(p.value_cache), (size_t)h * BS * D,
                            (size_t)H * BS * D, p.num_blocks, table, u.n_tok, warp, NW,

@@ -11,6 +11,7 @@
 #include "pagedkv.h"
 
 #include "cache_ops.cuh"
+#include "last_error.h"
 #include "decode.cuh"
 
 using namespace pagedkv;
@@ -33,23 +34,6 @@ constexpr int kMinAutoPartition = 128;
 constexpr int kAutoPartition = 2048;
 constexpr int kPartitionQuantum = 32;
 constexpr int kMaxDevices = 64;
-
-thread_local char g_last_error[512] = "";
-
-pa_status fail(pa_status s, const char *fmt, ...)
-{
-    va_list ap;
-    va_start(ap, fmt);
-    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
-    va_end(ap);
-    return s;
-}
-
-pa_status ok()
-{
-    g_last_error[0] = '\0';
-    return PA_OK;
-}
 
 pa_status cuda_fail(cudaError_t e, const char *what)
 {
@@ -231,8 +215,6 @@ const char *pa_status_string(pa_status s)
     return "unknown status";
 }
 
-const char *pa_last_error(void) { return g_last_error; }
-
 int32_t pa_version(void) { return 100; }
 
 pa_status pa_write_kv(const void *key, const void *value, int32_t num_tokens, int32_t num_heads,
@@ -297,12 +279,18 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads, int32_t he
                             partition_size == 0 ? sm_count_of_current_device() : 148);
 }
 
-pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t num_seqs,
-                    int32_t num_heads, const void *key_cache, const void *value_cache,
-                    const pa_cache_desc *cache, const int32_t *block_tables,
-                    int32_t max_blocks_per_seq, const int32_t *context_lens,
-                    int32_t max_context_len, float scale, int32_t partition_size,
-                    void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream)
+} // extern "C"
+
+namespace {
+
+// pa_decode, and pa_write_kv_decode when new_key/new_value are given.
+pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_t num_seqs,
+                        int32_t num_heads, const void *key_cache, const void *value_cache,
+                        const pa_cache_desc *cache, const int32_t *block_tables,
+                        int32_t max_blocks_per_seq, const int32_t *context_lens,
+                        int32_t max_context_len, float scale, int32_t partition_size,
+                        void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                        void *stream, const void *new_key, const void *new_value)
 {
     pa_status s = check_cache(cache);
     if (s != PA_OK)
@@ -325,6 +313,12 @@ pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t nu
         return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
     if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
         return fail(PA_ERR_INVALID_ARG, "query and caches must be 16-byte aligned");
+    if (new_key || new_value) {
+        if (!new_key || !new_value)
+            return fail(PA_ERR_INVALID_ARG, "NULL key or value");
+        if (!aligned16(new_key) || !aligned16(new_value))
+            return fail(PA_ERR_INVALID_ARG, "key and value must be 16-byte aligned");
+    }
     if (!(scale == scale))
         return fail(PA_ERR_INVALID_ARG, "scale is NaN");
 
@@ -350,6 +344,8 @@ pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t nu
     p.num_parts = (int32_t)parts;
     p.out_dtype = (int32_t)out_dtype;
     p.qk_scale_log2 = scale * 1.4426950408889634f;
+    p.new_key = new_key;
+    p.new_value = new_value;
     if (parts > 1) {
         const int64_t units = (int64_t)num_seqs * num_heads;
         const size_t need = workspace_bytes_for(units, parts, cache->head_dim);
@@ -366,6 +362,39 @@ pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t nu
     if (cache->dtype == PA_F16)
         return dispatch_d<__half>(p, cache->head_dim, cache->block_size, st);
     return dispatch_d<__nv_bfloat16>(p, cache->head_dim, cache->block_size, st);
+}
+
+} // namespace
+
+extern "C" {
+
+pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t num_seqs,
+                    int32_t num_heads, const void *key_cache, const void *value_cache,
+                    const pa_cache_desc *cache, const int32_t *block_tables,
+                    int32_t max_blocks_per_seq, const int32_t *context_lens,
+                    int32_t max_context_len, float scale, int32_t partition_size,
+                    void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream)
+{
+    return decode_common(out, out_dtype, query, num_seqs, num_heads, key_cache, value_cache,
+                         cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                         scale, partition_size, workspace, workspace_bytes, dev_err, stream,
+                         nullptr, nullptr);
+}
+
+pa_status pa_write_kv_decode(void *out, pa_dtype out_dtype, const void *query, const void *key,
+                             const void *value, int32_t num_seqs, int32_t num_heads,
+                             void *key_cache, void *value_cache, const pa_cache_desc *cache,
+                             const int32_t *block_tables, int32_t max_blocks_per_seq,
+                             const int32_t *context_lens, int32_t max_context_len, float scale,
+                             int32_t partition_size, void *workspace, size_t workspace_bytes,
+                             int32_t *dev_err, void *stream)
+{
+    if (num_seqs > 0 && (!key || !value))
+        return fail(PA_ERR_INVALID_ARG, "NULL key or value");
+    return decode_common(out, out_dtype, query, num_seqs, num_heads, key_cache, value_cache,
+                         cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                         scale, partition_size, workspace, workspace_bytes, dev_err, stream,
+                         num_seqs > 0 ? key : nullptr, num_seqs > 0 ? value : nullptr);
 }
 
 pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches, int32_t num_layers,

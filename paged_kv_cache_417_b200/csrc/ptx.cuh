@@ -81,6 +81,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+// Order this thread's generic-proxy writes to shared memory before later
+// async-proxy (bulk copy) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Programmatic dependent launch: let the next kernel in the stream start its
 // launch now / wait here until the previous kernel's writes are visible. Both
 // are no-ops when the launch did not ask for it.
@@ -92,15 +99,6 @@ __device__ __forceinline__ void pdl_launch_dependents()
 __device__ __forceinline__ void pdl_wait_prior_grid()
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr)
-{
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr));
-    return v;
 }
 
 __device__ __forceinline__ void report(int32_t *dev_err, int32_t bits)

@@ -66,3 +66,23 @@ def decode_case(c, partition_size=0, out_dtype=None, max_context_len=None):
               dev_err=err)
     torch.cuda.synchronize()
     return out, int(err.item())
+
+
+def run_step_fused(step, layers=None, partition_size=0, out_dtype=None):
+    """copy_blocks (all layers) -> per layer write_kv_decode (one launch)."""
+    layers = list(range(step.num_layers)) if layers is None else list(layers)
+    d = device_step(step, "cuda", layers)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if step.copy_pairs.shape[0]:
+        pk.copy_blocks(d["key_caches"], d["value_caches"], d["copy_pairs"], dev_err=err)
+    outs = []
+    for i, _ in enumerate(layers):
+        q = d["query"][i]
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device="cuda")
+        pk.write_kv_decode(out, q, d["new_key"][i], d["new_value"][i], d["key_caches"][i],
+                           d["value_caches"][i], d["block_tables"], d["context_lens"],
+                           step.max_context_len, float(step.scale),
+                           partition_size=partition_size, dev_err=err)
+        outs.append(out)
+    torch.cuda.synchronize()
+    return outs, d, int(err.item())

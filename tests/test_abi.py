@@ -12,8 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def lib():
-    from paged_kv_cache_417_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import paged_kv_cache_417_b200 as pk
     return pk
 
@@ -30,7 +30,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ["pa_write_kv", "pa_decode", "pa_copy_blocks", "pa_decode_workspace_size",
-              "pa_status_string", "pa_last_error", "pa_version"]:
+              "pa_write_kv_decode", "pa_status_string", "pa_last_error", "pa_version"]:
         assert n in names
 
 
