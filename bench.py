@@ -66,12 +66,16 @@ WORKLOADS = {
                        "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 16"),
     "full_step_bs32": (lambda seed: wl.full_step(seed=seed, block_size=32),
                        "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 32"),
+    "swap_resume": (lambda seed: wl.llama_layer(seed=seed),
+                    "swap_resume: llama7b_layer whose every 4th sequence (24 of 96) is swapped "
+                    "in from pinned host memory (pa_swap_blocks) before each decode"),
     "small_batch_step": (lambda seed: wl.full_step(seed=seed, block_size=16, num_seqs=8),
                          "small_batch_step: 32 layers, 8 seqs, ctx min(Geom(1/300),4096), "
                          "bs 16 (launch-bound)"),
 }
 SEEDS = {"tiny": 0, "llama7b_layer": 1, "long_context": 2, "prefix_cow": 3,
-         "full_step_bs8": 4, "full_step_bs16": 4, "full_step_bs32": 4, "small_batch_step": 5}
+         "full_step_bs8": 4, "full_step_bs16": 4, "full_step_bs32": 4, "small_batch_step": 5,
+         "swap_resume": 1}
 
 
 def algorithmic_bytes(step) -> dict:
@@ -398,9 +402,31 @@ def main():
         if flush:
             flush_buf.sum()
 
+    # Swap-resume workload: a pinned host pool holds the blocks of every 4th
+    # sequence; each step swaps them into their GPU blocks first.
+    swap = None
+    if args.config == "swap_resume":
+        blocks = sorted({int(b) for s_ in range(0, S, 4) for b in step.block_tables[s_]
+                         if b >= 0})
+        hk = [d["key_caches"][li][torch.tensor(blocks, device=dev)].cpu().pin_memory()
+              for li in range(L)]
+        hv = [d["value_caches"][li][torch.tensor(blocks, device=dev)].cpu().pin_memory()
+              for li in range(L)]
+        swap = {"host_k": hk, "host_v": hv, "blocks": len(blocks),
+                "map": torch.tensor([[i, b] for i, b in enumerate(blocks)],
+                                    dtype=torch.int64, device=dev),
+                "bytes": 2 * L * len(blocks) * hk[0][0].numel() * hk[0].element_size()}
+        launches_per_step += 1
+
+    def swap_in():
+        pk.swap_blocks(swap["host_k"], swap["host_v"], d["key_caches"], d["value_caches"],
+                       swap["map"])
+
     def one_step(dec_events=None, inputs=None, out_list=None):
         src = inputs or d
         dst = out_list or outs
+        if swap is not None:
+            swap_in()
         if has_copy:
             pk.copy_blocks(d["key_caches"], d["value_caches"], src["copy_pairs"])
         for li in range(L):
@@ -531,6 +557,36 @@ def main():
                 "kv_gbs": ab["kv"] / dec_avg_s / 1e9,
                 "frac_of_8tbs": achieved / NORTH_STAR_PEAK_GBS}
 
+    swap_stats = None
+    if swap is not None:
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier()
+        for k in range(args.steps):
+            ev0[k].record(stream)
+            swap_in()
+            ev1[k].record(stream)
+        barrier()
+        swap_s = statistics.mean(a.elapsed_time(b) for a, b in zip(ev0, ev1)) / 1e3
+        # Reference: one contiguous pinned-host -> device copy of the same bytes.
+        ref_src = torch.empty(swap["bytes"], dtype=torch.uint8).pin_memory()
+        ref_dst = torch.empty(swap["bytes"], dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            ref_dst.copy_(ref_src, non_blocking=True)
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(10):
+            ref_dst.copy_(ref_src, non_blocking=True)
+        b.record(stream)
+        barrier()
+        ref_s = a.elapsed_time(b) / 10 / 1e3
+        swap_stats = {"blocks": swap["blocks"], "bytes_per_step": swap["bytes"],
+                      "swap_us": swap_s * 1e6, "swap_gbs": swap["bytes"] / swap_s / 1e9,
+                      "pinned_memcpy_gbs": swap["bytes"] / ref_s / 1e9,
+                      "frac_of_memcpy": ref_s / swap_s}
+
     # End to end through the public API with host buffers: every step copies
     # its inputs from pinned host memory to the device and its outputs back,
     # as one packed DMA each way. Two input/output buffer sets and a copy
@@ -645,7 +701,7 @@ def main():
             "accumulate": "f32", "data": "synthetic", "config": config_desc,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
-            "host_paced_value": paced, "host_block_manager": bm_timing,
+            "host_paced_value": paced, "host_block_manager": bm_timing, "swap": swap_stats,
             "partition_size": P, "split": split,
         }
         print(json.dumps(line), flush=True)

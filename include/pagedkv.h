@@ -219,6 +219,32 @@ pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches,
                          int32_t num_pairs, const pa_cache_desc *cache, int32_t *dev_err,
                          void *stream);
 
+/* pa_swap_blocks - move whole blocks between two pools of the same block
+ * shape, typically the GPU pool and a pool in pinned host memory: swap out
+ * when GPU memory runs short, swap in before the sequence runs again
+ * ("啃透vLLM源码", §3, blocks_to_swap_out / blocks_to_swap_in). For each pair i
+ * and layer l, block block_mapping[i][0] of the source K and V caches of
+ * layer l is copied to block block_mapping[i][1] of the destination caches.
+ *
+ * src_key_caches ... dst_value_caches  HOST arrays of num_layers pointers,
+ *               each to device memory or to pinned host memory that CUDA has
+ *               mapped for the device (cudaHostAlloc / cudaHostRegister);
+ *               pageable host memory is refused (PA_ERR_INVALID_ARG) before
+ *               any launch. 16-byte aligned.
+ * src, dst      pool shapes; block_size, heads, head_dim and dtype must match,
+ *               num_blocks may differ.
+ * block_mapping int64 [num_pairs][2], device or pinned host memory. Ids
+ *               outside their pool set PA_DEVERR_COPY_PAIR and are skipped.
+ *               Destinations must be distinct. num_pairs == 0 is a no-op.
+ * One launch moves every pair of every layer; the GPU reads or writes the
+ * host pool directly over the host link.
+ */
+pa_status pa_swap_blocks(void *const *src_key_caches, void *const *src_value_caches,
+                         const pa_cache_desc *src, void *const *dst_key_caches,
+                         void *const *dst_value_caches, const pa_cache_desc *dst,
+                         int32_t num_layers, const int64_t *block_mapping, int32_t num_pairs,
+                         int32_t *dev_err, void *stream);
+
 /* Static text for a status. */
 const char *pa_status_string(pa_status status);
 

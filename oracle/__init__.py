@@ -10,6 +10,8 @@ Functions and the passages they follow:
   assigns ("vLLM基础", §2.2 steps 4-6; "啃透vLLM源码", §2.2 append_tokens).
 * :func:`copy_blocks` - copy-on-write duplication of shared blocks
   ("vLLM基础", §2.3).
+* :func:`swap_blocks` - blocks moved between a GPU pool and a host pool
+  ("啃透vLLM源码", §3, swap out / swap in).
 * :func:`decode` - attention over the cache reached through physical block
   indices ("VLLM源码解析", core technology: paged_attention_forward); exact
   attention, gathered then evaluated with the textbook softmax in fp64.
@@ -60,6 +62,10 @@ class Oracle:
         L.oracle_copy_blocks.restype = ctypes.c_int
         L.oracle_copy_blocks.argtypes = [ctypes.POINTER(P), ctypes.POINTER(P), ctypes.c_int32,
                                          P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+        L.oracle_swap_blocks.restype = ctypes.c_int
+        L.oracle_swap_blocks.argtypes = [ctypes.POINTER(P), ctypes.POINTER(P), ctypes.c_int64,
+                                         ctypes.POINTER(P), ctypes.POINTER(P), ctypes.c_int64,
+                                         ctypes.c_int32, P, ctypes.c_int64, ctypes.c_int64]
         L.oracle_kv_cache_bytes.restype = ctypes.c_int64
         L.oracle_kv_cache_bytes.argtypes = [ctypes.c_int64] * 5
         L.oracle_widen.restype = ctypes.c_double
@@ -107,6 +113,24 @@ class Oracle:
                                          elems)
         if rc:
             raise ValueError("oracle_copy_blocks: block id outside the pool")
+
+    def swap_blocks(self, src_keys, src_values, dst_keys, dst_values, mapping):
+        """In place on the destination pools; mapping int64 [N, 2] =
+        (source block, destination block)."""
+        mapping = np.ascontiguousarray(mapping, dtype=np.int64).reshape(-1, 2)
+        L = len(src_keys)
+        if L == 0:
+            return
+        elems = int(np.prod(src_keys[0].shape[1:]))
+        for c in list(src_keys) + list(src_values) + list(dst_keys) + list(dst_values):
+            assert c.flags.c_contiguous and c.dtype == np.uint16
+            assert int(np.prod(c.shape[1:])) == elems
+        arr = lambda cs: (ctypes.c_void_p * L)(*[c.ctypes.data for c in cs])  # noqa: E731
+        rc = self.lib.oracle_swap_blocks(arr(src_keys), arr(src_values), src_keys[0].shape[0],
+                                         arr(dst_keys), arr(dst_values), dst_keys[0].shape[0],
+                                         L, _ptr(mapping), mapping.shape[0], elems)
+        if rc:
+            raise ValueError("oracle_swap_blocks: block id outside its pool")
 
     def decode(self, query, key_cache, value_cache, block_tables, context_lens, scale,
                dtype="f16", threads=0):
@@ -174,6 +198,10 @@ def copy_blocks(*a, **k):
 
 def decode(*a, **k):
     return default().decode(*a, **k)
+
+
+def swap_blocks(*a, **k):
+    return default().swap_blocks(*a, **k)
 
 
 def run_step(*a, **k):

@@ -125,6 +125,30 @@ int oracle_copy_blocks(uint16_t **key_caches, uint16_t **value_caches, int32_t n
     return 0;
 }
 
+/* Swap: copy whole blocks from one pool set to another of the same block
+ * shape (a GPU pool and a pool in host memory, "啃透vLLM源码", §3: blocks go
+ * to CPU memory when GPU memory runs short and come back when needed).
+ * mapping is [num_pairs][2] = (block in the source pools, block in the
+ * destination pools). Returns -1 on an id outside its pool (nothing copied). */
+int oracle_swap_blocks(uint16_t **src_k, uint16_t **src_v, int64_t src_blocks, uint16_t **dst_k,
+                       uint16_t **dst_v, int64_t dst_blocks, int32_t num_layers,
+                       const int64_t *mapping, int64_t num_pairs, int64_t block_elems)
+{
+    for (int64_t i = 0; i < num_pairs; ++i)
+        if (mapping[2 * i] < 0 || mapping[2 * i] >= src_blocks || mapping[2 * i + 1] < 0 ||
+            mapping[2 * i + 1] >= dst_blocks)
+            return -1;
+    for (int32_t l = 0; l < num_layers; ++l)
+        for (int64_t i = 0; i < num_pairs; ++i) {
+            int64_t a = mapping[2 * i], b = mapping[2 * i + 1];
+            memcpy(dst_k[l] + b * block_elems, src_k[l] + a * block_elems,
+                   (size_t)block_elems * sizeof(uint16_t));
+            memcpy(dst_v[l] + b * block_elems, src_v[l] + a * block_elems,
+                   (size_t)block_elems * sizeof(uint16_t));
+        }
+    return 0;
+}
+
 /* One (sequence, head): gather, then textbook softmax attention in fp64. */
 static int decode_one(double *out, const uint16_t *q16, const uint16_t *key_cache,
                       const uint16_t *value_cache, int64_t num_blocks, int32_t num_heads,

@@ -66,6 +66,10 @@ _lib.pa_decode_noalloc.argtypes = [_P, ctypes.c_int, _P, _i32, _i32, _P, _P,
 _lib.pa_copy_blocks.restype = ctypes.c_int
 _lib.pa_copy_blocks.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_P), _i32, _P, _i32,
                                 ctypes.POINTER(CacheDesc), _P, _P]
+_lib.pa_swap_blocks.restype = ctypes.c_int
+_lib.pa_swap_blocks.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(CacheDesc),
+                                ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(CacheDesc),
+                                _i32, _P, _i32, _P, _P]
 _lib.pa_status_string.restype = ctypes.c_char_p
 _lib.pa_status_string.argtypes = [ctypes.c_int]
 _lib.pa_last_error.restype = ctypes.c_char_p
@@ -271,3 +275,29 @@ def copy_blocks(key_caches, value_caches, block_mapping, dev_err=None):
     n = block_mapping.shape[0] if block_mapping.numel() else 0
     _check(_lib.pa_copy_blocks(kp, vp, L, _ptr(block_mapping), n, ctypes.byref(desc),
                                _ptr(dev_err), _stream(key_caches[0])))
+
+
+def swap_blocks(src_key_caches, src_value_caches, dst_key_caches, dst_value_caches,
+                block_mapping, dev_err=None):
+    """Copy block ``block_mapping[i][0]`` of every source layer's K/V cache to
+    block ``block_mapping[i][1]`` of the destination caches. Pools may be CUDA
+    tensors or pinned CPU tensors (swap out / swap in); pageable CPU memory
+    is refused. Runs on the current CUDA stream."""
+    L = len(src_key_caches)
+    groups = (src_key_caches, src_value_caches, dst_key_caches, dst_value_caches)
+    if L == 0 or any(len(g) != L for g in groups):
+        raise ValueError("need the same, non-zero number of caches in every list")
+    for g in groups:
+        for c in g:
+            if not c.is_contiguous():
+                raise ValueError("caches must be contiguous")
+    if block_mapping.dtype != torch.int64 or not block_mapping.is_contiguous():
+        raise ValueError("block_mapping must be a contiguous int64 tensor")
+    sd, dd = cache_desc(src_key_caches[0]), cache_desc(dst_key_caches[0])
+    arr = lambda cs: (_P * L)(*[c.data_ptr() for c in cs])  # noqa: E731
+    n = block_mapping.shape[0] if block_mapping.numel() else 0
+    dev = next((c.device for g in groups for c in g if c.is_cuda), None)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    _check(_lib.pa_swap_blocks(arr(src_key_caches), arr(src_value_caches), ctypes.byref(sd),
+                               arr(dst_key_caches), arr(dst_value_caches), ctypes.byref(dd),
+                               L, _ptr(block_mapping), n, _ptr(dev_err), stream))

@@ -5,6 +5,13 @@
 // "啃透vLLM源码", §2.2 append_tokens). One CTA per token; every head's row
 // is head_dim * 2 bytes, moved as 16-byte vectors.
 //
+// swap_blocks_kernel: whole blocks between two pool sets of one block shape,
+// typically a GPU pool and a pool in pinned host memory that the GPU reaches
+// over PCIe ("啃透vLLM源码", §3: blocks go to CPU memory when GPU memory
+// runs short and come back when needed). One CTA per (pair, layer, K-or-V),
+// eight 16-byte loads in flight per thread to cover the longer latency of
+// host memory.
+//
 // copy_blocks_kernel: copy-on-write duplication of whole shared blocks
 // ("vLLM基础", §2.3). One CTA per (pair, layer, K-or-V) copies one
 // num_heads * block_size * head_dim block with 16-byte vectors, four loads in
@@ -99,6 +106,46 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const __grid_constant_
     const uint4 *from = base + src * p.block_vecs;
     uint4 *to = base + dst * p.block_vecs;
     constexpr int U = 4;
+    const int64_t stride = (int64_t)blockDim.x * U;
+    int64_t i = threadIdx.x;
+    for (; i + (U - 1) * blockDim.x < p.block_vecs; i += stride) {
+        uint4 r[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            r[u] = from[i + u * blockDim.x];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            to[i + u * blockDim.x] = r[u];
+    }
+    for (; i < p.block_vecs; i += blockDim.x)
+        to[i] = from[i];
+}
+
+struct SwapParams {
+    const uint4 *src_k[PA_MAX_LAYERS];
+    const uint4 *src_v[PA_MAX_LAYERS];
+    uint4 *dst_k[PA_MAX_LAYERS];
+    uint4 *dst_v[PA_MAX_LAYERS];
+    const int64_t *block_mapping; // [N][2] = (source block, destination block)
+    int32_t *dev_err;
+    int64_t block_vecs;
+    int64_t src_blocks, dst_blocks;
+};
+
+__global__ void __launch_bounds__(256) swap_blocks_kernel(const __grid_constant__ SwapParams p)
+{
+    pdl_launch_dependents();
+    pdl_wait_prior_grid();
+    const int pair = blockIdx.x, layer = blockIdx.y, which = blockIdx.z;
+    const int64_t a = p.block_mapping[2 * pair], b = p.block_mapping[2 * pair + 1];
+    if (a < 0 || a >= p.src_blocks || b < 0 || b >= p.dst_blocks) {
+        if (threadIdx.x == 0 && layer == 0 && which == 0)
+            report(p.dev_err, PA_DEVERR_COPY_PAIR);
+        return;
+    }
+    const uint4 *from = (which ? p.src_v[layer] : p.src_k[layer]) + a * p.block_vecs;
+    uint4 *to = (which ? p.dst_v[layer] : p.dst_k[layer]) + b * p.block_vecs;
+    constexpr int U = 8;
     const int64_t stride = (int64_t)blockDim.x * U;
     int64_t i = threadIdx.x;
     for (; i + (U - 1) * blockDim.x < p.block_vecs; i += stride) {

@@ -434,6 +434,90 @@ pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches, int
     return ok();
 }
 
+// The address a kernel uses for `p`: device memory as is, pinned host memory
+// through its device mapping. Pageable host memory (which no kernel may
+// touch) and unknown pointers are refused.
+static pa_status device_view(const void *p, const char *what, const void **out)
+{
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(PA_ERR_INVALID_ARG, "%s: not a CUDA-visible pointer", what);
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+        *out = p;
+        return PA_OK;
+    }
+    if (a.type == cudaMemoryTypeHost && a.devicePointer) {
+        *out = a.devicePointer;
+        return PA_OK;
+    }
+    return fail(PA_ERR_INVALID_ARG,
+                "%s: pageable host memory (the GPU can only reach pinned host memory)", what);
+}
+
+pa_status pa_swap_blocks(void *const *src_key_caches, void *const *src_value_caches,
+                         const pa_cache_desc *src, void *const *dst_key_caches,
+                         void *const *dst_value_caches, const pa_cache_desc *dst,
+                         int32_t num_layers, const int64_t *block_mapping, int32_t num_pairs,
+                         int32_t *dev_err, void *stream)
+{
+    pa_status s = check_cache(src);
+    if (s != PA_OK)
+        return s;
+    if ((s = check_cache(dst)) != PA_OK)
+        return s;
+    if (src->block_size != dst->block_size || src->num_kv_heads != dst->num_kv_heads ||
+        src->head_dim != dst->head_dim || src->dtype != dst->dtype)
+        return fail(PA_ERR_INVALID_ARG, "source and destination pools differ in block shape");
+    if (num_pairs < 0)
+        return fail(PA_ERR_INVALID_ARG, "num_pairs %d < 0", num_pairs);
+    if (num_layers < 1 || num_layers > PA_MAX_LAYERS)
+        return fail(PA_ERR_INVALID_ARG, "num_layers %d outside [1, %d]", num_layers, PA_MAX_LAYERS);
+    if (num_pairs == 0)
+        return ok();
+    if (!block_mapping || !src_key_caches || !src_value_caches || !dst_key_caches ||
+        !dst_value_caches)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
+    SwapParams p;
+    const void *v = nullptr;
+    if ((s = device_view(block_mapping, "block_mapping", &v)) != PA_OK)
+        return s;
+    p.block_mapping = static_cast<const int64_t *>(v);
+    void *const *arrays[4] = {src_key_caches, src_value_caches, dst_key_caches, dst_value_caches};
+    const char *names[4] = {"source key cache", "source value cache", "destination key cache",
+                            "destination value cache"};
+    for (int l = 0; l < num_layers; ++l) {
+        const void *views[4];
+        for (int k = 0; k < 4; ++k) {
+            const void *ptr = arrays[k][l];
+            if (!ptr || !aligned16(ptr))
+                return fail(PA_ERR_INVALID_ARG, "%s of layer %d is NULL or not 16-byte aligned",
+                            names[k], l);
+            if ((s = device_view(ptr, names[k], &views[k])) != PA_OK)
+                return s;
+        }
+        p.src_k[l] = static_cast<const uint4 *>(views[0]);
+        p.src_v[l] = static_cast<const uint4 *>(views[1]);
+        p.dst_k[l] = static_cast<uint4 *>(const_cast<void *>(views[2]));
+        p.dst_v[l] = static_cast<uint4 *>(const_cast<void *>(views[3]));
+    }
+    for (int l = num_layers; l < PA_MAX_LAYERS; ++l) {
+        p.src_k[l] = p.src_v[l] = nullptr;
+        p.dst_k[l] = p.dst_v[l] = nullptr;
+    }
+    p.dev_err = dev_err;
+    p.block_vecs = (int64_t)src->num_kv_heads * src->block_size * src->head_dim * 2 / 16;
+    p.src_blocks = src->num_blocks;
+    p.dst_blocks = dst->num_blocks;
+    cudaError_t e = launch_pdl(swap_blocks_kernel, dim3(num_pairs, num_layers, 2), dim3(256), 0,
+                               static_cast<cudaStream_t>(stream), p);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "swap_blocks launch");
+    return ok();
+}
+
 } // extern "C"
 
 // ---------------------------------------------------------------------------

@@ -254,5 +254,33 @@ def pin_copy_blocks(orc, seed=16):
                 assert np.array_equal(vs[l][b], v0[l][b]), "V block changed"
 
 
+def pin_swap_blocks(orc, seed=17):
+    """Swapping blocks out to a second pool and back restores every byte;
+    each destination block equals its source; nothing else changes."""
+    rng = np.random.default_rng(seed)
+    L, H, bs, D = 2, 2, 8, 64
+    gk = [rng.integers(0, 1 << 16, size=(12, H, bs, D), dtype=np.uint16) for _ in range(L)]
+    gv = [rng.integers(0, 1 << 16, size=(12, H, bs, D), dtype=np.uint16) for _ in range(L)]
+    hk = [rng.integers(0, 1 << 16, size=(5, H, bs, D), dtype=np.uint16) for _ in range(L)]
+    hv = [rng.integers(0, 1 << 16, size=(5, H, bs, D), dtype=np.uint16) for _ in range(L)]
+    g0 = [x.copy() for x in gk + gv]
+    h0 = [x.copy() for x in hk + hv]
+    out_map = np.array([[3, 0], [11, 4], [6, 2]], dtype=np.int64)
+    orc.swap_blocks(gk, gv, hk, hv, out_map)
+    for l in range(L):
+        for a, b in out_map:
+            assert np.array_equal(hk[l][b], gk[l][a]) and np.array_equal(hv[l][b], gv[l][a])
+        for b in (1, 3):
+            assert np.array_equal(hk[l][b], h0[l][b]) and np.array_equal(hv[l][b], h0[L + l][b])
+    # Clobber the source blocks, swap back in: the original bytes return.
+    for l in range(L):
+        for a, _ in out_map:
+            gk[l][a] = 0
+            gv[l][a] = 0
+    orc.swap_blocks(hk, hv, gk, gv, out_map[:, ::-1])
+    for l in range(L):
+        assert np.array_equal(gk[l], g0[l]) and np.array_equal(gv[l], g0[L + l])
+
+
 ALL_PINS = [pin_dense, pin_bruteforce, pin_closed_forms, pin_permutation, pin_write_kv,
-            pin_copy_blocks]
+            pin_copy_blocks, pin_swap_blocks]

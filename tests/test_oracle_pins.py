@@ -140,6 +140,10 @@ MUTANTS = [
      "memcpy(value_cache + dst, key + src,"),
     ("copy_value_from_key", "memcpy(value_caches[l] + dst * block_elems, value_caches[l] + src",
      "memcpy(value_caches[l] + dst * block_elems, key_caches[l] + src"),
+    ("swap_value_from_key", "memcpy(dst_v[l] + b * block_elems, src_v[l] + a * block_elems,",
+     "memcpy(dst_v[l] + b * block_elems, src_k[l] + a * block_elems,"),
+    ("swap_wrong_dst", "memcpy(dst_k[l] + b * block_elems, src_k[l] + a * block_elems,",
+     "memcpy(dst_k[l] + a % dst_blocks * block_elems, src_k[l] + a * block_elems,"),
     ("f16_exponent_bias", "v = ldexp((double)(f | 0x400), e - 25);",
      "v = ldexp((double)(f | 0x400), e - 24);"),
 ]
