@@ -16,6 +16,9 @@ Functions and the passages they follow:
   indices ("VLLM源码解析", core technology: paged_attention_forward); exact
   attention, gathered then evaluated with the textbook softmax in fp64.
 * :func:`kv_cache_bytes` - the per-sequence K/V sizing ("vLLM基础", §2.3).
+* :func:`write_kv_fp8`, :func:`decode_fp8` - the same write and decode on an
+  fp8 (e4m3) cache with one fp32 scale per row (KV-cache quantisation, named
+  by "vLLM基础", §2.5 as further tuning; the format is a reading).
 
 Pinned by ``tests/test_oracle_pins.py`` (closed forms, brute force in 50-digit
 decimal arithmetic, dense attention through scipy's softmax on the unpaged
@@ -66,6 +69,18 @@ class Oracle:
         L.oracle_swap_blocks.argtypes = [ctypes.POINTER(P), ctypes.POINTER(P), ctypes.c_int64,
                                          ctypes.POINTER(P), ctypes.POINTER(P), ctypes.c_int64,
                                          ctypes.c_int32, P, ctypes.c_int64, ctypes.c_int64]
+        L.oracle_write_kv_fp8.restype = ctypes.c_int
+        L.oracle_write_kv_fp8.argtypes = [P, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int32,
+                                          ctypes.c_int32, P, P, P, ctypes.c_int64,
+                                          ctypes.c_int32]
+        L.oracle_decode_fp8.restype = ctypes.c_int
+        L.oracle_decode_fp8.argtypes = [P, P, ctypes.c_int, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int32, P, P, ctypes.c_int64, ctypes.c_int32,
+                                        P, ctypes.c_int32, P, ctypes.c_double, ctypes.c_int]
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         L.oracle_kv_cache_bytes.restype = ctypes.c_int64
         L.oracle_kv_cache_bytes.argtypes = [ctypes.c_int64] * 5
         L.oracle_widen.restype = ctypes.c_double
@@ -132,6 +147,45 @@ class Oracle:
         if rc:
             raise ValueError("oracle_swap_blocks: block id outside its pool")
 
+    def e4m3_decode(self, code: int) -> float:
+        return self.lib.oracle_e4m3_decode(int(code))
+
+    def e4m3_encode(self, x: float) -> int:
+        return int(self.lib.oracle_e4m3_encode(float(x)))
+
+    def write_kv_fp8(self, key, value, slot_mapping, key_cache, value_cache, block_size,
+                     io_dtype="f16"):
+        """Quantise new tokens into fp8 pools (uint8 [NB, H, bs*D + 4*bs])."""
+        key, value = _u16(key), _u16(value)
+        slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        T, H, D = key.shape
+        for c in (key_cache, value_cache):
+            assert c.flags.c_contiguous and c.dtype == np.uint8
+            assert c.shape[1:] == (H, block_size * D + 4 * block_size)
+        rc = self.lib.oracle_write_kv_fp8(_ptr(key), _ptr(value), _DT[io_dtype], T, H, D,
+                                          _ptr(slots), _ptr(key_cache), _ptr(value_cache),
+                                          key_cache.shape[0], block_size)
+        if rc:
+            raise ValueError("oracle_write_kv_fp8: slot outside the pool")
+
+    def decode_fp8(self, query, key_cache, value_cache, block_tables, context_lens, scale,
+                   block_size, io_dtype="f16", threads=0):
+        query = _u16(query)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+        S, H, D = query.shape
+        assert key_cache.dtype == np.uint8 and value_cache.shape == key_cache.shape
+        assert key_cache.shape[1:] == (H, block_size * D + 4 * block_size)
+        out = np.zeros((S, H, D), dtype=np.float64)
+        rc = self.lib.oracle_decode_fp8(_ptr(out), _ptr(query), _DT[io_dtype], S, H, D,
+                                        _ptr(np.ascontiguousarray(key_cache)),
+                                        _ptr(np.ascontiguousarray(value_cache)),
+                                        key_cache.shape[0], block_size, _ptr(bt), bt.shape[1],
+                                        _ptr(ctx), float(scale), int(threads))
+        if rc:
+            raise ValueError("oracle_decode_fp8: block id or context length outside the pool")
+        return out
+
     def decode(self, query, key_cache, value_cache, block_tables, context_lens, scale,
                dtype="f16", threads=0):
         """fp64 [S, H, D] attention output."""
@@ -158,8 +212,18 @@ class Oracle:
         pools in their post-step state."""
         from workloads import host_pools
         kc, vc = host_pools(step, layer)
-        self.copy_blocks([kc], [vc], step.copy_pairs)
         L = step.layers[layer]
+        if step.dtype == "fp8":
+            # Whole-block copies are byte copies: view the pools as 16-bit.
+            k16 = kc.reshape(kc.shape[0], -1).view(np.uint16)
+            v16 = vc.reshape(vc.shape[0], -1).view(np.uint16)
+            self.copy_blocks([k16], [v16], step.copy_pairs)
+            self.write_kv_fp8(L.new_key, L.new_value, step.slot_mapping, kc, vc,
+                              step.block_size, step.io_dtype)
+            out = self.decode_fp8(L.query, kc, vc, step.block_tables, step.context_lens,
+                                  float(step.scale), step.block_size, step.io_dtype, threads)
+            return out, kc, vc
+        self.copy_blocks([kc], [vc], step.copy_pairs)
         self.write_kv(L.new_key, L.new_value, step.slot_mapping, kc, vc, step.block_size)
         out = self.decode(L.query, kc, vc, step.block_tables, step.context_lens,
                           float(step.scale), step.dtype, threads)
@@ -202,6 +266,14 @@ def decode(*a, **k):
 
 def swap_blocks(*a, **k):
     return default().swap_blocks(*a, **k)
+
+
+def write_kv_fp8(*a, **k):
+    return default().write_kv_fp8(*a, **k)
+
+
+def decode_fp8(*a, **k):
+    return default().decode_fp8(*a, **k)
 
 
 def run_step(*a, **k):

@@ -282,5 +282,97 @@ def pin_swap_blocks(orc, seed=17):
         assert np.array_equal(gk[l], g0[l]) and np.array_equal(gv[l], g0[L + l])
 
 
+def e4m3_table():
+    """Value of every e4m3 code, from torch's own float8_e4m3fn conversion."""
+    import torch
+    return torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+def e4m3_nearest(x):
+    """Brute force: the finite e4m3 code nearest to each float x, ties to the
+    even code (the even mantissa), magnitudes above 448 clamped to 448."""
+    vals = e4m3_table()
+    finite = [c for c in range(256) if np.isfinite(vals[c])]
+    fv = vals[finite]
+    out = []
+    for v in np.asarray(x, dtype=np.float64).reshape(-1):
+        v = float(np.clip(v, -448.0, 448.0))
+        d = np.abs(fv - v)
+        best = np.nonzero(d == d.min())[0]
+        cands = [finite[i] for i in best]
+        if len(cands) > 1:
+            same_sign = [c for c in cands if (c >> 7) == (1 if np.signbit(v) else 0)]
+            cands = same_sign or cands
+            even = [c for c in cands if c % 2 == 0]
+            cands = even or cands
+        out.append(cands[0])
+    return np.array(out, dtype=np.uint8)
+
+
+def pin_fp8(orc, seed=18):
+    """e4m3 decoding equals torch's for all 256 codes; encoding is the
+    brute-force nearest value; a paged fp8 cache written row by row decodes
+    like dense attention over the dequantised rows."""
+    table = e4m3_table()
+    for c in range(256):
+        got = orc.e4m3_decode(c)
+        assert (np.isnan(got) and np.isnan(table[c])) or got == table[c], f"code {c:#x}"
+    rng = np.random.default_rng(seed)
+    fv = table[np.isfinite(table)]
+    mids = (np.sort(fv)[1:] + np.sort(fv)[:-1]) / 2          # exact ties
+    xs = np.concatenate([rng.standard_normal(300) * 10.0 ** rng.uniform(-4, 3, 300),
+                         mids[::7], [448.0, 447.99, 464.0, 464.01, 1e4, 2.0 ** -10, 1e-9,
+                                     -0.0, 0.0, 2.0 ** -9 * 7.5]]).astype(np.float32)
+    got = np.array([orc.e4m3_encode(x) for x in xs], dtype=np.uint8)
+    want = e4m3_nearest(xs)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, f"encode differs at {xs[bad[:3]]}: {got[bad[:3]]} vs {want[bad[:3]]}"
+    # Paged fp8 cache, written through slots one token at a time.
+    H, D, bs = 2, 64, 16
+    ctxs = [1, 17, 40]
+    nb = sum(-(-c // bs) for c in ctxs) + 2
+    tb = bs * D + 4 * bs
+    perm = rng.permutation(nb)
+    kc = np.full((nb, H, tb), 0x7F, dtype=np.uint8)
+    vc = kc.copy()
+    bt = np.full((3, 3), -1, dtype=np.int32)
+    K, V, nxt = [], [], 0
+    for s, c in enumerate(ctxs):
+        blocks = perm[nxt: nxt + -(-c // bs)]
+        nxt += len(blocks)
+        bt[s, : len(blocks)] = blocks
+        k = to_storage_bits(rng.standard_normal((c, H, D), dtype=np.float32), "f16")
+        v = to_storage_bits(rng.standard_normal((c, H, D), dtype=np.float32), "f16")
+        for t in range(c):
+            slot = np.array([blocks[t // bs] * bs + t % bs], dtype=np.int64)
+            orc.write_kv_fp8(k[t:t + 1], v[t:t + 1], slot, kc, vc, bs)
+        K.append(k)
+        V.append(v)
+    q = to_storage_bits(rng.standard_normal((3, H, D), dtype=np.float32), "f16")
+    got = orc.decode_fp8(q, kc, vc, bt, np.array(ctxs, dtype=np.int32), np.float32(0.125), bs)
+    for s, c in enumerate(ctxs):
+        kd = np.zeros((c, H, D))
+        vd = np.zeros((c, H, D))
+        for t in range(c):
+            b, o = bt[s][t // bs], t % bs
+            for h in range(H):
+                for pool, raw, dq in ((kc, K[s], kd), (vc, V[s], vd)):
+                    codes = pool[b, h, o * D:(o + 1) * D]
+                    sc = pool[b, h, bs * D + 4 * o: bs * D + 4 * o + 4].view(np.float32)[0]
+                    x = raw[t, h].view(np.float16).astype(np.float32)
+                    amax = np.float32(np.max(np.abs(x)))
+                    assert sc == amax / np.float32(448.0), "row scale"
+                    inv = np.float32(448.0) / amax
+                    assert np.array_equal(codes, e4m3_nearest(x * inv)), "row codes"
+                    dq[t, h] = table[codes] * np.float64(sc)
+                    err = np.abs(dq[t, h] - x)
+                    assert np.all(err <= np.abs(x) / 16 + np.float64(sc) * 2.0 ** -9 + 1e-7)
+        qf = q[s].view(np.float16).astype(np.float64)
+        scores = 0.125 * np.einsum("hd,nhd->hn", qf, kd)
+        p = scipy.special.softmax(scores, axis=-1)
+        ref = np.einsum("hn,nhd->hd", p, vd)
+        assert np.max(np.abs(got[s] - ref)) <= 1e-12, "fp8 decode vs dense"
+
+
 ALL_PINS = [pin_dense, pin_bruteforce, pin_closed_forms, pin_permutation, pin_write_kv,
-            pin_copy_blocks, pin_swap_blocks]
+            pin_copy_blocks, pin_swap_blocks, pin_fp8]

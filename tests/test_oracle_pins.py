@@ -135,7 +135,19 @@ MUTANTS = [
      "((block * num_heads + 0) * block_size + j % block_size)"),
     ("table_index", "int64_t block = table[j / block_size];",
      "int64_t block = table[(j / block_size + 1) % table_len];"),
+    ("fp8_table_index", "int64_t block = table[j / block_size];",
+     "int64_t block = table[(j / block_size + 1) % table_len];", 1),
     ("write_offset", "offset = slot % block_size;", "offset = 0;"),
+    ("fp8_write_offset", "offset = slot % block_size;", "offset = 0;", 1),
+    ("fp8_scale_ignored", "* head_dim + d]) * sk;", "* head_dim + d]);"),
+    ("fp8_value_scale_from_key", "* head_dim + d]) * sv;", "* head_dim + d]) * sk;"),
+    ("e4m3_ties_up", "double m = rint((a / ldexp(1.0, e) - 1.0) * 8.0);",
+     "double m = floor((a / ldexp(1.0, e) - 1.0) * 8.0 + 0.5);"),
+    ("e4m3_subnormal_step", "double m = rint(a * 512.0);", "double m = rint(a * 256.0);"),
+    ("e4m3_bias", "v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 11);"),
+    ("fp8_row_scale", "*scale = amax / 448.0f;", "*scale = amax / 440.0f;"),
+    ("fp8_no_saturation", "if (a >= 448.0)\n        return sign | 0x7e;",
+     "if (a >= 480.0)\n        return sign | 0x7e;"),
     ("write_value_from_key", "memcpy(value_cache + dst, value + src,",
      "memcpy(value_cache + dst, key + src,"),
     ("copy_value_from_key", "memcpy(value_caches[l] + dst * block_elems, value_caches[l] + src",
@@ -149,12 +161,27 @@ MUTANTS = [
 ]
 
 
-@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_planted_mistake_is_caught(tmp_path, name, old, new):
+def _plant(src, old, new, occurrence):
+    """Replace the occurrence-th (0-based) copy of `old`; with occurrence
+    None, `old` must be unique."""
+    if occurrence is None:
+        assert src.count(old) == 1, "mutation anchor not unique"
+        return src.replace(old, new)
+    pos = -1
+    for _ in range(occurrence + 1):
+        pos = src.index(old, pos + 1)
+    return src[:pos] + new + src[pos + len(old):]
+
+
+@pytest.mark.parametrize("mutant", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(tmp_path, mutant):
+    name, old, new = mutant[:3]
+    occurrence = mutant[3] if len(mutant) > 3 else None
     src = open(ORACLE_SRC).read()
-    assert src.count(old) == 1, f"mutation anchor for {name} not unique"
+    if occurrence is None and src.count(old) > 1:
+        occurrence = 0
     path = tmp_path / "oracle_mut.c"
-    path.write_text(src.replace(old, new))
+    path.write_text(_plant(src, old, new, occurrence))
     lib = tmp_path / "liboracle_mut.so"
     subprocess.run(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11", str(path),
                     "-o", str(lib), "-lm"], check=True)

@@ -20,8 +20,13 @@ def _bits_to_tensor(bits: np.ndarray, dtype: str, device) -> torch.Tensor:
 
 
 def device_pools(step: DecodeStep, layer: int, device, base_dev=None):
-    """Pre-step (key_cache, value_cache) of one layer, [NB, H, bs, D]."""
+    """Pre-step (key_cache, value_cache) of one layer, [NB, H, bs, D]
+    (fp8: uint8 [NB, H, bs*D + 4*bs], built on the host)."""
     bs, H, D = step.block_size, step.num_heads, step.head_dim
+    if step.dtype == "fp8":
+        from .steps import host_pools
+        k, v = host_pools(step, layer)
+        return torch.from_numpy(k).to(device), torch.from_numpy(v).to(device)
     if base_dev is None:
         base_dev = _bits_to_tensor(step.base, step.dtype, device)
     L = step.layers[layer]
@@ -43,7 +48,7 @@ def device_pools(step: DecodeStep, layer: int, device, base_dev=None):
 def device_step(step: DecodeStep, device, layers=None):
     """All inputs of a step on ``device`` as a dict of tensors."""
     layers = range(step.num_layers) if layers is None else layers
-    base_dev = _bits_to_tensor(step.base, step.dtype, device)
+    base_dev = None if step.dtype == "fp8" else _bits_to_tensor(step.base, step.dtype, device)
     out = {
         "context_lens": torch.from_numpy(step.context_lens).to(device),
         "block_tables": torch.from_numpy(step.block_tables).to(device),
@@ -57,8 +62,8 @@ def device_step(step: DecodeStep, device, layers=None):
         L = step.layers[li]
         out["key_caches"].append(kc)
         out["value_caches"].append(vc)
-        out["query"].append(_bits_to_tensor(L.query, step.dtype, device))
-        out["new_key"].append(_bits_to_tensor(L.new_key, step.dtype, device))
-        out["new_value"].append(_bits_to_tensor(L.new_value, step.dtype, device))
+        out["query"].append(_bits_to_tensor(L.query, step.io_dtype, device))
+        out["new_key"].append(_bits_to_tensor(L.new_key, step.io_dtype, device))
+        out["new_value"].append(_bits_to_tensor(L.new_value, step.io_dtype, device))
     del base_dev
     return out

@@ -28,7 +28,15 @@ from .allocator import BlockAllocator, Sequence, allocate_tokens, append_token
 
 F16_NAN = np.uint16(0x7E00)
 BF16_NAN = np.uint16(0x7FC0)
+E4M3_NAN = np.uint8(0x7F)
+F32_NAN_BYTES = np.array([np.nan], dtype=np.float32).view(np.uint8)
 MAX_BANK_ROWS = 32768
+
+
+def fp8_tile_bytes(block_size: int, head_dim: int) -> int:
+    """Bytes of one (block, head) tile of an fp8 pool: block_size rows of
+    head_dim e4m3 codes, then block_size fp32 row scales."""
+    return block_size * head_dim + 4 * block_size
 
 
 def to_storage_bits(x: np.ndarray, dtype: str) -> np.ndarray:
@@ -48,6 +56,12 @@ def to_storage_bits(x: np.ndarray, dtype: str) -> np.ndarray:
 
 def nan_bits(dtype: str) -> np.uint16:
     return F16_NAN if dtype == "f16" else BF16_NAN
+
+
+def io_dtype_of(dtype: str) -> str:
+    """The dtype of query/key/value rows: the cache's own for 16-bit caches,
+    fp16 for fp8 caches."""
+    return "f16" if dtype == "fp8" else dtype
 
 
 @dataclass
@@ -74,7 +88,7 @@ class DecodeStep:
     slot_mapping: np.ndarray   # int64 [S], slot of each new token
     copy_pairs: np.ndarray     # int64 [N, 2], (src, dst) to copy before writing
     valid_slots: np.ndarray    # int32 [NB], filled slots per block before the step
-    base: np.ndarray           # uint16 [R, bs*D] tile bank
+    base: np.ndarray           # uint16 [R, bs*D] tile bank (fp8: uint8 [R, tile bytes])
     layers: list = field(default_factory=list)
     ref_count: np.ndarray = None  # int64 [NB], after the step
     meta: dict = field(default_factory=dict)
@@ -82,6 +96,10 @@ class DecodeStep:
     @property
     def num_layers(self) -> int:
         return len(self.layers)
+
+    @property
+    def io_dtype(self) -> str:
+        return io_dtype_of(self.dtype)
 
     @property
     def max_blocks_per_seq(self) -> int:
@@ -94,6 +112,15 @@ class DecodeStep:
 
 def _draw_bits(rng, shape, dtype):
     return to_storage_bits(rng.standard_normal(shape, dtype=np.float32), dtype)
+
+
+def _draw_fp8_tiles(rng, rows, block_size, head_dim):
+    """fp8 tiles: codes uniform over the finite e4m3 codes (0x7F and 0xFF
+    are NaN), then one positive fp32 scale per row."""
+    codes = rng.integers(0, 254, size=(rows, block_size * head_dim), dtype=np.uint16)
+    codes = np.where(codes >= 0x7F, codes + 1, codes).astype(np.uint8)   # skip 0x7F
+    scales = rng.uniform(0.002, 0.008, size=(rows, block_size)).astype(np.float32)
+    return np.concatenate([codes, scales.view(np.uint8)], axis=1)
 
 
 def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
@@ -109,7 +136,7 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
     filled last block a second holder (a forked sibling that is not decoded),
     so appending into it triggers copy-on-write.
     """
-    if dtype not in ("f16", "bf16"):
+    if dtype not in ("f16", "bf16", "fp8"):
         raise ValueError(dtype)
     bs, H, D = int(block_size), int(num_heads), int(head_dim)
     S = len(pre_tokens)
@@ -155,7 +182,11 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
     filled = np.nonzero(valid > 0)[0]
     n_tiles = 2 * len(filled) * H
     rows = max(1, min(n_tiles, MAX_BANK_ROWS))
-    base = _draw_bits(rng, (rows, bs * D), dtype)
+    if dtype == "fp8":
+        base = _draw_fp8_tiles(rng, rows, bs, D)
+    else:
+        base = _draw_bits(rng, (rows, bs * D), dtype)
+    io = io_dtype_of(dtype)
     layers = []
     for _ in range(num_layers):
         if n_tiles <= rows:
@@ -169,9 +200,9 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
         tk[filled] = pick[0]
         tv[filled] = pick[1]
         layers.append(LayerInputs(
-            query=_draw_bits(rng, (S, H, D), dtype),
-            new_key=_draw_bits(rng, (S, H, D), dtype),
-            new_value=_draw_bits(rng, (S, H, D), dtype),
+            query=_draw_bits(rng, (S, H, D), io),
+            new_key=_draw_bits(rng, (S, H, D), io),
+            new_value=_draw_bits(rng, (S, H, D), io),
             tile_rows_k=tk, tile_rows_v=tv))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
@@ -273,9 +304,11 @@ CONFIGS = {
 
 def host_pools(step: DecodeStep, layer: int = 0):
     """Return the pre-step (key_pool, value_pool) of one layer as uint16
-    arrays [NB, H, bs, D]."""
+    arrays [NB, H, bs, D] (fp8: uint8 [NB, H, bs*D + 4*bs])."""
     bs, H, D = step.block_size, step.num_heads, step.head_dim
     L = step.layers[layer]
+    if step.dtype == "fp8":
+        return _host_pools_fp8(step, L)
     nan = nan_bits(step.dtype)
     pools = []
     for rows in (L.tile_rows_k, L.tile_rows_v):
@@ -284,6 +317,24 @@ def host_pools(step: DecodeStep, layer: int = 0):
         p[rows < 0] = nan
         mask = np.arange(bs)[None, :] >= step.valid_slots[:, None]
         p.transpose(0, 2, 1, 3)[mask] = nan
+        pools.append(p)
+    return pools[0], pools[1]
+
+
+def _host_pools_fp8(step, L):
+    bs, H, D = step.block_size, step.num_heads, step.head_dim
+    tb = fp8_tile_bytes(bs, D)
+    dead = np.arange(bs)[None, :] >= step.valid_slots[:, None]          # [NB, bs]
+    pools = []
+    for rows in (L.tile_rows_k, L.tile_rows_v):
+        p = step.base[np.maximum(rows, 0).reshape(-1)].reshape(step.num_blocks, H, tb).copy()
+        p[rows < 0] = E4M3_NAN
+        codes = p[:, :, : bs * D].reshape(step.num_blocks, H, bs, D)
+        scales = p[:, :, bs * D:].reshape(step.num_blocks, H, bs, 4)
+        codes.transpose(0, 2, 1, 3)[dead] = E4M3_NAN
+        scales.transpose(0, 2, 1, 3)[dead] = F32_NAN_BYTES
+        for b in np.nonzero((rows < 0).any(axis=1))[0]:
+            scales[b][rows[b] < 0] = F32_NAN_BYTES
         pools.append(p)
     return pools[0], pools[1]
 
@@ -324,6 +375,7 @@ def subset(step: DecodeStep, seq_ids) -> DecodeStep:
 
 def kv_bytes_read(step: DecodeStep) -> int:
     """K/V bytes one decode over every sequence of one layer must read:
-    context_len tokens x heads x head_dim x 2 (K and V) x element bytes."""
-    return int(np.sum(step.context_lens.astype(np.int64))) * step.num_heads * \
-        step.head_dim * 2 * 2
+    context_len tokens x heads x 2 (K and V) x the bytes of a row (head_dim
+    x 2 for 16-bit caches; head_dim codes + a 4-byte scale for fp8)."""
+    per_row = step.head_dim + 4 if step.dtype == "fp8" else step.head_dim * 2
+    return int(np.sum(step.context_lens.astype(np.int64))) * step.num_heads * per_row * 2
