@@ -48,28 +48,28 @@ FALLBACK_PEAK_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
 WORKLOADS = {
-    "tiny": (lambda seed: wl.tiny(seed=seed),
+    "tiny": (lambda seed, dt="f16": wl.tiny(seed=seed, dtype=dt),
              "tiny: 4 seqs, 4 heads, head_dim 64, block_size 16, ctx {1,17,33,100}, "
              "64-block pool"),
-    "llama7b_layer": (lambda seed: wl.llama_layer(seed=seed),
+    "llama7b_layer": (lambda seed, dt="f16": wl.llama_layer(seed=seed, dtype=dt),
                       "llama7b_layer: 96 seqs, 32 heads, head_dim 128, block_size 16, "
                       "ctx U[128,2048], 8192-block pool, write_kv + decode"),
-    "long_context": (lambda seed: wl.long_context(seed=seed),
+    "long_context": (lambda seed, dt="f16": wl.long_context(seed=seed, dtype=dt),
                      "long_context: 8 seqs, 32 heads, head_dim 128, block_size 16, "
                      "ctx U[16384,32768], 20000-block pool, split decode + reduce"),
-    "prefix_cow": (lambda seed: wl.prefix_cow(seed=seed),
+    "prefix_cow": (lambda seed, dt="f16": wl.prefix_cow(seed=seed, dtype=dt),
                    "prefix_cow: 64 seqs sharing a 1024-token prefix, suffix U[1,512], "
                    "32 heads, head_dim 128, copy_blocks + write_kv + decode"),
-    "full_step_bs8": (lambda seed: wl.full_step(seed=seed, block_size=8),
+    "full_step_bs8": (lambda seed, dt="f16": wl.full_step(seed=seed, block_size=8, dtype=dt),
                       "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 8"),
-    "full_step_bs16": (lambda seed: wl.full_step(seed=seed, block_size=16),
+    "full_step_bs16": (lambda seed, dt="f16": wl.full_step(seed=seed, block_size=16, dtype=dt),
                        "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 16"),
-    "full_step_bs32": (lambda seed: wl.full_step(seed=seed, block_size=32),
+    "full_step_bs32": (lambda seed, dt="f16": wl.full_step(seed=seed, block_size=32, dtype=dt),
                        "full_step: 32 layers, 256 seqs, ctx min(Geom(1/300),4096), bs 32"),
-    "swap_resume": (lambda seed: wl.llama_layer(seed=seed),
+    "swap_resume": (lambda seed, dt="f16": wl.llama_layer(seed=seed, dtype=dt),
                     "swap_resume: llama7b_layer whose every 4th sequence (24 of 96) is swapped "
                     "in from pinned host memory (pa_swap_blocks) before each decode"),
-    "small_batch_step": (lambda seed: wl.full_step(seed=seed, block_size=16, num_seqs=8),
+    "small_batch_step": (lambda seed, dt="f16": wl.full_step(seed=seed, block_size=16, num_seqs=8, dtype=dt),
                          "small_batch_step: 32 layers, 8 seqs, ctx min(Geom(1/300),4096), "
                          "bs 16 (launch-bound)"),
 }
@@ -85,7 +85,7 @@ def algorithmic_bytes(step) -> dict:
     counted."""
     H, D = step.num_heads, step.head_dim
     ctx = step.context_lens.astype(np.int64)
-    kv = int(ctx.sum()) * H * D * 2 * 2
+    kv = wl.kv_bytes_read(step)      # K and V rows (fp8: codes + a 4-byte scale per row)
     qo = step.num_seqs * H * D * 2 * 2
     table = int(np.sum(-(-ctx // step.block_size))) * 4
     return {"kv": kv, "total": kv + qo + table}
@@ -196,11 +196,7 @@ def time_oracle(sub, layers, pools):
     import oracle
     t0 = time.perf_counter()
     for li, (kc, vc) in zip(layers, pools):
-        L = sub.layers[li]
-        oracle.copy_blocks([kc], [vc], sub.copy_pairs)
-        oracle.write_kv(L.new_key, L.new_value, sub.slot_mapping, kc, vc, sub.block_size)
-        oracle.decode(L.query, kc, vc, sub.block_tables, sub.context_lens, float(sub.scale),
-                      sub.dtype)
+        oracle.default().step_on_pools(sub, li, kc, vc)
     return time.perf_counter() - t0
 
 
@@ -291,7 +287,7 @@ def job_throughput(world, seqs_per_rank, steps, max_ms):
 
 
 def run_reference(args, config_desc):
-    step = WORKLOADS[args.config][0](SEEDS[args.config])
+    step = WORKLOADS[args.config][0](SEEDS[args.config], args.kv_dtype)
     sub = oracle_sample(step, 2.0)
     layers = [0]
     pools = oracle_inputs(sub, layers)
@@ -333,6 +329,8 @@ def main():
                     help="llama7b_layer only: this many sequences (pool scaled to match), "
                          "for profiler captures on a smaller case of the same kernel")
     ap.add_argument("--soak-seconds", type=float, default=1.0)
+    ap.add_argument("--kv-dtype", default="f16", choices=["f16", "bf16", "fp8"],
+                    help="cache storage (fp8: e4m3 codes + fp32 row scales, fp16 rows)")
     ap.add_argument("--separate", action="store_true",
                     help="pa_write_kv then pa_decode instead of the fused pa_write_kv_decode")
     ap.add_argument("--no-graph", action="store_true",
@@ -378,11 +376,17 @@ def main():
         if args.config != "llama7b_layer":
             ap.error("--seqs applies to llama7b_layer only")
         step = wl.llama_layer(seed=SEEDS[args.config] + 1000 * rank, num_seqs=args.seqs,
-                              num_blocks=max(256, 8192 * args.seqs // 96))
+                              num_blocks=max(256, 8192 * args.seqs // 96), dtype=args.kv_dtype)
         config_desc["workload"] += f" (reduced to {args.seqs} seqs)"
     else:
-        step = WORKLOADS[args.config][0](SEEDS[args.config] + 1000 * rank)
+        step = WORKLOADS[args.config][0](SEEDS[args.config] + 1000 * rank, args.kv_dtype)
+    if args.kv_dtype != "f16":
+        config_desc["kv_dtype"] = args.kv_dtype
     d = device_step(step, dev)
+    if step.dtype == "fp8":
+        for key in ("key_caches", "value_caches"):
+            d[key] = [pk.Fp8Cache(t, step.block_size, step.head_dim, torch.float16)
+                      for t in d[key]]
     L, S = step.num_layers, step.num_seqs
     stream = torch.cuda.current_stream(dev)
     outs = [torch.empty_like(q) for q in d["query"]]

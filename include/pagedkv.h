@@ -17,6 +17,14 @@
  *   (fp16 or bf16), row-major. Token t of a sequence lives in physical block
  *   block_table[t / block_size] at offset t % block_size; its "slot" is
  *   block * block_size + offset.
+ * - fp8 caches (PA_FP8_E4M3; KV-cache quantisation, which "vLLM基础", §2.5
+ *   names as further tuning on top of paging): each (block, head) tile is
+ *   block_size rows of head_dim OCP e4m3 codes followed by block_size fp32
+ *   row scales, [num_blocks][num_kv_heads][block_size*head_dim + 4*block_size]
+ *   bytes; a row's values are its codes times its scale. Writes quantise a
+ *   row x as scale = amax/448, codes = e4m3(x * (448/amax)) (fp32 steps,
+ *   round to nearest even, saturating). Query, key, value and outputs are
+ *   then of the descriptor's io_dtype (PA_F16 or PA_BF16).
  * - Supported shapes: head_dim 64 or 128; block_size 8, 16 or 32;
  *   num_heads == num_kv_heads (one query head per KV head).
  * - Ownership: the caller owns every buffer, including the decode
@@ -52,16 +60,19 @@ typedef enum {
     PA_ERR_CUDA = 4         /* a CUDA launch or attribute call failed */
 } pa_status;
 
-typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 } pa_dtype;
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2, PA_FP8_E4M3 = 3 } pa_dtype;
 
-/* Shape of one layer's K (and, identically, V) cache. dtype is PA_F16 or
- * PA_BF16. */
+/* Shape of one layer's K (and, identically, V) cache. dtype is the storage:
+ * PA_F16, PA_BF16 or PA_FP8_E4M3. io_dtype is read for fp8 caches only: the
+ * type of query, key and value rows (PA_F16 or PA_BF16); 16-bit caches take
+ * rows of their own dtype. */
 typedef struct {
     int32_t num_blocks;
     int32_t block_size;
     int32_t num_kv_heads;
     int32_t head_dim;
     pa_dtype dtype;
+    pa_dtype io_dtype;
 } pa_cache_desc;
 
 /* Bits the kernels OR into *dev_err. */

@@ -205,13 +205,10 @@ class Oracle:
             raise ValueError("oracle_decode: block id or context length outside the pool")
         return out
 
-    def run_step(self, step, layer=0, threads=0):
-        """The whole step on the host for one layer of a
-        :class:`workloads.DecodeStep`: copy-on-write, write the new tokens,
-        then decode. Returns (out fp64 [S,H,D], key_pool, value_pool), the
-        pools in their post-step state."""
-        from workloads import host_pools
-        kc, vc = host_pools(step, layer)
+    def step_on_pools(self, step, layer, kc, vc, threads=0):
+        """Copy-on-write, write the new tokens, decode: one layer of a
+        :class:`workloads.DecodeStep` on the given host pools (in place).
+        Returns the fp64 output [S, H, D]."""
         L = step.layers[layer]
         if step.dtype == "fp8":
             # Whole-block copies are byte copies: view the pools as 16-bit.
@@ -220,13 +217,21 @@ class Oracle:
             self.copy_blocks([k16], [v16], step.copy_pairs)
             self.write_kv_fp8(L.new_key, L.new_value, step.slot_mapping, kc, vc,
                               step.block_size, step.io_dtype)
-            out = self.decode_fp8(L.query, kc, vc, step.block_tables, step.context_lens,
-                                  float(step.scale), step.block_size, step.io_dtype, threads)
-            return out, kc, vc
+            return self.decode_fp8(L.query, kc, vc, step.block_tables, step.context_lens,
+                                   float(step.scale), step.block_size, step.io_dtype, threads)
         self.copy_blocks([kc], [vc], step.copy_pairs)
         self.write_kv(L.new_key, L.new_value, step.slot_mapping, kc, vc, step.block_size)
-        out = self.decode(L.query, kc, vc, step.block_tables, step.context_lens,
-                          float(step.scale), step.dtype, threads)
+        return self.decode(L.query, kc, vc, step.block_tables, step.context_lens,
+                           float(step.scale), step.dtype, threads)
+
+    def run_step(self, step, layer=0, threads=0):
+        """The whole step on the host for one layer of a
+        :class:`workloads.DecodeStep`: copy-on-write, write the new tokens,
+        then decode. Returns (out fp64 [S,H,D], key_pool, value_pool), the
+        pools in their post-step state."""
+        from workloads import host_pools
+        kc, vc = host_pools(step, layer)
+        out = self.step_on_pools(step, layer, kc, vc, threads)
         return out, kc, vc
 
 

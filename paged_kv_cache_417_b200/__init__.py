@@ -27,7 +27,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = range(5)
-PA_F16, PA_BF16, PA_F32 = 0, 1, 2
+PA_F16, PA_BF16, PA_F32, PA_FP8_E4M3 = 0, 1, 2, 3
 PA_DEVERR_BLOCK_ID = 1
 PA_DEVERR_CONTEXT_LEN = 2
 PA_DEVERR_SLOT = 4
@@ -41,7 +41,52 @@ _DTYPE = {torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.float32: PA_F32}
 class CacheDesc(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("io_dtype", ctypes.c_int)]
+
+
+class Fp8Cache:
+    """An fp8 (e4m3) K or V cache: a uint8 tensor [num_blocks, num_heads,
+    block_size*head_dim + 4*block_size] whose (block, head) tiles hold
+    block_size rows of head_dim codes and then one fp32 scale per row.
+    ``io_dtype`` is the dtype of the query/key/value rows used with it."""
+
+    def __init__(self, data, block_size, head_dim, io_dtype=torch.float16):
+        if data.dtype != torch.uint8 or data.dim() != 3:
+            raise ValueError("fp8 cache data must be uint8 [num_blocks, heads, tile bytes]")
+        if data.shape[2] != block_size * head_dim + 4 * block_size:
+            raise ValueError("tile bytes must be block_size*head_dim + 4*block_size")
+        if io_dtype not in (torch.float16, torch.bfloat16):
+            raise ValueError("io_dtype must be float16 or bfloat16")
+        self.data, self.block_size, self.head_dim, self.io_dtype = data, block_size, head_dim, \
+            io_dtype
+
+    @classmethod
+    def empty(cls, num_blocks, num_heads, block_size, head_dim, io_dtype=torch.float16,
+              device="cuda"):
+        data = torch.empty(num_blocks, num_heads, block_size * head_dim + 4 * block_size,
+                           dtype=torch.uint8, device=device)
+        return cls(data, block_size, head_dim, io_dtype)
+
+    def data_ptr(self):
+        return self.data.data_ptr()
+
+    def is_contiguous(self):
+        return self.data.is_contiguous()
+
+    def is_pinned(self):
+        return self.data.is_pinned()
+
+    @property
+    def is_cuda(self):
+        return self.data.is_cuda
+
+    @property
+    def device(self):
+        return self.data.device
+
+    @property
+    def shape(self):
+        return self.data.shape
 
 
 _P = ctypes.c_void_p
@@ -99,22 +144,43 @@ def _stream(t: torch.Tensor) -> int:
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
-def cache_desc(key_cache: torch.Tensor) -> CacheDesc:
+def cache_desc(key_cache) -> CacheDesc:
+    if isinstance(key_cache, Fp8Cache):
+        nb, h, _ = key_cache.data.shape
+        return CacheDesc(nb, key_cache.block_size, h, key_cache.head_dim, PA_FP8_E4M3,
+                         _DTYPE[key_cache.io_dtype])
     if key_cache.dim() != 4:
         raise ValueError("cache must be [num_blocks, num_heads, block_size, head_dim]")
     nb, h, bs, d = key_cache.shape
     if key_cache.dtype not in (torch.float16, torch.bfloat16):
         raise ValueError("cache dtype must be float16 or bfloat16")
-    return CacheDesc(nb, bs, h, d, _DTYPE[key_cache.dtype])
+    return CacheDesc(nb, bs, h, d, _DTYPE[key_cache.dtype], _DTYPE[key_cache.dtype])
 
 
-def _need(t: torch.Tensor, name: str, dtype=None):
+def io_dtype(cache) -> torch.dtype:
+    """dtype of the query/key/value rows used with a cache."""
+    return cache.io_dtype if isinstance(cache, Fp8Cache) else cache.dtype
+
+
+def _need(t, name: str, dtype=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _need_cache(c, name: str, like=None):
+    if isinstance(c, Fp8Cache):
+        _need(c.data, name)
+        if like is not None and (not isinstance(like, Fp8Cache) or c.shape != like.shape):
+            raise ValueError(f"{name} does not match the other cache")
+        return
+    _need(c, name)
+    if like is not None and (isinstance(like, Fp8Cache) or c.dtype != like.dtype or
+                             c.shape != like.shape):
+        raise ValueError(f"{name} does not match the other cache")
 
 
 def version() -> int:
@@ -124,11 +190,12 @@ def version() -> int:
 def write_kv(key, value, slot_mapping, key_cache, value_cache, dev_err=None):
     """Store new tokens' K/V ([T, H, D]) at ``slot_mapping`` (int64 [T]) in
     the caches; negative slots are skipped."""
-    for t, n in ((key, "key"), (value, "value"), (key_cache, "key_cache"),
-                 (value_cache, "value_cache")):
-        _need(t, n, key_cache.dtype)
+    _need_cache(key_cache, "key_cache")
+    _need_cache(value_cache, "value_cache", key_cache)
+    for t, n in ((key, "key"), (value, "value")):
+        _need(t, n, io_dtype(key_cache))
     _need(slot_mapping, "slot_mapping", torch.int64)
-    if value_cache.shape != key_cache.shape or key.shape != value.shape:
+    if key.shape != value.shape:
         raise ValueError("shape mismatch")
     desc = cache_desc(key_cache)
     _check(_lib.pa_write_kv(_ptr(key), _ptr(value), key.shape[0], key.shape[1],
@@ -164,15 +231,15 @@ def decode(out, query, key_cache, value_cache, block_tables, context_lens, max_c
     """out[s,h,:] = softmax(scale * q K^T) V over each sequence's cached
     tokens. ``out`` may be fp16, bf16 or fp32; ``workspace`` is allocated
     here when not given."""
-    _need(query, "query", key_cache.dtype)
-    _need(key_cache, "key_cache")
-    _need(value_cache, "value_cache", key_cache.dtype)
+    _need_cache(key_cache, "key_cache")
+    _need_cache(value_cache, "value_cache", key_cache)
+    _need(query, "query", io_dtype(key_cache))
     _need(block_tables, "block_tables", torch.int32)
     _need(context_lens, "context_lens", torch.int32)
     _need(out, "out")
     if out.dtype not in _DTYPE:
         raise ValueError("out dtype must be float16, bfloat16 or float32")
-    if out.shape != query.shape or value_cache.shape != key_cache.shape:
+    if out.shape != query.shape:
         raise ValueError("shape mismatch")
     desc = cache_desc(key_cache)
     S, H, D = query.shape
@@ -197,18 +264,17 @@ def write_kv_decode(out, query, key, value, key_cache, value_cache, block_tables
     rows, stored at position ``context_lens[s] - 1`` of each sequence (the
     slot its block table gives), and attention covers every token including
     them."""
-    _need(query, "query", key_cache.dtype)
-    _need(key, "key", key_cache.dtype)
-    _need(value, "value", key_cache.dtype)
-    _need(key_cache, "key_cache")
-    _need(value_cache, "value_cache", key_cache.dtype)
+    _need_cache(key_cache, "key_cache")
+    _need_cache(value_cache, "value_cache", key_cache)
+    _need(query, "query", io_dtype(key_cache))
+    _need(key, "key", io_dtype(key_cache))
+    _need(value, "value", io_dtype(key_cache))
     _need(block_tables, "block_tables", torch.int32)
     _need(context_lens, "context_lens", torch.int32)
     _need(out, "out")
     if out.dtype not in _DTYPE:
         raise ValueError("out dtype must be float16, bfloat16 or float32")
-    if not (out.shape == query.shape == key.shape == value.shape) or \
-            value_cache.shape != key_cache.shape:
+    if not (out.shape == query.shape == key.shape == value.shape):
         raise ValueError("shape mismatch")
     desc = cache_desc(key_cache)
     S, H, D = query.shape
@@ -237,15 +303,15 @@ def decode_noalloc(out, query, key_cache, value_cache, block_tables, context_len
     fixed 32 MiB array inside the library instead of a workspace. Calls that
     overlap on the GPU share that array and race; the first call on a device
     looks up its address and should come before any stream capture."""
-    _need(query, "query", key_cache.dtype)
-    _need(key_cache, "key_cache")
-    _need(value_cache, "value_cache", key_cache.dtype)
+    _need_cache(key_cache, "key_cache")
+    _need_cache(value_cache, "value_cache", key_cache)
+    _need(query, "query", io_dtype(key_cache))
     _need(block_tables, "block_tables", torch.int32)
     _need(context_lens, "context_lens", torch.int32)
     _need(out, "out")
     if out.dtype not in _DTYPE:
         raise ValueError("out dtype must be float16, bfloat16 or float32")
-    if out.shape != query.shape or value_cache.shape != key_cache.shape:
+    if out.shape != query.shape:
         raise ValueError("shape mismatch")
     desc = cache_desc(key_cache)
     S, H, D = query.shape
@@ -265,9 +331,7 @@ def copy_blocks(key_caches, value_caches, block_mapping, dev_err=None):
         raise ValueError("need the same, non-zero number of K and V caches")
     _need(block_mapping, "block_mapping", torch.int64)
     for c in list(key_caches) + list(value_caches):
-        _need(c, "cache", key_caches[0].dtype)
-        if c.shape != key_caches[0].shape:
-            raise ValueError("all caches must have one shape")
+        _need_cache(c, "cache", key_caches[0])
     desc = cache_desc(key_caches[0])
     L = len(key_caches)
     kp = (_P * L)(*[c.data_ptr() for c in key_caches])

@@ -20,6 +20,10 @@
 
 #include <cstdint>
 
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "pagedkv.h"
 #include "ptx.cuh"
 
@@ -79,6 +83,85 @@ __global__ void __launch_bounds__(128) write_kv_kernel(const __grid_constant__ W
                 p.value_cache[dst] = vr[u];
             }
         }
+    }
+}
+
+// write_kv_fp8_kernel: the same write into an fp8 cache. A warp quantises
+// one (token, head) row of K and one of V: amax over the row, scale =
+// amax / 448, codes = e4m3(x * (448 / amax)) with round-to-nearest-even and
+// saturation; lane l stores codes [l*D/32, (l+1)*D/32), lane 0 the scale.
+// One CTA (4 warps) per token, warps striding over the heads.
+struct WriteFp8Params {
+    const void *key; // [T][H][D] of QT
+    const void *value;
+    const int64_t *slot_mapping;
+    uint8_t *key_cache; // [NB][H][BS*D codes + BS fp32 scales]
+    uint8_t *value_cache;
+    int32_t *dev_err;
+    int64_t num_slots;
+    int32_t num_heads, head_dim, block_size;
+};
+
+template <typename QT, int D>
+__device__ __forceinline__ void quantize_row_to(const QT *x, uint8_t *codes, float *scale,
+                                                int lane)
+{
+    constexpr int EPL = D / 32; // elements per lane
+    float v[EPL];
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        v[e] = static_cast<float>(x[lane * EPL + e]);
+        amax = fmaxf(amax, fabsf(v[e]));
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float inv = amax > 0.f ? 448.f / amax : 0.f;
+    uint32_t packed = 0;
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2) {
+        const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(
+            make_float2(v[e] * inv, v[e + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+        packed |= (uint32_t)c2 << (8 * e);
+    }
+    if constexpr (EPL == 4)
+        reinterpret_cast<uint32_t *>(codes)[lane] = packed;
+    else
+        reinterpret_cast<uint16_t *>(codes)[lane] = (uint16_t)packed;
+    if (lane == 0)
+        *scale = amax / 448.f;
+}
+
+template <typename QT, int D>
+__global__ void __launch_bounds__(128) write_kv_fp8_kernel(const __grid_constant__ WriteFp8Params p)
+{
+    pdl_launch_dependents();
+    pdl_wait_prior_grid();
+    const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t slot = p.slot_mapping[t];
+    if (slot < 0)
+        return;
+    if (slot >= p.num_slots) {
+        if (threadIdx.x == 0)
+            report(p.dev_err, PA_DEVERR_SLOT);
+        return;
+    }
+    const int64_t blk = slot / p.block_size, off = slot % p.block_size;
+    const size_t tile_bytes = (size_t)p.block_size * D + 4 * (size_t)p.block_size;
+    for (int h = warp; h < p.num_heads; h += blockDim.x >> 5) {
+        const size_t row = ((size_t)t * p.num_heads + h) * D;
+        const size_t tile = ((size_t)blk * p.num_heads + h) * tile_bytes;
+        quantize_row_to<QT, D>(static_cast<const QT *>(p.key) + row,
+                               p.key_cache + tile + (size_t)off * D,
+                               reinterpret_cast<float *>(p.key_cache + tile +
+                                                         (size_t)p.block_size * D) + off,
+                               lane);
+        quantize_row_to<QT, D>(static_cast<const QT *>(p.value) + row,
+                               p.value_cache + tile + (size_t)off * D,
+                               reinterpret_cast<float *>(p.value_cache + tile +
+                                                         (size_t)p.block_size * D) + off,
+                               lane);
     }
 }
 

@@ -40,8 +40,10 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "pagedkv.h"
 #include "ptx.cuh"
@@ -90,13 +92,137 @@ template <> struct Elem<__nv_bfloat16> {
     }
 };
 
-template <typename T>
-__device__ __forceinline__ void unpack8(const uint4 &raw, float (&f)[8])
+template <typename T> __device__ __forceinline__ void unpack8_to(const uint4 &raw, float *f)
 {
     float2 a = Elem<T>::pair(raw.x), b = Elem<T>::pair(raw.y);
     float2 c = Elem<T>::pair(raw.z), d = Elem<T>::pair(raw.w);
     f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
     f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4 &raw, float (&f)[8])
+{
+    unpack8_to<T>(raw, f);
+}
+
+// Storage tag of an fp8 cache: OCP e4m3 codes, one fp32 scale per row.
+struct E4M3 {};
+
+// Four e4m3 codes (little-endian bytes of u) to floats, through the
+// hardware fp8x2 -> f16x2 conversion.
+__device__ __forceinline__ void e4m3x4_to_float(uint32_t u, float *f)
+{
+    __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(u & 0xffffu), __NV_E4M3);
+    __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(u >> 16), __NV_E4M3);
+    __half2 a, b;
+    memcpy(&a, &lo, 4);
+    memcpy(&b, &hi, 4);
+    float2 fa = __half22float2(a), fb = __half22float2(b);
+    f[0] = fa.x; f[1] = fa.y; f[2] = fb.x; f[3] = fb.y;
+}
+
+// Mixed-precision FMAs of sm_100 (fp32 accumulator, f16 multiplicands):
+// d = c + a.lo*b.lo + a.hi*b.hi for f16 pairs a, b (the products are exact in
+// fp32), and (c0, c1) += p * (v.lo, v.hi).
+__device__ __forceinline__ float fma2_f16(uint32_t a, uint32_t b, float c)
+{
+    float d;
+    asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\t"
+        "mov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+        "fma.rn.f32.f16 %0, a0, b0, %3;\n\tfma.rn.f32.f16 %0, a1, b1, %0;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ void axpy2_f16(uint16_t p, uint32_t v, float &c0, float &c1)
+{
+    asm("{\n\t.reg .f16 v0, v1;\n\tmov.b32 {v0, v1}, %2;\n\t"
+        "fma.rn.f32.f16 %0, %3, v0, %0;\n\tfma.rn.f32.f16 %1, %3, v1, %1;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "r"(v), "h"(p));
+}
+
+// Packed fp32 FMA of sm_100: (d0, d1) = (a0*b0 + d0, a1*b1 + d1).
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rd, {%0, %1};\n\tfma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Bytes of K codes per stage for fp8 caches (16-bit caches: 4 KiB).
+#ifndef PA_FP8_STAGE_BYTES
+#define PA_FP8_STAGE_BYTES 2048
+#endif
+
+// Which arithmetic the stream uses. The macros exist for tuning sweeps.
+#ifndef PA_QK_MIXED
+#define PA_QK_MIXED 1 // q.k with fma.rn.f32.f16 for f16 caches with f16 queries
+#endif
+#ifndef PA_FFMA2
+#define PA_FFMA2 1 // packed fp32 FMAs on the fp32 (non-mixed) paths
+#endif
+#ifndef PA_PV_MIXED
+#define PA_PV_MIXED 1 // p.v with fma.rn.f32.f16 (p rounded to f16) for f16 caches
+#endif
+
+// Cached element formats. kPer16: elements per 16-byte load.
+template <typename T> struct Store {
+    static constexpr int kBytes = 2, kPer16 = 8;
+    static constexpr bool kScaled = false;
+    static __device__ __forceinline__ void unpack(const uint4 &raw, float (&f)[8])
+    {
+        unpack8<T>(raw, f);
+    }
+    // The 16 bytes as f16 pairs (meaningful for __half storage).
+    static __device__ __forceinline__ void to_h2(const uint4 &raw, uint32_t (&w)[4])
+    {
+        w[0] = raw.x; w[1] = raw.y; w[2] = raw.z; w[3] = raw.w;
+    }
+};
+template <> struct Store<E4M3> {
+    static constexpr int kBytes = 1, kPer16 = 16;
+    static constexpr bool kScaled = true;
+    static __device__ __forceinline__ void unpack(const uint4 &raw, float (&f)[16])
+    {
+        e4m3x4_to_float(raw.x, f);
+        e4m3x4_to_float(raw.y, f + 4);
+        e4m3x4_to_float(raw.z, f + 8);
+        e4m3x4_to_float(raw.w, f + 12);
+    }
+    // 16 codes as 8 f16 pairs (e4m3 values are exact in f16).
+    static __device__ __forceinline__ void to_h2(const uint4 &raw, uint32_t (&w)[8])
+    {
+        const uint32_t c[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            __half2_raw lo =
+                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(c[k] & 0xffffu), __NV_E4M3);
+            __half2_raw hi =
+                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(c[k] >> 16), __NV_E4M3);
+            w[2 * k] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
+            w[2 * k + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+        }
+    }
+};
+
+// Quantise 16 floats with a precomputed 448/amax to e4m3 codes (round to
+// nearest even, saturating at 448), packed little-endian.
+__device__ __forceinline__ uint4 quantize16_e4m3(const float (&x)[16], float inv)
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+            make_float2(x[4 * k] * inv, x[4 * k + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+            make_float2(x[4 * k + 2] * inv, x[4 * k + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+        w[k] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 __device__ __forceinline__ void store_out(void *out, int dtype, size_t idx, float v)
@@ -122,56 +248,107 @@ __device__ __forceinline__ int checked_context(const DecodeParams &p, int raw, i
     return raw;
 }
 
+// Geometry of a warp's stream for cache format T (a 16-bit type or E4M3).
+// Every lane holds 32 dims of a row, as J 16-byte pieces of E elements.
 template <typename T, int D, int BS, int NS> struct ChunkCfg {
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
+    using S = Store<T>;
+    static constexpr int kE = S::kPer16;                   // elements per 16 bytes
+    static constexpr int kJ = 32 / kE;                     // 16-byte pieces per lane and row
     static constexpr int kLPR = D / 32;                    // lanes per row
     static constexpr int kRPS = 32 / kLPR;                 // rows per warp step
     static constexpr int kQR = 8 / kLPR;                   // rows per quarter-warp
-    static constexpr int kChunk = 4096 / (D * 2);          // tokens per stage (4 KiB of K)
+    static constexpr int kRow = D * S::kBytes;             // bytes of a cached row
+    static constexpr int kRow16 = kRow / 16;
+    static constexpr int kChunk = (S::kScaled ? PA_FP8_STAGE_BYTES : 4096) / kRow; // rows per stage
     static constexpr int kSteps = kChunk / kRPS;
     static constexpr int kSeg = BS < kChunk ? BS : kChunk; // rows per bulk copy
-    static constexpr int kTile = kChunk * D;               // elements of K (or V) per stage
-    static constexpr int kRingBytes = NS * 2 * kTile * 2;  // one warp's stages
+    static constexpr int kTileBytes = BS * kRow + (S::kScaled ? 4 * BS : 0); // (block, head)
+    static constexpr int kData = kChunk * kRow;            // K (or V) codes of a stage
+    static constexpr int kScales = S::kScaled ? 4 * kChunk : 0;
+    static constexpr int kStage = 2 * (kData + kScales);
+    static constexpr int kRingBytes = NS * kStage;         // one warp's stages
     static_assert(kSteps >= 1 && kChunk % kRPS == 0, "chunk geometry");
+    static_assert((kRow16 % 8 == 0 && kQR <= kJ) || (kRow16 == 4 && kJ == 2 && kQR == 4),
+                  "swizzle");
+    static_assert(kChunk % 4 == 0, "scale copies start 16-byte aligned");
+    static_assert(kTileBytes % 16 == 0 && kData % 16 == 0 && kScales % 16 == 0, "alignment");
 };
 
 // One warp's online-softmax state over the chunks it streamed. After
-// finish(), the lanes with r == 0 (lane < D/32) hold the warp's sums for
-// dims (qd + LPR*j)*8 + e, j < 4, e < 8; every lane holds m and l.
-template <typename T, int D, int BS, int NS> struct WarpStream {
+// finish(), lanes with r == 0 (lane < D/32) hold the warp's sums for dims
+// (qd + LPR*j)*E + e, j < J, e < E; every lane holds m and l.
+template <typename T, typename QT, int D, int BS, int NS> struct WarpStream {
     using C = ChunkCfg<T, D, BS, NS>;
+    using S = typename C::S;
     static constexpr int LPR = C::kLPR, RPS = C::kRPS, QR = C::kQR, CHUNK = C::kChunk;
-    static constexpr int STEPS = C::kSteps, TILE = C::kTile;
+    static constexpr int STEPS = C::kSteps, E = C::kE, J = C::kJ, ROW = C::kRow;
+    static constexpr int DATA = C::kData, SCL = C::kScales, STAGE = C::kStage;
     static constexpr unsigned FULL = 0xffffffffu;
+    // q.k on raw f16 query pairs with mixed FMAs, the scale applied per row;
+    // else on fp32 copies of the query pre-scaled by scale*log2(e).
+    static constexpr bool kQKMixed =
+        PA_QK_MIXED && std::is_same<QT, __half>::value && std::is_same<T, __half>::value;
+    static constexpr bool kPVMixed = PA_PV_MIXED && std::is_same<T, __half>::value;
 
-    float qf[4][8];
-    float acc[4][8];
+    float qf[kQKMixed ? 1 : J][kQKMixed ? 1 : E];
+    uint32_t qh[kQKMixed ? J : 1][kQKMixed ? E / 2 : 1];
+    float qscale;
+    float acc[J][E];
     float m, l;
     int qd, r, rx, lane;
     int bad_id; // lane 0: a block id outside the pool was met
     // Fused append: local chunk patch_i holds the new token at row
-    // patch_row. Lanes < 2*D/8 carry 16 bytes of its K (then V) row in
-    // patch_val, which replace that row in shared memory once the chunk has
-    // landed and go to the cache at patch_dst (NULL: the block id was bad).
+    // patch_row. Lanes < 2*ROW/16 carry 16 bytes of its K (then V) row in
+    // patch_val (fp8: codes, plus the row scale in patch_scale on the first
+    // lane of each half), which replace that row in shared memory once the
+    // chunk has landed and go to the cache at patch_dst / patch_sdst (NULL:
+    // the block id was bad).
     int patch_i, patch_row;
     uint4 patch_val;
+    float patch_scale;
     uint4 *patch_dst;
+    float *patch_sdst;
 
-    __device__ __forceinline__ void init(const T *q, float qk_scale_log2, int lane_)
+    // XOR key of the 16-byte piece a lane of row r reads in slot j, chosen
+    // so the 8 lanes of a quarter-warp hit 8 distinct bank groups.
+    static __device__ __forceinline__ int swizzle_key(int row)
+    {
+        if constexpr (C::kRow16 % 8 == 0)
+            return row & (QR - 1);
+        else
+            return (row >> 1) & (J - 1);
+    }
+
+    __device__ __forceinline__ void init(const QT *q, float qk_scale_log2, int lane_)
     {
         lane = lane_;
         qd = lane % LPR;
         r = lane / LPR;
-        rx = r & (QR - 1);
+        rx = swizzle_key(r);
+        qscale = qk_scale_log2;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < J; ++j) {
             const int u = qd + LPR * (j ^ rx);
-            unpack8<T>(*reinterpret_cast<const uint4 *>(q + u * 8), qf[j]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                qf[j][e] *= qk_scale_log2;
-                acc[j][e] = 0.f;
+            for (int h8 = 0; h8 < E / 8; ++h8) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(q + u * E + h8 * 8);
+                if constexpr (kQKMixed) {
+                    qh[j][h8 * 4 + 0] = raw.x;
+                    qh[j][h8 * 4 + 1] = raw.y;
+                    qh[j][h8 * 4 + 2] = raw.z;
+                    qh[j][h8 * 4 + 3] = raw.w;
+                } else {
+                    float t[8];
+                    unpack8<QT>(raw, t);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        qf[j][h8 * 8 + e] = t[e] * qk_scale_log2;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc[j][h8 * 8 + e] = 0.f;
             }
         }
         m = -INFINITY;
@@ -179,27 +356,36 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
         bad_id = 0;
         patch_i = -1;
         patch_row = 0;
+        patch_scale = 0.f;
         patch_dst = nullptr;
+        patch_sdst = nullptr;
     }
 
     // Stream chunks c0, c0 + cstride, ... (count of them) of a unit with
-    // n_tok tokens whose block ids are table[0..]. Lane 0 issues the copies;
-    // an id outside [0, num_blocks) is replaced by block 0 and sets bad_id.
-    // Returns false if a wait ran out of time (the copies in flight have been
-    // waited for, boundedly, before returning).
-    __device__ __forceinline__ bool run(const T *kc, const T *vc, size_t head_off,
-                                        size_t block_elems, int num_blocks,
+    // n_tok tokens whose block ids are table[0..]. kc/vc are the pools'
+    // bytes; a block's tile for this head starts at b * block_bytes +
+    // head_off. Lane 0 issues the copies; an id outside [0, num_blocks) is
+    // replaced by block 0 and sets bad_id. Returns false if a wait ran out of
+    // time (the copies in flight have been waited for, boundedly, before
+    // returning).
+    __device__ __forceinline__ bool run(const char *kc, const char *vc, size_t head_off,
+                                        size_t block_bytes, int num_blocks,
                                         const int32_t *table, int n_tok, int c0, int cstride,
-                                        int count, T *ring, uint32_t bar0)
+                                        int count, char *ring, uint32_t bar0)
     {
         auto issue = [&](int i) {
             const int tok0 = (c0 + i * cstride) * CHUNK;
             const int rows = min(CHUNK, n_tok - tok0);
             const int st = i % NS;
-            T *dk = ring + st * 2 * TILE;
-            T *dv = dk + TILE;
+            char *dk = ring + st * STAGE;
+            char *dks = dk + DATA;
+            char *dv = dks + SCL;
+            char *dvs = dv + DATA;
             const uint32_t bar = bar0 + st * 8;
-            mbar_arrive_expect_tx(bar, 2u * rows * D * sizeof(T));
+            uint32_t tx = 2u * rows * ROW;
+            if constexpr (S::kScaled) // one 4-byte scale per row, copied 16 bytes at a time
+                tx += 2u * ((rows / C::kSeg) * C::kSeg + ((rows % C::kSeg + 3) & ~3)) * 4u;
+            mbar_arrive_expect_tx(bar, tx);
             for (int r0 = 0; r0 < rows; r0 += C::kSeg) {
                 const int tok = tok0 + r0;
                 int b = table[tok / BS];
@@ -207,10 +393,17 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
                     bad_id = 1;
                     b = 0;
                 }
-                const size_t src = (size_t)b * block_elems + head_off + (size_t)(tok % BS) * D;
-                const uint32_t bytes = (uint32_t)(min(C::kSeg, rows - r0) * D * sizeof(T));
-                bulk_g2s(smem_addr(dk + r0 * D), kc + src, bytes, bar);
-                bulk_g2s(smem_addr(dv + r0 * D), vc + src, bytes, bar);
+                const int rb = min(C::kSeg, rows - r0);
+                const size_t tile = (size_t)b * block_bytes + head_off;
+                const size_t src = tile + (size_t)(tok % BS) * ROW;
+                bulk_g2s(smem_addr(dk + r0 * ROW), kc + src, (uint32_t)(rb * ROW), bar);
+                bulk_g2s(smem_addr(dv + r0 * ROW), vc + src, (uint32_t)(rb * ROW), bar);
+                if constexpr (S::kScaled) {
+                    const size_t ssrc = tile + (size_t)BS * ROW + (size_t)(tok % BS) * 4;
+                    const uint32_t sb = (uint32_t)((rb + 3) & ~3) * 4u;
+                    bulk_g2s(smem_addr(dks + r0 * 4), kc + ssrc, sb, bar);
+                    bulk_g2s(smem_addr(dvs + r0 * 4), vc + ssrc, sb, bar);
+                }
             }
         };
 
@@ -225,15 +418,24 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
             if (__any_sync(FULL, !ok))
                 break;
             const int rows = min(CHUNK, n_tok - (c0 + i * cstride) * CHUNK);
-            T *sk = ring + st * 2 * TILE;
-            T *sv = sk + TILE;
+            char *sk = ring + st * STAGE;
+            const float *sks = reinterpret_cast<const float *>(sk + DATA);
+            char *sv = sk + DATA + SCL;
+            const float *svs = reinterpret_cast<const float *>(sv + DATA);
             if (i == patch_i) { // warp-uniform
-                constexpr int RV = D * 2 / 16;
+                constexpr int RV = ROW / 16;
                 if (lane < 2 * RV) {
-                    T *srow = (lane >= RV ? sv : sk) + patch_row * D;
-                    reinterpret_cast<uint4 *>(srow)[lane % RV] = patch_val;
+                    char *base = lane >= RV ? sv : sk;
+                    reinterpret_cast<uint4 *>(base + patch_row * ROW)[lane % RV] = patch_val;
                     if (patch_dst)
                         *patch_dst = patch_val;
+                    if constexpr (S::kScaled) {
+                        if (lane % RV == 0) {
+                            reinterpret_cast<float *>(base + DATA)[patch_row] = patch_scale;
+                            if (patch_sdst)
+                                *patch_sdst = patch_scale;
+                        }
+                    }
                     fence_proxy_async_smem(); // before the stage is refilled by a bulk copy
                 }
                 __syncwarp();
@@ -243,20 +445,41 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
 #pragma unroll
             for (int t = 0; t < STEPS; ++t) {
                 const int row = t * RPS + r;
-                const T *kr = sk + row * D;
+                const char *kr = sk + row * ROW;
                 float dot = 0.f;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float kf[8];
-                    unpack8<T>(*reinterpret_cast<const uint4 *>(kr + (qd + LPR * (j ^ rx)) * 8),
-                               kf);
+                for (int j = 0; j < J; ++j) {
+                    const uint4 raw =
+                        *reinterpret_cast<const uint4 *>(kr + (qd + LPR * (j ^ rx)) * 16);
+                    if constexpr (kQKMixed) {
+                        uint32_t kh[E / 2];
+                        S::to_h2(raw, kh);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        dot = fmaf(qf[j][e], kf[e], dot);
+                        for (int w = 0; w < E / 2; ++w)
+                            dot = fma2_f16(qh[j][w], kh[w], dot);
+                    } else {
+                        float kf[E];
+                        S::unpack(raw, kf);
+                        if constexpr (PA_FFMA2) {
+                            float d1 = 0.f;
+#pragma unroll
+                            for (int e = 0; e < E; e += 2)
+                                ffma2(dot, d1, qf[j][e], qf[j][e + 1], kf[e], kf[e + 1]);
+                            dot += d1;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < E; ++e)
+                                dot = fmaf(qf[j][e], kf[e], dot);
+                        }
+                    }
                 }
 #pragma unroll
                 for (int o = 1; o < LPR; o <<= 1)
                     dot += __shfl_xor_sync(FULL, dot, o);
+                if constexpr (kQKMixed)
+                    dot *= qscale;
+                if constexpr (S::kScaled)
+                    dot *= sks[row];
                 sc[t] = row < rows ? dot : -INFINITY;
             }
             float cm = sc[0];
@@ -271,9 +494,9 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
             m = m_new;
             l *= corr;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < J; ++j)
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
+                for (int e = 0; e < E; ++e)
                     acc[j][e] *= corr;
 #pragma unroll
             for (int t = 0; t < STEPS; ++t) {
@@ -281,15 +504,39 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
                 const float pt = exp2f(sc[t] - m_new);
                 l += pt;
                 if (row < rows) {
-                    const T *vr = sv + row * D;
+                    const char *vr = sv + row * ROW;
+                    float pv = pt;
+                    if constexpr (S::kScaled)
+                        pv *= svs[row];
+                    if constexpr (kPVMixed) {
+                        const uint16_t ph = __half_as_ushort(__float2half_rn(pv));
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float vf[8];
-                        unpack8<T>(
-                            *reinterpret_cast<const uint4 *>(vr + (qd + LPR * (j ^ rx)) * 8), vf);
+                        for (int j = 0; j < J; ++j) {
+                            uint32_t vh[E / 2];
+                            S::to_h2(*reinterpret_cast<const uint4 *>(
+                                         vr + (qd + LPR * (j ^ rx)) * 16),
+                                     vh);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            acc[j][e] = fmaf(pt, vf[e], acc[j][e]);
+                            for (int w = 0; w < E / 2; ++w)
+                                axpy2_f16(ph, vh[w], acc[j][2 * w], acc[j][2 * w + 1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < J; ++j) {
+                            float vf[E];
+                            S::unpack(*reinterpret_cast<const uint4 *>(
+                                          vr + (qd + LPR * (j ^ rx)) * 16),
+                                      vf);
+                            if constexpr (PA_FFMA2) {
+#pragma unroll
+                                for (int e = 0; e < E; e += 2)
+                                    ffma2(acc[j][e], acc[j][e + 1], pv, pv, vf[e], vf[e + 1]);
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < E; ++e)
+                                    acc[j][e] = fmaf(pv, vf[e], acc[j][e]);
+                            }
+                        }
                     }
                 }
             }
@@ -310,31 +557,35 @@ template <typename T, int D, int BS, int NS> struct WarpStream {
         return true;
     }
 
-    // Put the swizzled slots back in order (slot j <- sub-chunk qd + LPR*j)
-    // and sum acc and l over the rows the warp's lanes covered.
+    // Put the swizzled slots back in order (slot j <- piece qd + LPR*j) and
+    // sum acc and l over the rows the warp's lanes covered.
     __device__ __forceinline__ void finish()
     {
         if (rx & 1) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float t0 = acc[0][e]; acc[0][e] = acc[1][e]; acc[1][e] = t0;
-                float t2 = acc[2][e]; acc[2][e] = acc[3][e]; acc[3][e] = t2;
-            }
-        }
-        if (rx & 2) {
+            for (int j = 0; j < J; j += 2)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float t0 = acc[0][e]; acc[0][e] = acc[2][e]; acc[2][e] = t0;
-                float t1 = acc[1][e]; acc[1][e] = acc[3][e]; acc[3][e] = t1;
+                for (int e = 0; e < E; ++e) {
+                    float t0 = acc[j][e]; acc[j][e] = acc[j + 1][e]; acc[j + 1][e] = t0;
+                }
+        }
+        if constexpr (J >= 4) {
+            if (rx & 2) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        float t0 = acc[j][e]; acc[j][e] = acc[j + 2][e]; acc[j + 2][e] = t0;
+                    }
             }
         }
 #pragma unroll
         for (int o = LPR; o < 32; o <<= 1) {
             l += __shfl_xor_sync(FULL, l, o);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < J; ++j)
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
+                for (int e = 0; e < E; ++e)
                     acc[j][e] += __shfl_xor_sync(FULL, acc[j][e], o);
         }
     }
@@ -380,15 +631,18 @@ template <typename T, int D, int BS, int NW, int NS> struct SplitCfg {
     }
 };
 
-template <typename T, int D, int BS, int NW, int NS>
+// T: cache format (__half, __nv_bfloat16 or E4M3); QT: query / new-row /
+// output-element type (T itself for 16-bit caches).
+template <typename T, typename QT, int D, int BS, int NW, int NS>
 __global__ void __launch_bounds__(NW * 32)
     decode_split_kernel(const __grid_constant__ DecodeParams p)
 {
-    using W = WarpStream<T, D, BS, NS>;
+    using W = WarpStream<T, QT, D, BS, NS>;
     using Cfg = SplitCfg<T, D, BS, NW, NS>;
-    constexpr int LPR = W::LPR;
+    constexpr int LPR = W::LPR, E = W::E, J = W::J, ROW = W::ROW;
+    constexpr int TILE = W::C::kTileBytes;
     extern __shared__ __align__(128) unsigned char smem[];
-    T *rings = reinterpret_cast<T *>(smem);
+    char *rings = reinterpret_cast<char *>(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kRingsBytes);
     float *merge = reinterpret_cast<float *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes);
     int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
@@ -416,39 +670,65 @@ __global__ void __launch_bounds__(NW * 32)
     __syncthreads();
 
     W ws;
-    ws.init(static_cast<const T *>(p.query) + ((size_t)s * H + h) * D, p.qk_scale_log2, lane);
+    ws.init(static_cast<const QT *>(p.query) + ((size_t)s * H + h) * D, p.qk_scale_log2, lane);
     const int n_chunks = (u.n_tok + W::CHUNK - 1) / W::CHUNK;
     const int my_chunks = n_chunks <= warp ? 0 : (n_chunks - warp + NW - 1) / NW;
     if (p.new_key != nullptr && part == u.num_parts - 1 && u.n_tok > 0) {
         // This CTA holds the sequence's last token: the warp owning its
         // chunk puts the new K/V row in place (shared memory and cache).
         const int c_last = (u.n_tok - 1) / W::CHUNK;
-        if (c_last % NW == warp) {
-            constexpr int RV = D * 2 / 16;
+        if (c_last % NW == warp) { // warp-uniform
+            constexpr int RV = ROW / 16; // lanes per cached row: K on lanes [0, RV), V after
             ws.patch_i = c_last / NW;
             ws.patch_row = (u.n_tok - 1) - c_last * W::CHUNK;
+            const bool isv = lane >= RV;
+            const int piece = lane % RV;
+            const QT *src = static_cast<const QT *>(isv ? p.new_value : p.new_key) +
+                            ((size_t)s * H + h) * D + (size_t)piece * E;
+            if constexpr (Store<T>::kScaled) {
+                // Quantise the new row: amax over its D inputs, then
+                // codes = e4m3(x * (448 / amax)) and scale = amax / 448.
+                float x[16];
+                float amax = 0.f;
+                if (lane < 2 * RV) {
+                    unpack8_to<QT>(*reinterpret_cast<const uint4 *>(src), x);
+                    unpack8_to<QT>(*reinterpret_cast<const uint4 *>(src + 8), x + 8);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        amax = fmaxf(amax, fabsf(x[e]));
+                }
+#pragma unroll
+                for (int o = 1; o < RV; o <<= 1)
+                    amax = fmaxf(amax, __shfl_xor_sync(W::FULL, amax, o));
+                if (lane < 2 * RV) {
+                    const float inv = amax > 0.f ? 448.f / amax : 0.f;
+                    ws.patch_val = quantize16_e4m3(x, inv);
+                    ws.patch_scale = amax / 448.f;
+                }
+            } else {
+                if (lane < 2 * RV)
+                    ws.patch_val = *reinterpret_cast<const uint4 *>(src);
+            }
             if (lane < 2 * RV) {
-                const bool isv = lane >= RV;
-                const int e = lane % RV;
-                ws.patch_val = reinterpret_cast<const uint4 *>(isv ? p.new_value : p.new_key)
-                    [((size_t)s * H + h) * RV + e];
                 const int b = table[(u.n_tok - 1) / BS];
                 if (b >= 0 && b < p.num_blocks) {
-                    T *cache = const_cast<T *>(
-                        static_cast<const T *>(isv ? p.value_cache : p.key_cache));
-                    ws.patch_dst = reinterpret_cast<uint4 *>(
-                                       cache + (size_t)b * H * BS * D + (size_t)h * BS * D +
-                                       (size_t)((u.n_tok - 1) % BS) * D) +
-                                   e;
+                    char *cache =
+                        const_cast<char *>(static_cast<const char *>(isv ? p.value_cache
+                                                                           : p.key_cache));
+                    char *tile = cache + ((size_t)b * H + h) * TILE;
+                    const int off = (u.n_tok - 1) % BS;
+                    ws.patch_dst = reinterpret_cast<uint4 *>(tile + (size_t)off * ROW) + piece;
+                    if (Store<T>::kScaled && piece == 0)
+                        ws.patch_sdst =
+                            reinterpret_cast<float *>(tile + (size_t)BS * ROW) + off;
                 }
             }
         }
     }
-    const bool ok = ws.run(static_cast<const T *>(p.key_cache),
-                           static_cast<const T *>(p.value_cache), (size_t)h * BS * D,
-                           (size_t)H * BS * D, p.num_blocks, table, u.n_tok, warp, NW,
-                           my_chunks, rings + (size_t)warp * NS * 2 * W::TILE,
-                           smem_addr(&bars[warp * NS]));
+    const bool ok = ws.run(static_cast<const char *>(p.key_cache),
+                           static_cast<const char *>(p.value_cache), (size_t)h * TILE,
+                           (size_t)H * TILE, p.num_blocks, table, u.n_tok, warp, NW, my_chunks,
+                           rings + (size_t)warp * W::C::kRingBytes, smem_addr(&bars[warp * NS]));
     if (lane == 0) {
         if (!ok) {
             report(p.dev_err, PA_DEVERR_TIMEOUT);
@@ -461,10 +741,10 @@ __global__ void __launch_bounds__(NW * 32)
     float *mw = merge + warp * (D + 2);
     if (lane < LPR) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < J; ++j)
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                mw[(ws.qd + LPR * j) * 8 + e] = ws.acc[j][e];
+            for (int e = 0; e < E; ++e)
+                mw[(ws.qd + LPR * j) * E + e] = ws.acc[j][e];
     }
     if (lane == 0) {
         mw[D] = ws.m;

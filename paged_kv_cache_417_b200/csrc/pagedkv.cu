@@ -67,14 +67,27 @@ pa_status check_cache(const pa_cache_desc *c)
         return fail(PA_ERR_INVALID_ARG, "cache descriptor is NULL");
     if (c->num_blocks < 0 || c->block_size <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0)
         return fail(PA_ERR_INVALID_ARG, "cache descriptor has a non-positive size");
-    if (c->dtype != PA_F16 && c->dtype != PA_BF16)
-        return fail(PA_ERR_UNSUPPORTED, "cache dtype %d (need PA_F16 or PA_BF16)", (int)c->dtype);
+    if (c->dtype != PA_F16 && c->dtype != PA_BF16 && c->dtype != PA_FP8_E4M3)
+        return fail(PA_ERR_UNSUPPORTED, "cache dtype %d (need PA_F16, PA_BF16 or PA_FP8_E4M3)",
+                    (int)c->dtype);
+    if (c->dtype == PA_FP8_E4M3 && c->io_dtype != PA_F16 && c->io_dtype != PA_BF16)
+        return fail(PA_ERR_UNSUPPORTED, "fp8 cache io_dtype %d (need PA_F16 or PA_BF16)",
+                    (int)c->io_dtype);
     if (c->head_dim != 64 && c->head_dim != 128)
         return fail(PA_ERR_UNSUPPORTED, "head_dim %d (built: 64, 128)", c->head_dim);
     if (c->block_size != 8 && c->block_size != 16 && c->block_size != 32)
         return fail(PA_ERR_UNSUPPORTED, "block_size %d (built: 8, 16, 32)", c->block_size);
     return PA_OK;
 }
+
+// Bytes of one (block, head) tile and of one block (all heads).
+size_t tile_bytes(const pa_cache_desc *c)
+{
+    const size_t rows = (size_t)c->block_size;
+    return c->dtype == PA_FP8_E4M3 ? rows * c->head_dim + 4 * rows : rows * c->head_dim * 2;
+}
+
+size_t block_bytes(const pa_cache_desc *c) { return tile_bytes(c) * (size_t)c->num_kv_heads; }
 
 // Partition (tokens per work unit) for a decode; >= max_context_len means a
 // single pass. Automatic choice: 2048 tokens, halved (down to 128) while the
@@ -160,11 +173,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <typename T, int D, int BS>
+template <typename T, typename QT, int D, int BS>
 pa_status launch_decode(const DecodeParams &p, cudaStream_t stream)
 {
     using Cfg = SplitCfg<T, D, BS, kSplitWarps, kSplitStages>;
-    auto kernel = decode_split_kernel<T, D, BS, kSplitWarps, kSplitStages>;
+    auto kernel = decode_split_kernel<T, QT, D, BS, kSplitWarps, kSplitStages>;
     static std::atomic<size_t> smem_set[kMaxDevices];
     cudaError_t e = allow_smem(kernel, Cfg::smem_bytes(kMaxPartition), smem_set);
     if (e != cudaSuccess)
@@ -182,21 +195,34 @@ pa_status launch_decode(const DecodeParams &p, cudaStream_t stream)
     return ok();
 }
 
-template <typename T, int D> pa_status dispatch_bs(const DecodeParams &p, int bs, cudaStream_t st)
+template <typename T, typename QT, int D>
+pa_status dispatch_bs(const DecodeParams &p, int bs, cudaStream_t st)
 {
     switch (bs) {
-    case 8: return launch_decode<T, D, 8>(p, st);
-    case 16: return launch_decode<T, D, 16>(p, st);
-    case 32: return launch_decode<T, D, 32>(p, st);
+    case 8: return launch_decode<T, QT, D, 8>(p, st);
+    case 16: return launch_decode<T, QT, D, 16>(p, st);
+    case 32: return launch_decode<T, QT, D, 32>(p, st);
     }
     return fail(PA_ERR_UNSUPPORTED, "block_size %d", bs);
 }
 
-template <typename T> pa_status dispatch_d(const DecodeParams &p, int d, int bs, cudaStream_t st)
+template <typename T, typename QT>
+pa_status dispatch_d(const DecodeParams &p, int d, int bs, cudaStream_t st)
 {
     if (d == 64)
-        return dispatch_bs<T, 64>(p, bs, st);
-    return dispatch_bs<T, 128>(p, bs, st);
+        return dispatch_bs<T, QT, 64>(p, bs, st);
+    return dispatch_bs<T, QT, 128>(p, bs, st);
+}
+
+pa_status dispatch_decode(const DecodeParams &p, const pa_cache_desc *c, cudaStream_t st)
+{
+    if (c->dtype == PA_F16)
+        return dispatch_d<__half, __half>(p, c->head_dim, c->block_size, st);
+    if (c->dtype == PA_BF16)
+        return dispatch_d<__nv_bfloat16, __nv_bfloat16>(p, c->head_dim, c->block_size, st);
+    if (c->io_dtype == PA_F16)
+        return dispatch_d<E4M3, __half>(p, c->head_dim, c->block_size, st);
+    return dispatch_d<E4M3, __nv_bfloat16>(p, c->head_dim, c->block_size, st);
 }
 
 } // namespace
@@ -235,6 +261,31 @@ pa_status pa_write_kv(const void *key, const void *value, int32_t num_tokens, in
         return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
     if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
         return fail(PA_ERR_INVALID_ARG, "key, value and caches must be 16-byte aligned");
+    if (cache->dtype == PA_FP8_E4M3) {
+        WriteFp8Params q;
+        q.key = key;
+        q.value = value;
+        q.slot_mapping = slot_mapping;
+        q.key_cache = static_cast<uint8_t *>(key_cache);
+        q.value_cache = static_cast<uint8_t *>(value_cache);
+        q.dev_err = dev_err;
+        q.num_slots = (int64_t)cache->num_blocks * cache->block_size;
+        q.num_heads = num_heads;
+        q.head_dim = cache->head_dim;
+        q.block_size = cache->block_size;
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        const bool f16 = cache->io_dtype == PA_F16;
+        cudaError_t e;
+        if (cache->head_dim == 64)
+            e = f16 ? launch_pdl(write_kv_fp8_kernel<__half, 64>, dim3(num_tokens), dim3(128), 0, st, q)
+                    : launch_pdl(write_kv_fp8_kernel<__nv_bfloat16, 64>, dim3(num_tokens), dim3(128), 0, st, q);
+        else
+            e = f16 ? launch_pdl(write_kv_fp8_kernel<__half, 128>, dim3(num_tokens), dim3(128), 0, st, q)
+                    : launch_pdl(write_kv_fp8_kernel<__nv_bfloat16, 128>, dim3(num_tokens), dim3(128), 0, st, q);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "write_kv launch");
+        return ok();
+    }
     WriteParams p;
     p.key = static_cast<const uint4 *>(key);
     p.value = static_cast<const uint4 *>(value);
@@ -358,10 +409,7 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
         p.ws_acc = static_cast<float *>(workspace);
         p.ws_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) + (acc + 255) / 256 * 256);
     }
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cache->dtype == PA_F16)
-        return dispatch_d<__half>(p, cache->head_dim, cache->block_size, st);
-    return dispatch_d<__nv_bfloat16>(p, cache->head_dim, cache->block_size, st);
+    return dispatch_decode(p, cache, static_cast<cudaStream_t>(stream));
 }
 
 } // namespace
@@ -425,7 +473,7 @@ pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches, int
         p.key_caches[l] = p.value_caches[l] = nullptr;
     p.block_mapping = block_mapping;
     p.dev_err = dev_err;
-    p.block_vecs = (int64_t)cache->num_kv_heads * cache->block_size * cache->head_dim * 2 / 16;
+    p.block_vecs = (int64_t)(block_bytes(cache) / 16);
     p.num_blocks = cache->num_blocks;
     cudaError_t e = launch_pdl(copy_blocks_kernel, dim3(num_pairs, num_layers, 2), dim3(256), 0,
                                static_cast<cudaStream_t>(stream), p);
@@ -469,7 +517,8 @@ pa_status pa_swap_blocks(void *const *src_key_caches, void *const *src_value_cac
     if ((s = check_cache(dst)) != PA_OK)
         return s;
     if (src->block_size != dst->block_size || src->num_kv_heads != dst->num_kv_heads ||
-        src->head_dim != dst->head_dim || src->dtype != dst->dtype)
+        src->head_dim != dst->head_dim || src->dtype != dst->dtype ||
+        block_bytes(src) != block_bytes(dst))
         return fail(PA_ERR_INVALID_ARG, "source and destination pools differ in block shape");
     if (num_pairs < 0)
         return fail(PA_ERR_INVALID_ARG, "num_pairs %d < 0", num_pairs);
@@ -508,7 +557,7 @@ pa_status pa_swap_blocks(void *const *src_key_caches, void *const *src_value_cac
         p.dst_k[l] = p.dst_v[l] = nullptr;
     }
     p.dev_err = dev_err;
-    p.block_vecs = (int64_t)src->num_kv_heads * src->block_size * src->head_dim * 2 / 16;
+    p.block_vecs = (int64_t)(block_bytes(src) / 16);
     p.src_blocks = src->num_blocks;
     p.dst_blocks = dst->num_blocks;
     cudaError_t e = launch_pdl(swap_blocks_kernel, dim3(num_pairs, num_layers, 2), dim3(256), 0,

@@ -10,8 +10,20 @@ from workloads.device import device_step
 TOL = 2e-3  # max |gpu - oracle| for fp16 output, fp32 accumulation
 
 
-def to_bits(t: torch.Tensor) -> np.ndarray:
+def to_bits(t) -> np.ndarray:
+    """Raw storage of a cache or tensor: uint16 patterns, or bytes for fp8."""
+    if isinstance(t, pk.Fp8Cache):
+        return t.data.detach().cpu().numpy()
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def wrap_caches(step, d):
+    """fp8 pools come from device_step as uint8 tensors: wrap them."""
+    if step.dtype == "fp8":
+        for key in ("key_caches", "value_caches"):
+            d[key] = [pk.Fp8Cache(t, step.block_size, step.head_dim, torch.float16)
+                      for t in d[key]]
+    return d
 
 
 def to_f64(t: torch.Tensor) -> np.ndarray:
@@ -22,7 +34,7 @@ def run_step(step, layers=None, partition_size=0, out_dtype=None, keep_pre=False
     """copy_blocks (all layers) -> per layer write_kv, decode. Returns
     (outs list, device dict, dev_err int)."""
     layers = list(range(step.num_layers)) if layers is None else list(layers)
-    d = device_step(step, "cuda", layers)
+    d = wrap_caches(step, device_step(step, "cuda", layers))
     if keep_pre:
         d["pre_key"] = [k.clone() for k in d["key_caches"]]
         d["pre_value"] = [v.clone() for v in d["value_caches"]]
@@ -71,7 +83,7 @@ def decode_case(c, partition_size=0, out_dtype=None, max_context_len=None):
 def run_step_fused(step, layers=None, partition_size=0, out_dtype=None):
     """copy_blocks (all layers) -> per layer write_kv_decode (one launch)."""
     layers = list(range(step.num_layers)) if layers is None else list(layers)
-    d = device_step(step, "cuda", layers)
+    d = wrap_caches(step, device_step(step, "cuda", layers))
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     if step.copy_pairs.shape[0]:
         pk.copy_blocks(d["key_caches"], d["value_caches"], d["copy_pairs"], dev_err=err)
