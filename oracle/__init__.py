@@ -57,8 +57,9 @@ class Oracle:
         P = ctypes.c_void_p
         L.oracle_decode.restype = ctypes.c_int
         L.oracle_decode.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
-                                    P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int,
-                                    P, ctypes.c_int32, P, ctypes.c_double, ctypes.c_int]
+                                    ctypes.c_int32, P, P, ctypes.c_int64, ctypes.c_int32,
+                                    ctypes.c_int, P, ctypes.c_int32, P, ctypes.c_double,
+                                    ctypes.c_int]
         L.oracle_write_kv.restype = ctypes.c_int
         L.oracle_write_kv.argtypes = [P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                       P, P, P, ctypes.c_int64, ctypes.c_int32]
@@ -75,8 +76,9 @@ class Oracle:
                                           ctypes.c_int32]
         L.oracle_decode_fp8.restype = ctypes.c_int
         L.oracle_decode_fp8.argtypes = [P, P, ctypes.c_int, ctypes.c_int32, ctypes.c_int32,
-                                        ctypes.c_int32, P, P, ctypes.c_int64, ctypes.c_int32,
-                                        P, ctypes.c_int32, P, ctypes.c_double, ctypes.c_int]
+                                        ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_int64,
+                                        ctypes.c_int32, P, ctypes.c_int32, P, ctypes.c_double,
+                                        ctypes.c_int]
         L.oracle_e4m3_decode.restype = ctypes.c_double
         L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
@@ -174,10 +176,11 @@ class Oracle:
         bt = np.ascontiguousarray(block_tables, dtype=np.int32)
         ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
         S, H, D = query.shape
+        Hk = key_cache.shape[1]
         assert key_cache.dtype == np.uint8 and value_cache.shape == key_cache.shape
-        assert key_cache.shape[1:] == (H, block_size * D + 4 * block_size)
+        assert key_cache.shape[2] == block_size * D + 4 * block_size and H % Hk == 0
         out = np.zeros((S, H, D), dtype=np.float64)
-        rc = self.lib.oracle_decode_fp8(_ptr(out), _ptr(query), _DT[io_dtype], S, H, D,
+        rc = self.lib.oracle_decode_fp8(_ptr(out), _ptr(query), _DT[io_dtype], S, H, Hk, D,
                                         _ptr(np.ascontiguousarray(key_cache)),
                                         _ptr(np.ascontiguousarray(value_cache)),
                                         key_cache.shape[0], block_size, _ptr(bt), bt.shape[1],
@@ -194,11 +197,11 @@ class Oracle:
         bt = np.ascontiguousarray(block_tables, dtype=np.int32)
         ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
         S, H, D = query.shape
-        NB, Hc, bs, Dc = key_cache.shape
-        assert (Hc, Dc) == (H, D) and value_cache.shape == key_cache.shape
+        NB, Hk, bs, Dc = key_cache.shape
+        assert Dc == D and H % Hk == 0 and value_cache.shape == key_cache.shape
         assert bt.ndim == 2 and bt.shape[0] == S and ctx.shape == (S,)
         out = np.zeros((S, H, D), dtype=np.float64)
-        rc = self.lib.oracle_decode(_ptr(out), _ptr(query), S, H, D, _ptr(key_cache),
+        rc = self.lib.oracle_decode(_ptr(out), _ptr(query), S, H, Hk, D, _ptr(key_cache),
                                     _ptr(value_cache), NB, bs, _DT[dtype], _ptr(bt),
                                     bt.shape[1], _ptr(ctx), float(scale), int(threads))
         if rc:

@@ -27,6 +27,9 @@
  * Layout (a reading; the pages never print one): each pool is
  * [num_blocks][num_heads][block_size][head_dim], elements as raw 16-bit
  * patterns (fp16 or bf16). query/key/value/out are [rows][num_heads][head_dim].
+ * Grouped heads (a reading; not on the pages): with num_heads query heads
+ * over num_kv_heads K/V heads, query head h reads K/V head
+ * h / (num_heads / num_kv_heads).
  * An fp8 pool (KV-cache quantisation, named by "vLLM基础", §2.5 as further
  * tuning on top of paging; the format below is a reading) holds per
  * (block, head) block_size rows of head_dim OCP e4m3 codes followed by
@@ -286,9 +289,9 @@ int oracle_write_kv_fp8(const uint16_t *key, const uint16_t *value, int io_dtype
 /* One (sequence, head) of a 16-bit cache: gather the context through the
  * block table, then textbook attention. */
 static int decode_one(double *out, const uint16_t *q16, const uint16_t *key_cache,
-                      const uint16_t *value_cache, int64_t num_blocks, int32_t num_heads,
+                      const uint16_t *value_cache, int64_t num_blocks, int32_t num_kv_heads,
                       int32_t block_size, int32_t head_dim, int dtype, const int32_t *table,
-                      int32_t table_len, int32_t ctx, int32_t h, double scale)
+                      int32_t table_len, int32_t ctx, int32_t kvh, double scale)
 {
     if (ctx <= 0) {
         for (int32_t d = 0; d < head_dim; ++d)
@@ -317,7 +320,8 @@ static int decode_one(double *out, const uint16_t *q16, const uint16_t *key_cach
             rc = -1;
             goto done;
         }
-        size_t base = (size_t)(((block * num_heads + h) * block_size + j % block_size) * head_dim);
+        size_t base =
+            (size_t)(((block * num_kv_heads + kvh) * block_size + j % block_size) * head_dim);
         for (int32_t d = 0; d < head_dim; ++d) {
             K[(size_t)j * head_dim + d] = widen(key_cache[base + d], dtype);
             V[(size_t)j * head_dim + d] = widen(value_cache[base + d], dtype);
@@ -336,9 +340,9 @@ done:
  * codes times their row scales. */
 static int decode_one_fp8(double *out, const uint16_t *q16, int io_dtype,
                           const uint8_t *key_cache, const uint8_t *value_cache,
-                          int64_t num_blocks, int32_t num_heads, int32_t block_size,
+                          int64_t num_blocks, int32_t num_kv_heads, int32_t block_size,
                           int32_t head_dim, const int32_t *table, int32_t table_len, int32_t ctx,
-                          int32_t h, double scale)
+                          int32_t kvh, double scale)
 {
     if (ctx <= 0) {
         for (int32_t d = 0; d < head_dim; ++d)
@@ -365,7 +369,7 @@ static int decode_one_fp8(double *out, const uint16_t *q16, int io_dtype,
             rc = -1;
             goto done;
         }
-        size_t base = (size_t)(block * num_heads + h) * tile;
+        size_t base = (size_t)(block * num_kv_heads + kvh) * tile;
         int32_t off = j % block_size;
         float sk, sv;
         memcpy(&sk, key_cache + base + (size_t)block_size * head_dim + 4 * off, 4);
@@ -390,11 +394,14 @@ done:
  * OpenMP default. Returns 0, or -1 if some block id or context length does
  * not fit the pool or the table (that (seq, head) is then left unwritten). */
 int oracle_decode(double *out, const uint16_t *query, int32_t num_seqs, int32_t num_heads,
-                  int32_t head_dim, const uint16_t *key_cache, const uint16_t *value_cache,
-                  int64_t num_blocks, int32_t block_size, int dtype,
+                  int32_t num_kv_heads, int32_t head_dim, const uint16_t *key_cache,
+                  const uint16_t *value_cache, int64_t num_blocks, int32_t block_size, int dtype,
                   const int32_t *block_tables, int32_t max_blocks_per_seq,
                   const int32_t *context_lens, double scale, int num_threads)
 {
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads)
+        return -1;
+    int32_t group = num_heads / num_kv_heads;
     int rc = 0;
     int64_t units = (int64_t)num_seqs * num_heads;
 #ifdef _OPENMP
@@ -405,9 +412,9 @@ int oracle_decode(double *out, const uint16_t *query, int32_t num_seqs, int32_t 
     for (int64_t u = 0; u < units; ++u) {
         int32_t s = (int32_t)(u / num_heads), h = (int32_t)(u % num_heads);
         int r = decode_one(out + u * head_dim, query + u * head_dim, key_cache, value_cache,
-                           num_blocks, num_heads, block_size, head_dim, dtype,
+                           num_blocks, num_kv_heads, block_size, head_dim, dtype,
                            block_tables + (int64_t)s * max_blocks_per_seq,
-                           max_blocks_per_seq, context_lens[s], h, scale);
+                           max_blocks_per_seq, context_lens[s], h / group, scale);
         if (r < rc)
             rc = r;
     }
@@ -418,11 +425,15 @@ int oracle_decode(double *out, const uint16_t *query, int32_t num_seqs, int32_t 
 /* oracle_decode for fp8 pools (uint8, tiles of codes then row scales);
  * query in io_dtype. */
 int oracle_decode_fp8(double *out, const uint16_t *query, int io_dtype, int32_t num_seqs,
-                      int32_t num_heads, int32_t head_dim, const uint8_t *key_cache,
-                      const uint8_t *value_cache, int64_t num_blocks, int32_t block_size,
-                      const int32_t *block_tables, int32_t max_blocks_per_seq,
-                      const int32_t *context_lens, double scale, int num_threads)
+                      int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                      const uint8_t *key_cache, const uint8_t *value_cache, int64_t num_blocks,
+                      int32_t block_size, const int32_t *block_tables,
+                      int32_t max_blocks_per_seq, const int32_t *context_lens, double scale,
+                      int num_threads)
 {
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads)
+        return -1;
+    int32_t group = num_heads / num_kv_heads;
     int rc = 0;
     int64_t units = (int64_t)num_seqs * num_heads;
 #ifdef _OPENMP
@@ -433,9 +444,9 @@ int oracle_decode_fp8(double *out, const uint16_t *query, int io_dtype, int32_t 
     for (int64_t u = 0; u < units; ++u) {
         int32_t s = (int32_t)(u / num_heads), h = (int32_t)(u % num_heads);
         int r = decode_one_fp8(out + u * head_dim, query + u * head_dim, io_dtype, key_cache,
-                               value_cache, num_blocks, num_heads, block_size, head_dim,
+                               value_cache, num_blocks, num_kv_heads, block_size, head_dim,
                                block_tables + (int64_t)s * max_blocks_per_seq,
-                               max_blocks_per_seq, context_lens[s], h, scale);
+                               max_blocks_per_seq, context_lens[s], h / group, scale);
         if (r < rc)
             rc = r;
     }

@@ -374,5 +374,20 @@ def pin_fp8(orc, seed=18):
         assert np.max(np.abs(got[s] - ref)) <= 1e-12, "fp8 decode vs dense"
 
 
-ALL_PINS = [pin_dense, pin_bruteforce, pin_closed_forms, pin_permutation, pin_write_kv,
+def pin_grouped_heads(orc, seed=19):
+    """Grouped heads: query head h attends to K/V head h // G, as dense
+    attention on the unpaged copy with the K/V heads repeated G times."""
+    rng = np.random.default_rng(seed)
+    for Hk, G, dtype in [(2, 4, "f16"), (1, 3, "f16"), (2, 2, "bf16")]:
+        c = paged_case(rng, [1, 20, 75], Hk, 64, 16, dtype=dtype)
+        q = to_storage_bits(rng.standard_normal((3, Hk * G, 64), dtype=np.float32), dtype)
+        got = orc.decode(q, c["kpool"], c["vpool"], c["bt"], c["ctx"], c["scale"], dtype)
+        for s in range(3):
+            K = np.repeat(c["K"][s], G, axis=1)
+            V = np.repeat(c["V"][s], G, axis=1)
+            ref = dense_attention(q[s], K, V, c["scale"], dtype)
+            assert np.max(np.abs(got[s] - ref)) <= 1e-12, "grouped heads vs dense"
+
+
+ALL_PINS = [pin_grouped_heads, pin_dense, pin_bruteforce, pin_closed_forms, pin_permutation, pin_write_kv,
             pin_copy_blocks, pin_swap_blocks, pin_fp8]

@@ -131,8 +131,8 @@ MUTANTS = [
     ("no_normalise", "out[d] = acc / z;", "out[d] = acc;"),
     ("slot_offset", "* block_size + j % block_size) * head_dim);",
      "* block_size + (j + 1) % block_size) * head_dim);"),
-    ("head_index", "((block * num_heads + h) * block_size + j % block_size)",
-     "((block * num_heads + 0) * block_size + j % block_size)"),
+    ("head_index", "(((block * num_kv_heads + kvh) * block_size + j % block_size)",
+     "(((block * num_kv_heads + 0) * block_size + j % block_size)"),
     ("table_index", "int64_t block = table[j / block_size];",
      "int64_t block = table[(j / block_size + 1) % table_len];"),
     ("fp8_table_index", "int64_t block = table[j / block_size];",
@@ -156,6 +156,8 @@ MUTANTS = [
      "memcpy(dst_v[l] + b * block_elems, src_k[l] + a * block_elems,"),
     ("swap_wrong_dst", "memcpy(dst_k[l] + b * block_elems, src_k[l] + a * block_elems,",
      "memcpy(dst_k[l] + a % dst_blocks * block_elems, src_k[l] + a * block_elems,"),
+    ("gqa_head_map", "context_lens[s], h / group, scale);",
+     "context_lens[s], h % num_kv_heads, scale);"),
     ("f16_exponent_bias", "v = ldexp((double)(f | 0x400), e - 25);",
      "v = ldexp((double)(f | 0x400), e - 24);"),
 ]
