@@ -331,6 +331,8 @@ def main():
     ap.add_argument("--soak-seconds", type=float, default=1.0)
     ap.add_argument("--kv-dtype", default="f16", choices=["f16", "bf16", "fp8"],
                     help="cache storage (fp8: e4m3 codes + fp32 row scales, fp16 rows)")
+    ap.add_argument("--kv-heads", type=int, default=0,
+                    help="llama7b_layer / full_step: K/V heads (grouped query heads)")
     ap.add_argument("--separate", action="store_true",
                     help="pa_write_kv then pa_decode instead of the fused pa_write_kv_decode")
     ap.add_argument("--no-graph", action="store_true",
@@ -378,6 +380,16 @@ def main():
         step = wl.llama_layer(seed=SEEDS[args.config] + 1000 * rank, num_seqs=args.seqs,
                               num_blocks=max(256, 8192 * args.seqs // 96), dtype=args.kv_dtype)
         config_desc["workload"] += f" (reduced to {args.seqs} seqs)"
+    elif args.kv_heads:
+        seed = SEEDS[args.config] + 1000 * rank
+        if args.config == "llama7b_layer":
+            step = wl.llama_layer(seed=seed, dtype=args.kv_dtype, num_kv_heads=args.kv_heads)
+        elif args.config.startswith("full_step_bs"):
+            step = wl.full_step(seed=seed, dtype=args.kv_dtype, num_kv_heads=args.kv_heads,
+                                block_size=int(args.config[len("full_step_bs"):]))
+        else:
+            ap.error("--kv-heads applies to llama7b_layer and full_step_bs*")
+        config_desc["workload"] += f" with {args.kv_heads} K/V heads (grouped query heads)"
     else:
         step = WORKLOADS[args.config][0](SEEDS[args.config] + 1000 * rank, args.kv_dtype)
     if args.kv_dtype != "f16":

@@ -25,8 +25,9 @@
  *   row x as scale = amax/448, codes = e4m3(x * (448/amax)) (fp32 steps,
  *   round to nearest even, saturating). Query, key, value and outputs are
  *   then of the descriptor's io_dtype (PA_F16 or PA_BF16).
- * - Supported shapes: head_dim 64 or 128; block_size 8, 16 or 32;
- *   num_heads == num_kv_heads (one query head per KV head).
+ * - Supported shapes: head_dim 64 or 128; block_size 8, 16 or 32; num_heads
+ *   a multiple of num_kv_heads. With G = num_heads / num_kv_heads > 1
+ *   (grouped heads, not on the pages), query head h reads K/V head h / G.
  * - Ownership: the caller owns every buffer, including the decode
  *   workspace. The library allocates no memory, keeps no per-call state and
  *   never synchronises; every call only enqueues kernels on `stream` (a
@@ -123,7 +124,9 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads, int32_t he
  *
  * out           device [num_seqs][num_heads][head_dim] of out_dtype
  *               (PA_F16, PA_BF16 or PA_F32).
- * query         device [num_seqs][num_heads][head_dim], cache dtype.
+ * query         device [num_seqs][num_heads][head_dim], cache dtype (fp8
+ *               caches: the descriptor's io_dtype). num_heads must be a
+ *               multiple of cache->num_kv_heads.
  * block_tables  device int32 [num_seqs][max_blocks_per_seq]; only the first
  *               ceil(context_len / block_size) entries of a row are read.
  * context_lens  device int32 [num_seqs]; 0 gives a zero output row.
@@ -158,8 +161,9 @@ pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t nu
  * sequence s is its last context token, position context_lens[s] - 1, and
  * its slot is the one the block table gives that position (the in-order
  * fill of "啃透vLLM源码", §2.2 append_tokens). key/value (device
- * [num_seqs][num_heads][head_dim], cache dtype, 16-byte aligned) hold the
- * new rows. The result equals pa_write_kv with that slot mapping followed by
+ * [num_seqs][num_kv_heads][head_dim], cache io dtype, 16-byte aligned)
+ * hold the new rows, one per K/V head.
+ * The result equals pa_write_kv with that slot mapping followed by
  * pa_decode; the kernel that reads the sequence's last chunk puts the new
  * row into its staged copy and into the cache, so no other launch is needed.
  * Preconditions: the block that receives the new token is read by no other

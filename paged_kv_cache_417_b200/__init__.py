@@ -274,7 +274,8 @@ def write_kv_decode(out, query, key, value, key_cache, value_cache, block_tables
     _need(out, "out")
     if out.dtype not in _DTYPE:
         raise ValueError("out dtype must be float16, bfloat16 or float32")
-    if not (out.shape == query.shape == key.shape == value.shape):
+    if out.shape != query.shape or key.shape != value.shape or key.shape[0] != query.shape[0] \
+            or key.shape[2] != query.shape[2]:
         raise ValueError("shape mismatch")
     desc = cache_desc(key_cache)
     S, H, D = query.shape

@@ -63,12 +63,12 @@ struct DecodeParams {
     float *ws_acc; // [S][H][num_parts][D]
     float *ws_ml;  // [S][H][num_parts][2] = (max, sum), base-2 domain
     int32_t *dev_err;
-    int32_t num_seqs, num_heads, num_blocks, max_blocks_per_seq, max_context_len;
+    int32_t num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq, max_context_len;
     int32_t partition_size, num_parts;
     int32_t out_dtype; // 0 f16, 1 bf16, 2 f32
     float qk_scale_log2;
     // Fused append (pa_write_kv_decode): the new token of sequence s, at
-    // position context_lens[s] - 1, has K/V rows new_key/new_value[s][h][:];
+    // position context_lens[s] - 1, has K/V rows new_key/new_value[s][kv head][:];
     // NULL for a plain decode.
     const void *new_key;
     const void *new_value;
@@ -653,7 +653,9 @@ __global__ void __launch_bounds__(NW * 32)
     pdl_launch_dependents();
     const int h = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = p.num_heads;
+    const int H = p.num_heads, HK = p.num_kv_heads;
+    const int group = H / HK;  // query heads per K/V head
+    const int kvh = h / group; // the K/V head this query head reads
 
     if (tid == 0)
         cta_flags = 0;
@@ -684,7 +686,7 @@ __global__ void __launch_bounds__(NW * 32)
             const bool isv = lane >= RV;
             const int piece = lane % RV;
             const QT *src = static_cast<const QT *>(isv ? p.new_value : p.new_key) +
-                            ((size_t)s * H + h) * D + (size_t)piece * E;
+                            ((size_t)s * HK + kvh) * D + (size_t)piece * E;
             if constexpr (Store<T>::kScaled) {
                 // Quantise the new row: amax over its D inputs, then
                 // codes = e4m3(x * (448 / amax)) and scale = amax / 448.
@@ -709,13 +711,13 @@ __global__ void __launch_bounds__(NW * 32)
                 if (lane < 2 * RV)
                     ws.patch_val = *reinterpret_cast<const uint4 *>(src);
             }
-            if (lane < 2 * RV) {
+            if (lane < 2 * RV && h % group == 0) { // one query head per group writes
                 const int b = table[(u.n_tok - 1) / BS];
                 if (b >= 0 && b < p.num_blocks) {
                     char *cache =
                         const_cast<char *>(static_cast<const char *>(isv ? p.value_cache
                                                                            : p.key_cache));
-                    char *tile = cache + ((size_t)b * H + h) * TILE;
+                    char *tile = cache + ((size_t)b * HK + kvh) * TILE;
                     const int off = (u.n_tok - 1) % BS;
                     ws.patch_dst = reinterpret_cast<uint4 *>(tile + (size_t)off * ROW) + piece;
                     if (Store<T>::kScaled && piece == 0)
@@ -726,8 +728,8 @@ __global__ void __launch_bounds__(NW * 32)
         }
     }
     const bool ok = ws.run(static_cast<const char *>(p.key_cache),
-                           static_cast<const char *>(p.value_cache), (size_t)h * TILE,
-                           (size_t)H * TILE, p.num_blocks, table, u.n_tok, warp, NW, my_chunks,
+                           static_cast<const char *>(p.value_cache), (size_t)kvh * TILE,
+                           (size_t)HK * TILE, p.num_blocks, table, u.n_tok, warp, NW, my_chunks,
                            rings + (size_t)warp * W::C::kRingBytes, smem_addr(&bars[warp * NS]));
     if (lane == 0) {
         if (!ok) {

@@ -348,8 +348,8 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
         return s;
     if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq < 0 || max_context_len < 0)
         return fail(PA_ERR_INVALID_ARG, "negative size argument");
-    if (num_heads != cache->num_kv_heads)
-        return fail(PA_ERR_UNSUPPORTED, "num_heads %d != num_kv_heads %d (grouped heads not built)",
+    if (num_heads % cache->num_kv_heads != 0)
+        return fail(PA_ERR_UNSUPPORTED, "num_heads %d is not a multiple of num_kv_heads %d",
                     num_heads, cache->num_kv_heads);
     if (out_dtype != PA_F16 && out_dtype != PA_BF16 && out_dtype != PA_F32)
         return fail(PA_ERR_INVALID_ARG, "out_dtype %d", (int)out_dtype);
@@ -388,6 +388,7 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
     p.dev_err = dev_err;
     p.num_seqs = num_seqs;
     p.num_heads = num_heads;
+    p.num_kv_heads = cache->num_kv_heads;
     p.num_blocks = cache->num_blocks;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.max_context_len = max_context_len;

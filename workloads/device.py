@@ -22,7 +22,7 @@ def _bits_to_tensor(bits: np.ndarray, dtype: str, device) -> torch.Tensor:
 def device_pools(step: DecodeStep, layer: int, device, base_dev=None):
     """Pre-step (key_cache, value_cache) of one layer, [NB, H, bs, D]
     (fp8: uint8 [NB, H, bs*D + 4*bs], built on the host)."""
-    bs, H, D = step.block_size, step.num_heads, step.head_dim
+    bs, H, D = step.block_size, step.num_kv_heads, step.head_dim
     if step.dtype == "fp8":
         from .steps import host_pools
         k, v = host_pools(step, layer)

@@ -69,8 +69,8 @@ class LayerInputs:
     query: np.ndarray       # uint16 [S, H, D]
     new_key: np.ndarray     # uint16 [S, H, D]
     new_value: np.ndarray   # uint16 [S, H, D]
-    tile_rows_k: np.ndarray  # int64 [NB, H], row of ``base`` or -1 (NaN tile)
-    tile_rows_v: np.ndarray  # int64 [NB, H]
+    tile_rows_k: np.ndarray  # int64 [NB, Hkv], row of ``base`` or -1 (NaN tile)
+    tile_rows_v: np.ndarray  # int64 [NB, Hkv]
 
 
 @dataclass
@@ -92,6 +92,11 @@ class DecodeStep:
     layers: list = field(default_factory=list)
     ref_count: np.ndarray = None  # int64 [NB], after the step
     meta: dict = field(default_factory=dict)
+    num_kv_heads: int = 0      # K/V heads (0: same as num_heads)
+
+    def __post_init__(self):
+        if not self.num_kv_heads:
+            self.num_kv_heads = self.num_heads
 
     @property
     def num_layers(self) -> int:
@@ -125,7 +130,7 @@ def _draw_fp8_tiles(rng, rows, block_size, head_dim):
 
 def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
                pre_tokens, num_layers=1, scale=None, dtype="f16",
-               prefix_tokens=0, fork_partial_tail=False, order=None):
+               prefix_tokens=0, fork_partial_tail=False, order=None, num_kv_heads=None):
     """Build one decode step.
 
     ``pre_tokens[s]`` tokens of sequence ``s`` are in the cache before the
@@ -139,6 +144,9 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
     if dtype not in ("f16", "bf16", "fp8"):
         raise ValueError(dtype)
     bs, H, D = int(block_size), int(num_heads), int(head_dim)
+    Hk = int(num_kv_heads or num_heads)
+    if H % Hk:
+        raise ValueError("num_heads must be a multiple of num_kv_heads")
     S = len(pre_tokens)
     if order is None:
         order = rng.permutation(num_blocks)
@@ -180,7 +188,7 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
     # Tile bank: a distinct row per filled tile when that fits the bank,
     # else rows drawn with replacement.
     filled = np.nonzero(valid > 0)[0]
-    n_tiles = 2 * len(filled) * H
+    n_tiles = 2 * len(filled) * Hk
     rows = max(1, min(n_tiles, MAX_BANK_ROWS))
     if dtype == "fp8":
         base = _draw_fp8_tiles(rng, rows, bs, D)
@@ -193,16 +201,16 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
             pick = rng.permutation(rows)[:n_tiles] if n_tiles else np.zeros(0, np.int64)
         else:
             pick = rng.integers(0, rows, size=n_tiles)
-        pick = pick.astype(np.int64).reshape(2, len(filled), H) if n_tiles else \
-            np.zeros((2, 0, H), np.int64)
-        tk = np.full((num_blocks, H), -1, dtype=np.int64)
-        tv = np.full((num_blocks, H), -1, dtype=np.int64)
+        pick = pick.astype(np.int64).reshape(2, len(filled), Hk) if n_tiles else \
+            np.zeros((2, 0, Hk), np.int64)
+        tk = np.full((num_blocks, Hk), -1, dtype=np.int64)
+        tv = np.full((num_blocks, Hk), -1, dtype=np.int64)
         tk[filled] = pick[0]
         tv[filled] = pick[1]
         layers.append(LayerInputs(
             query=_draw_bits(rng, (S, H, D), io),
-            new_key=_draw_bits(rng, (S, H, D), io),
-            new_value=_draw_bits(rng, (S, H, D), io),
+            new_key=_draw_bits(rng, (S, Hk, D), io),
+            new_value=_draw_bits(rng, (S, Hk, D), io),
             tile_rows_k=tk, tile_rows_v=tv))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
@@ -215,7 +223,7 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
         valid_slots=valid, base=base, layers=layers,
         ref_count=alloc.ref_count.copy(),
         meta={"allocator": alloc, "seqs": seqs, "phantom_holders": phantom,
-              "prefix_tokens": prefix_tokens})
+              "prefix_tokens": prefix_tokens}, num_kv_heads=Hk)
     return step
 
 
@@ -234,7 +242,7 @@ def tiny(seed=0, dtype="f16", context_lens=(1, 17, 33, 100)):
 
 
 def llama_layer(seed=1, dtype="f16", num_seqs=96, ctx_range=(128, 2048),
-                num_blocks=8192, num_heads=32, head_dim=128, block_size=16):
+                num_blocks=8192, num_heads=32, head_dim=128, block_size=16, num_kv_heads=None):
     """Llama-7B-shaped single-layer decode: 96 sequences, 32 heads,
     head_dim 128, block_size 16, context_lens uniform in [128, 2048], block
     ids from a seeded shuffle of an 8192-block pool."""
@@ -242,7 +250,7 @@ def llama_layer(seed=1, dtype="f16", num_seqs=96, ctx_range=(128, 2048),
     ctx = rng.integers(ctx_range[0], ctx_range[1] + 1, size=num_seqs)
     return build_step(rng, "llama7b_layer_b%d" % num_seqs, num_blocks=num_blocks,
                       block_size=block_size, num_heads=num_heads, head_dim=head_dim,
-                      pre_tokens=ctx - 1, dtype=dtype)
+                      pre_tokens=ctx - 1, dtype=dtype, num_kv_heads=num_kv_heads)
 
 
 def long_context(seed=2, dtype="f16", num_seqs=8, ctx_range=(16384, 32768),
@@ -276,7 +284,7 @@ def prefix_cow(seed=3, dtype="f16", num_seqs=64, prefix_tokens=1024,
 
 
 def full_step(seed=4, dtype="f16", block_size=16, num_seqs=256, num_layers=32,
-              mean_ctx=300, max_ctx=4096, num_heads=32, head_dim=128):
+              mean_ctx=300, max_ctx=4096, num_heads=32, head_dim=128, num_kv_heads=None):
     """All layers of a Llama-7B-shaped cache for 256 sequences whose
     context_lens are geometric with mean 300, capped at 4096. The block
     tables are shared by all layers; each layer has its own pool."""
@@ -286,7 +294,8 @@ def full_step(seed=4, dtype="f16", block_size=16, num_seqs=256, num_layers=32,
     num_blocks = int(math.ceil(need * 1.25)) + 1
     return build_step(rng, "full_step_bs%d" % block_size, num_blocks=num_blocks,
                       block_size=block_size, num_heads=num_heads, head_dim=head_dim,
-                      pre_tokens=ctx - 1, num_layers=num_layers, dtype=dtype)
+                      pre_tokens=ctx - 1, num_layers=num_layers, dtype=dtype,
+                      num_kv_heads=num_kv_heads)
 
 
 CONFIGS = {
@@ -305,7 +314,7 @@ CONFIGS = {
 def host_pools(step: DecodeStep, layer: int = 0):
     """Return the pre-step (key_pool, value_pool) of one layer as uint16
     arrays [NB, H, bs, D] (fp8: uint8 [NB, H, bs*D + 4*bs])."""
-    bs, H, D = step.block_size, step.num_heads, step.head_dim
+    bs, H, D = step.block_size, step.num_kv_heads, step.head_dim
     L = step.layers[layer]
     if step.dtype == "fp8":
         return _host_pools_fp8(step, L)
@@ -322,7 +331,7 @@ def host_pools(step: DecodeStep, layer: int = 0):
 
 
 def _host_pools_fp8(step, L):
-    bs, H, D = step.block_size, step.num_heads, step.head_dim
+    bs, H, D = step.block_size, step.num_kv_heads, step.head_dim
     tb = fp8_tile_bytes(bs, D)
     dead = np.arange(bs)[None, :] >= step.valid_slots[:, None]          # [NB, bs]
     pools = []
@@ -370,7 +379,8 @@ def subset(step: DecodeStep, seq_ids) -> DecodeStep:
         context_lens=step.context_lens[seq_ids].copy(), block_tables=new_bt,
         slot_mapping=new_slots.astype(np.int64), copy_pairs=new_pairs,
         valid_slots=step.valid_slots[blocks].copy(), base=step.base, layers=layers,
-        ref_count=None, meta={"parent": step.name, "seq_ids": seq_ids})
+        ref_count=None, meta={"parent": step.name, "seq_ids": seq_ids},
+        num_kv_heads=step.num_kv_heads)
 
 
 def kv_bytes_read(step: DecodeStep) -> int:
@@ -378,4 +388,4 @@ def kv_bytes_read(step: DecodeStep) -> int:
     context_len tokens x heads x 2 (K and V) x the bytes of a row (head_dim
     x 2 for 16-bit caches; head_dim codes + a 4-byte scale for fp8)."""
     per_row = step.head_dim + 4 if step.dtype == "fp8" else step.head_dim * 2
-    return int(np.sum(step.context_lens.astype(np.int64))) * step.num_heads * per_row * 2
+    return int(np.sum(step.context_lens.astype(np.int64))) * step.num_kv_heads * per_row * 2
