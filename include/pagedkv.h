@@ -260,6 +260,14 @@ pa_status pa_swap_blocks(void *const *src_key_caches, void *const *src_value_cac
                          int32_t num_layers, const int64_t *block_mapping, int32_t num_pairs,
                          int32_t *dev_err, void *stream);
 
+/* Self-test of failure detection: one warp waits on a shared-memory barrier
+ * that nothing will complete, through the same bounded wait every kernel
+ * uses on its bulk copies, giving up after limit_us microseconds (1 ..
+ * 1000000). It must then OR PA_DEVERR_TIMEOUT into *dev_err (device memory)
+ * and return, leaving the context usable: the way a kernel stuck on a copy
+ * reports instead of hanging. No counterpart on the pages. */
+pa_status pa_selftest_wait_timeout(int32_t *dev_err, uint32_t limit_us, void *stream);
+
 /* Static text for a status. */
 const char *pa_status_string(pa_status status);
 

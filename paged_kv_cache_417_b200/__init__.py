@@ -115,6 +115,8 @@ _lib.pa_swap_blocks.restype = ctypes.c_int
 _lib.pa_swap_blocks.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(CacheDesc),
                                 ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(CacheDesc),
                                 _i32, _P, _i32, _P, _P]
+_lib.pa_selftest_wait_timeout.restype = ctypes.c_int
+_lib.pa_selftest_wait_timeout.argtypes = [_P, ctypes.c_uint32, _P]
 _lib.pa_status_string.restype = ctypes.c_char_p
 _lib.pa_status_string.argtypes = [ctypes.c_int]
 _lib.pa_last_error.restype = ctypes.c_char_p
@@ -366,3 +368,13 @@ def swap_blocks(src_key_caches, src_value_caches, dst_key_caches, dst_value_cach
     _check(_lib.pa_swap_blocks(arr(src_key_caches), arr(src_value_caches), ctypes.byref(sd),
                                arr(dst_key_caches), arr(dst_value_caches), ctypes.byref(dd),
                                L, _ptr(block_mapping), n, _ptr(dev_err), stream))
+
+
+def selftest_wait_timeout(limit_us: int = 1000, device="cuda") -> int:
+    """Run the bounded-wait self-test and return the device error bits it
+    produced (PA_DEVERR_TIMEOUT expected)."""
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(_lib.pa_selftest_wait_timeout(_ptr(err), int(limit_us),
+                                         torch.cuda.current_stream(err.device).cuda_stream))
+    torch.cuda.synchronize(err.device)
+    return int(err.item())

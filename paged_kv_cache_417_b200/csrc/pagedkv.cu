@@ -483,6 +483,34 @@ pa_status pa_copy_blocks(void *const *key_caches, void *const *value_caches, int
     return ok();
 }
 
+// Self-test of the bounded wait every kernel uses on its shared-memory
+// copies: one warp waits on an mbarrier that nothing will complete.
+__global__ void bounded_wait_selftest_kernel(int32_t *dev_err, uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0)
+        mbar_init(smem_addr(&bar), 1);
+    fence_mbar_init();
+    __syncwarp();
+    const bool ok = mbar_wait_bounded(smem_addr(&bar), 0, limit_ns);
+    if (__any_sync(0xffffffffu, !ok) && threadIdx.x == 0)
+        report(dev_err, PA_DEVERR_TIMEOUT);
+}
+
+pa_status pa_selftest_wait_timeout(int32_t *dev_err, uint32_t limit_us, void *stream)
+{
+    if (!dev_err)
+        return fail(PA_ERR_INVALID_ARG, "dev_err is NULL");
+    if (limit_us == 0 || limit_us > 1000000u)
+        return fail(PA_ERR_INVALID_ARG, "limit_us %u outside [1, 1000000]", limit_us);
+    bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        dev_err, (uint64_t)limit_us * 1000u);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "self-test launch");
+    return ok();
+}
+
 // The address a kernel uses for `p`: device memory as is, pinned host memory
 // through its device mapping. Pageable host memory (which no kernel may
 // touch) and unknown pointers are refused.

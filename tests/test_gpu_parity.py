@@ -297,3 +297,13 @@ def test_maximum_partition_and_many_partitions():
     for partition in (8192, 32):
         out, err = decode_case(c, partition_size=partition)
         assert err == 0 and max_err(out, ref) <= TOL
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait that nothing completes gives up after its limit, reports
+    PA_DEVERR_TIMEOUT, and the next decode on the same context is correct."""
+    assert pk.selftest_wait_timeout(2000) & pk.PA_DEVERR_TIMEOUT
+    rng = np.random.default_rng(41)
+    c = pc.paged_case(rng, [30, 300], 2, 128, 16)
+    out, err = decode_case(c)
+    assert err == 0 and max_err(out, orc_decode(c)) <= TOL
