@@ -91,12 +91,12 @@ def algorithmic_bytes(step) -> dict:
     return {"kv": kv, "total": kv + qo + table}
 
 
-def kernel_source_hash() -> str:
-    """Hash of the decode kernel's own sources (the ncu traffic record is
-    void once they change)."""
+def kernel_source_hash(sources=("decode.cuh", "ptx.cuh")) -> str:
+    """Hash of a decode kernel's own sources (an ncu traffic record is void
+    once they change)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_417_b200", "csrc")
-    for name in ("decode.cuh", "ptx.cuh"):
+    for name in sources:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -111,6 +111,19 @@ def measured_peak():
         return FALLBACK_PEAK_GBS, "fallback"
 
 
+def traffic_key(args):
+    """Name of the workload in profiles/traffic.json: the config, plus the
+    K/V dtype and head count when they differ from the config's own."""
+    key = args.config
+    if args.kv_dtype != "f16":
+        key += f"_{args.kv_dtype}"
+    if args.kv_heads:
+        key += f"_kvh{args.kv_heads}"
+    if args.seqs:
+        key += f"_s{args.seqs}"
+    return key
+
+
 def recorded_traffic(config):
     """DRAM bytes per decode launch from an ncu capture, if one was taken on
     the current kernel sources (profiles/traffic.json); else None."""
@@ -120,7 +133,8 @@ def recorded_traffic(config):
             rec = json.load(f).get(config)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("kernel_source_hash") != kernel_source_hash():
+    if not rec or rec.get("kernel_source_hash") != kernel_source_hash(
+            tuple(rec.get("sources", ("decode.cuh", "ptx.cuh")))):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -406,8 +420,8 @@ def main():
     outs = [torch.empty_like(q) for q in d["query"]]
     ws = pk.alloc_workspace(S, step.num_heads, step.head_dim, step.max_context_len,
                             args.partition, dev)
-    P = pk.decode_partition_size(S, step.num_heads, step.head_dim, step.block_size,
-                                 step.max_context_len, args.partition)
+    P = pk.decode_partition_size(S, step.num_heads, d["key_caches"][0], step.max_context_len,
+                                 args.partition)
     split = step.max_context_len > P
     has_copy = step.copy_pairs.shape[0] > 0
     launches_per_step = (1 if has_copy else 0) + L * ((1 if args.fused else 2) +
@@ -565,7 +579,7 @@ def main():
     achieved = ab["total"] / dec_avg_s / 1e9
     peak, peak_kind = measured_peak()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": recorded_traffic(args.config),
+                "frac": achieved / peak, "traffic": recorded_traffic(traffic_key(args)),
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "kernel": "pa_decode (decode kernel + reduce kernel when split)",

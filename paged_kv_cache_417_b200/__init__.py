@@ -96,7 +96,7 @@ _lib.pa_write_kv.argtypes = [_P, _P, _i32, _i32, _P, _P, _P, ctypes.POINTER(Cach
 _lib.pa_decode_workspace_size.restype = ctypes.c_size_t
 _lib.pa_decode_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
 _lib.pa_decode_partition_size.restype = _i32
-_lib.pa_decode_partition_size.argtypes = [_i32] * 6
+_lib.pa_decode_partition_size.argtypes = [_i32, _i32, ctypes.POINTER(CacheDesc), _i32, _i32]
 _lib.pa_decode.restype = ctypes.c_int
 _lib.pa_decode.argtypes = [_P, ctypes.c_int, _P, _i32, _i32, _P, _P, ctypes.POINTER(CacheDesc),
                            _P, _i32, _P, _i32, ctypes.c_float, _i32, _P, ctypes.c_size_t, _P, _P]
@@ -213,9 +213,10 @@ def decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len, partit
     return int(n)
 
 
-def decode_partition_size(num_seqs, num_heads, head_dim, block_size, max_context_len,
-                          partition_size=0):
-    n = _lib.pa_decode_partition_size(num_seqs, num_heads, head_dim, block_size,
+def decode_partition_size(num_seqs, num_heads, cache, max_context_len, partition_size=0):
+    """``cache``: a key cache (tensor or Fp8Cache) or a CacheDesc."""
+    desc = cache if isinstance(cache, CacheDesc) else cache_desc(cache)
+    n = _lib.pa_decode_partition_size(num_seqs, num_heads, ctypes.byref(desc),
                                       max_context_len, partition_size)
     if n < 0:
         raise ValueError("invalid arguments to decode_partition_size")

@@ -1,8 +1,10 @@
 // pagedkv.cu - the C ABI (include/pagedkv.h): host-side argument checks,
 // launch-shape choices and kernel launches. Nothing here allocates memory or
 // synchronises.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -13,6 +15,7 @@
 #include "cache_ops.cuh"
 #include "last_error.h"
 #include "decode.cuh"
+#include "decode_group.cuh"
 
 using namespace pagedkv;
 
@@ -29,6 +32,14 @@ namespace {
 #endif
 constexpr int kSplitWarps = PA_SPLIT_WARPS;
 constexpr int kSplitStages = PA_SPLIT_STAGES;
+// Grouped-heads decode: 4 warps x 2 TMA stages of 16 tokens (8 KiB at
+// head_dim 128) per warp, 3 CTAs per SM. PA_GROUP_KERNEL=0 builds a variant
+// that sends grouped heads to decode_split_kernel, for comparisons.
+#ifndef PA_GROUP_KERNEL
+#define PA_GROUP_KERNEL 1
+#endif
+constexpr int kGroupWarps = 4;
+constexpr int kGroupStages = 2;
 constexpr int kTargetCtasPerSm = 12; // ~4 waves of 3 resident CTAs
 constexpr int kMinAutoPartition = 128;
 constexpr int kAutoPartition = 2048;
@@ -89,16 +100,37 @@ size_t tile_bytes(const pa_cache_desc *c)
 
 size_t block_bytes(const pa_cache_desc *c) { return tile_bytes(c) * (size_t)c->num_kv_heads; }
 
+// Grouped query heads go to decode_group_kernel (one CTA per K/V head and
+// group) for 16-bit caches, 2 <= G <= 16, and pools whose rows
+// (num_blocks * num_kv_heads * block_size) index as int32 tensor-map
+// coordinates; everything else to decode_split_kernel (one CTA per query
+// head).
+bool use_group_kernel(const pa_cache_desc *c, int32_t num_heads)
+{
+    if (!PA_GROUP_KERNEL || c->num_kv_heads <= 0 || num_heads % c->num_kv_heads != 0)
+        return false;
+    const int G = num_heads / c->num_kv_heads;
+    const int64_t rows = (int64_t)c->num_blocks * c->num_kv_heads * c->block_size;
+    return G >= 2 && G <= kGroupMaxHeads && c->dtype != PA_FP8_E4M3 && rows > 0 &&
+           rows <= INT32_MAX;
+}
+
+// CTA rows of a decode grid per partition: one per (sequence, query head),
+// or per (sequence, K/V head) for the grouped kernel.
+int64_t decode_units(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c)
+{
+    return (int64_t)num_seqs * (use_group_kernel(c, num_heads) ? c->num_kv_heads : num_heads);
+}
+
 // Partition (tokens per work unit) for a decode; >= max_context_len means a
 // single pass. Automatic choice: 2048 tokens, halved (down to 128) while the
-// grid would give fewer than about four waves of resident CTAs.
-int choose_partition(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, int32_t requested,
-                     int sm_count)
+// grid of `units` CTA rows would give fewer than about four waves of
+// resident CTAs.
+int choose_partition(int64_t units, int32_t max_ctx, int32_t requested, int sm_count)
 {
     int P = requested;
     if (P == 0) {
         P = kAutoPartition;
-        const int64_t units = (int64_t)num_seqs * num_heads;
         while (P > kMinAutoPartition &&
                units * ((max_ctx + P - 1) / P) < (int64_t)kTargetCtasPerSm * sm_count)
             P /= 2;
@@ -206,6 +238,112 @@ pa_status dispatch_bs(const DecodeParams &p, int bs, cudaStream_t st)
     return fail(PA_ERR_UNSUPPORTED, "block_size %d", bs);
 }
 
+// The 2-D row view of a 16-bit pool that decode_group_kernel copies from:
+// rows of head_dim elements, boxes of 64 elements x min(block_size, 16) rows,
+// 128-byte swizzle. The encoder is the driver's, looked up once.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tensor_map_encoder()
+{
+    static std::atomic<EncodeTiledFn> cached{nullptr};
+    EncodeTiledFn f = cached.load(std::memory_order_acquire);
+    if (f)
+        return f;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    f = reinterpret_cast<EncodeTiledFn>(fn);
+    cached.store(f, std::memory_order_release);
+    return f;
+}
+
+pa_status encode_pool_rows(CUtensorMap *map, const void *pool, const pa_cache_desc *c)
+{
+    EncodeTiledFn enc = tensor_map_encoder();
+    if (!enc)
+        return fail(PA_ERR_CUDA, "the driver has no cuTensorMapEncodeTiled");
+    const cuuint64_t dims[2] = {(cuuint64_t)c->head_dim,
+                                (cuuint64_t)c->num_blocks * c->num_kv_heads * c->block_size};
+    const cuuint64_t strides[1] = {(cuuint64_t)c->head_dim * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)std::min<int32_t>(c->block_size, 16)};
+    const cuuint32_t elem_strides[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(pool), dims,
+                           strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return PA_OK;
+}
+
+template <typename T, int D, int BS, bool TWO>
+pa_status launch_group(const GroupParams &gp, cudaStream_t stream)
+{
+    using Cfg = GroupCfg<D, BS, kGroupWarps, kGroupStages>;
+    auto kernel = decode_group_kernel<T, D, BS, kGroupWarps, kGroupStages, TWO>;
+    static std::atomic<size_t> smem_set[kMaxDevices];
+    const DecodeParams &p = gp.p;
+    cudaError_t e = allow_smem(kernel, Cfg::smem_bytes(kMaxPartition), smem_set);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute(group decode)");
+    e = launch_pdl(kernel, dim3(p.num_kv_heads, p.num_seqs, p.num_parts),
+                   dim3(kGroupWarps * 32), Cfg::smem_bytes(p.partition_size), stream, gp);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "group decode launch");
+    if (p.num_parts > 1) {
+        e = launch_pdl(reduce_kernel<D>, dim3(p.num_heads, p.num_seqs, 1), dim3(D), 0, stream, p,
+                       (int)BS);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "reduce launch");
+    }
+    return ok();
+}
+
+template <typename T, int D, int BS>
+pa_status group_rows(const GroupParams &gp, cudaStream_t st)
+{
+    if (gp.p.num_heads / gp.p.num_kv_heads > 8)
+        return launch_group<T, D, BS, true>(gp, st);
+    return launch_group<T, D, BS, false>(gp, st);
+}
+
+template <typename T, int D>
+pa_status group_bs(const GroupParams &gp, int bs, cudaStream_t st)
+{
+    switch (bs) {
+    case 8: return group_rows<T, D, 8>(gp, st);
+    case 16: return group_rows<T, D, 16>(gp, st);
+    case 32: return group_rows<T, D, 32>(gp, st);
+    }
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d", bs);
+}
+
+pa_status dispatch_group(const DecodeParams &p, const pa_cache_desc *c, cudaStream_t st)
+{
+    GroupParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    gp.p = p;
+    pa_status s = encode_pool_rows(&gp.tk, p.key_cache, c);
+    if (s == PA_OK)
+        s = encode_pool_rows(&gp.tv, p.value_cache, c);
+    if (s != PA_OK)
+        return s;
+    const bool bf = c->dtype == PA_BF16;
+    if (c->head_dim == 64)
+        return bf ? group_bs<__nv_bfloat16, 64>(gp, c->block_size, st)
+                  : group_bs<__half, 64>(gp, c->block_size, st);
+    return bf ? group_bs<__nv_bfloat16, 128>(gp, c->block_size, st)
+              : group_bs<__half, 128>(gp, c->block_size, st);
+}
+
 template <typename T, typename QT>
 pa_status dispatch_d(const DecodeParams &p, int d, int bs, cudaStream_t st)
 {
@@ -216,6 +354,8 @@ pa_status dispatch_d(const DecodeParams &p, int d, int bs, cudaStream_t st)
 
 pa_status dispatch_decode(const DecodeParams &p, const pa_cache_desc *c, cudaStream_t st)
 {
+    if (use_group_kernel(c, p.num_heads))
+        return dispatch_group(p, c, st);
     if (c->dtype == PA_F16)
         return dispatch_d<__half, __half>(p, c->head_dim, c->block_size, st);
     if (c->dtype == PA_BF16)
@@ -317,16 +457,16 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t hea
     return workspace_bytes_for((int64_t)num_seqs * num_heads, parts, head_dim);
 }
 
-int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
-                                 int32_t block_size, int32_t max_context_len,
+int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
+                                 const pa_cache_desc *cache, int32_t max_context_len,
                                  int32_t partition_size)
 {
-    (void)head_dim;
-    (void)block_size;
-    if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0 ||
+    if (check_cache(cache) != PA_OK || num_seqs < 0 || num_heads <= 0 ||
+        num_heads % cache->num_kv_heads != 0 || max_context_len < 0 ||
         check_partition_request(partition_size) != PA_OK)
         return -1;
-    return choose_partition(num_seqs, num_heads, max_context_len, partition_size,
+    return choose_partition(decode_units(num_seqs, num_heads, cache), max_context_len,
+                            partition_size,
                             partition_size == 0 ? sm_count_of_current_device() : 148);
 }
 
@@ -372,9 +512,11 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
     }
     if (!(scale == scale))
         return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+    if (cache->num_blocks == 0 && max_context_len > 0)
+        return fail(PA_ERR_INVALID_ARG, "empty pool with max_context_len %d", max_context_len);
 
-    const int P = choose_partition(num_seqs, num_heads, max_context_len, partition_size,
-                                   sm_count_of_current_device());
+    const int P = choose_partition(decode_units(num_seqs, num_heads, cache), max_context_len,
+                                   partition_size, sm_count_of_current_device());
     const int64_t parts = max_context_len > P ? (max_context_len + P - 1) / P : 1;
     if (parts > 65535)
         return fail(PA_ERR_UNSUPPORTED, "too many partitions (%lld)", (long long)parts);
@@ -648,8 +790,11 @@ extern "C" pa_status pa_decode_noalloc(void *out, pa_dtype out_dtype, const void
         return s;
     if (num_seqs == 0)
         return ok();
-    const int P = choose_partition(num_seqs, num_heads, max_context_len, partition_size,
-                                   sm_count_of_current_device());
+    if (num_heads % cache->num_kv_heads != 0)
+        return fail(PA_ERR_UNSUPPORTED, "num_heads %d is not a multiple of num_kv_heads %d",
+                    num_heads, cache->num_kv_heads);
+    const int P = choose_partition(decode_units(num_seqs, num_heads, cache), max_context_len,
+                                   partition_size, sm_count_of_current_device());
     const int64_t parts = max_context_len > P ? (max_context_len + P - 1) / P : 1;
     if (parts > 1) {
         const size_t need =

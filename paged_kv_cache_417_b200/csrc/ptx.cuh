@@ -2,6 +2,10 @@
 //
 // mbarrier + cp.async.bulk: a 1-D bulk copy global -> shared that signals an
 // mbarrier with its byte count (the TMA unit's non-tensor path).
+// cp.async.bulk.tensor: a 2-D tiled copy described by a tensor map (the
+// TMA unit's tensor path), here with the 128-byte swizzle.
+// ldmatrix / mma.sync m16n8k16: warp-level tensor-core tiles fed from
+// shared memory, for the grouped-heads decode.
 // griddepcontrol: programmatic dependent launch between back-to-back kernels.
 #pragma once
 
@@ -79,6 +83,56 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         "[%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
+}
+
+// Tiled tensor copy of one box at coordinates (x, y) of a 2-D tensor map
+// (kernel-parameter memory) into shared memory, completing on `bar`. x must
+// be a multiple of 16 bytes' worth of elements; dst 1024-byte aligned for
+// the 128-byte swizzle.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int x, int y,
+                                            uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Four 8x8 tiles of 16-bit elements; lanes 8i..8i+7 give the row addresses
+// of tile i, register i receives it (.trans: transposed).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+// d += a * b for a 16x16 (row-major) by 16x8 (column-major) tile of f16 or
+// bf16 inputs with fp32 accumulation.
+template <bool kBf16>
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1)
+{
+    if constexpr (kBf16)
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+                     "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    else
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+                     "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // Order this thread's generic-proxy writes to shared memory before later

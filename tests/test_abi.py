@@ -123,9 +123,22 @@ def test_workspace_and_partition_sizes(lib):
                                                                                    128)
     with pytest.raises(ValueError):
         lib.decode_workspace_size(S, H, D, ctx, 40)
-    assert lib.decode_partition_size(S, H, D, 16, 100, 0) == 128  # single pass, rounded to 32
-    assert lib.decode_partition_size(96, 32, 128, 16, 2048, 0) == 2048  # single pass
-    assert lib.decode_partition_size(8, 32, 128, 16, 32768, 0) == 2048
-    assert lib.decode_partition_size(1, 32, 128, 16, 32768, 0) == 512
-    assert lib.decode_partition_size(96, 32, 128, 16, 2048, 1024) == 1024
-    assert lib.decode_partition_size(1, 1, 128, 16, 30000, 0) == 128
+    def desc(hkv, dtype=lib.PA_F16, nb=8192, d=128, bs=16):
+        return lib.CacheDesc(nb, bs, hkv, d, dtype, dtype if dtype != lib.PA_FP8_E4M3
+                             else lib.PA_F16)
+
+    assert lib.decode_partition_size(S, H, desc(H, d=D), 100, 0) == 128  # single, rounded to 32
+    assert lib.decode_partition_size(96, 32, desc(32), 2048, 0) == 2048  # single pass
+    assert lib.decode_partition_size(8, 32, desc(32), 32768, 0) == 2048
+    assert lib.decode_partition_size(1, 32, desc(32), 32768, 0) == 512
+    assert lib.decode_partition_size(96, 32, desc(32), 2048, 1024) == 1024
+    assert lib.decode_partition_size(1, 1, desc(1), 30000, 0) == 128
+    # Grouped heads (G = 4) on a 16-bit cache: one CTA row per K/V head, so
+    # 96 x 8 rows need 4 partitions of 512 for four waves; the fp8 cache
+    # stays on one CTA row per query head.
+    assert lib.decode_partition_size(96, 32, desc(8), 2048, 0) == 512
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_BF16), 2048, 0) == 512
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3), 2048, 0) == 2048
+    with pytest.raises(ValueError):
+        lib.decode_partition_size(96, 32, desc(7), 2048, 0)  # 32 % 7 != 0
+    assert lib.decode_partition_size(96, 32, desc(1), 2048, 0) == 2048  # G = 32 > 16
