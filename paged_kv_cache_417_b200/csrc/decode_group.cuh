@@ -7,14 +7,17 @@
 // and the G query rows share every staged tile. The outputs, the split
 // workspace and the reduce are those of decode_split_kernel (per query head).
 //
-// Staging: each pool is viewed as a 2-D tensor of rows (row = one token of
-// one (block, head) tile, D 16-bit elements; row index (block*Hkv + kvh)*bs
-// + offset). A warp's stage receives 16 tokens of K and of V through tiled
-// TMA copies (cp.async.bulk.tensor) of 64-element x min(bs, 16)-row boxes
-// with the 128-byte swizzle: 16-byte piece c of row r lands at piece c ^
-// (r % 8) of its 128-byte line, so the 8 row addresses of an 8x8 ldmatrix
-// tile fall in 8 distinct bank groups. A stage is [K | V] x [D/64 column
-// slabs] x [16 rows x 128 B]; every slab starts on a 1024-byte boundary.
+// Staging: each pool is viewed as a tensor of rows (row = one token of one
+// (block, head) tile, D 16-bit elements; row index (block*Hkv + kvh)*bs +
+// offset), each row split into D/64 128-byte units: dims (64 elements,
+// D/64 units, rows). A warp's stage receives 16 tokens of K and of V
+// through tiled TMA copies (cp.async.bulk.tensor) of min(bs, 16) whole rows
+// per box, contiguous in global memory, with the 128-byte swizzle: 16-byte
+// piece c of 128-byte unit u of the stage lands at piece c ^ (u % 8) of that
+// unit. A stage is [K | V] x [16 rows x D*2 bytes], each half starting on a
+// 1024-byte boundary; row t's unit h is unit t*D/64 + h, so the 8 rows of an
+// 8x8 ldmatrix tile hit 8 distinct bank groups at D = 64 and 4 (2-way) at
+// D = 128.
 //
 // Math per 16-token chunk in one warp, on tensor-core tiles (mma.sync
 // m16n8k16, fp32 accumulation); the G query heads are the M rows, padded to
@@ -50,8 +53,8 @@ namespace pagedkv {
 constexpr int kGroupMaxHeads = 16;
 
 struct GroupParams {
-    CUtensorMap tk; // key pool rows: dims (D, NB*Hkv*bs), box (64, min(bs, 16)), 128B swizzle
-    CUtensorMap tv; // value pool rows, same geometry
+    CUtensorMap tk; // key pool: dims (64, D/64, NB*Hkv*bs), box (64, D/64, min(bs, 16)), 128B swizzle
+    CUtensorMap tv; // value pool, same geometry
     DecodeParams p;
 };
 
@@ -59,9 +62,9 @@ template <int D, int BS, int NW, int NS> struct GroupCfg {
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
     static constexpr int kChunk = 16;                      // tokens per warp step
-    static constexpr int kSlabs = D / 64;                  // 128-byte column slabs per row
-    static constexpr int kSlabBytes = kChunk * 128;        // one slab of a stage: 2 KiB
-    static constexpr int kHalf = kSlabs * kSlabBytes;      // the K (or V) rows of a stage
+    static constexpr int kUnits = D / 64;                  // 128-byte units per row
+    static constexpr int kRow = D * 2;                     // bytes per row
+    static constexpr int kHalf = kChunk * kRow;            // the K (or V) rows of a stage
     static constexpr int kStage = 2 * kHalf;
     static constexpr int kRing = NS * kStage;              // one warp's stages
     static constexpr int kSeg = BS < kChunk ? BS : kChunk; // rows per TMA box
@@ -71,7 +74,7 @@ template <int D, int BS, int NW, int NS> struct GroupCfg {
     // After its last chunk a warp leaves (O, m, l) of its rows in its ring.
     static constexpr int kMergeStride = D + 2;
     static_assert(kGroupMaxHeads * kMergeStride * 4 <= kRing, "merge area fits a ring");
-    static_assert(kSlabBytes % 1024 == 0 && kStage % 1024 == 0, "swizzle atoms");
+    static_assert(kHalf % 1024 == 0 && (kSeg * kRow) % 1024 == 0, "swizzle atoms");
     // 1 KiB of slack to align the rings to 1024 bytes.
     static size_t smem_bytes(int partition)
     {
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(NW * 32)
 {
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     using Cfg = GroupCfg<D, BS, NW, NS>;
-    constexpr int CH = Cfg::kChunk, SLB = Cfg::kSlabBytes, SEG = Cfg::kSeg;
+    constexpr int CH = Cfg::kChunk, SEG = Cfg::kSeg, ROW = Cfg::kRow, U = Cfg::kUnits;
     constexpr int KT = D / 16; // k-steps of q.k = pairs of 8-wide d tiles of O
     constexpr int MS = Cfg::kMergeStride;
     constexpr unsigned FULL = 0xffffffffu;
@@ -214,7 +217,7 @@ __global__ void __launch_bounds__(NW * 32)
         const int st = i % NS;
         const uint32_t dk = ring_s + st * Cfg::kStage, dv = dk + Cfg::kHalf;
         const uint32_t bar = bar0 + st * 8;
-        mbar_arrive_expect_tx(bar, (uint32_t)(nseg * SEG * 128 * Cfg::kSlabs * 2));
+        mbar_arrive_expect_tx(bar, (uint32_t)(nseg * SEG * ROW * 2));
         for (int sg = 0; sg < nseg; ++sg) {
             const int tok = tok0 + sg * SEG;
             int b = table[tok / BS];
@@ -223,11 +226,8 @@ __global__ void __launch_bounds__(NW * 32)
                 b = 0;
             }
             const int y = (b * HK + kvh) * BS + tok % BS;
-#pragma unroll
-            for (int sl = 0; sl < Cfg::kSlabs; ++sl) {
-                tma_load_2d(dk + sl * SLB + sg * SEG * 128, &gp.tk, sl * 64, y, bar);
-                tma_load_2d(dv + sl * SLB + sg * SEG * 128, &gp.tv, sl * 64, y, bar);
-            }
+            tma_load_3d(dk + sg * SEG * ROW, &gp.tk, 0, 0, y, bar);
+            tma_load_3d(dv + sg * SEG * ROW, &gp.tv, 0, 0, y, bar);
         }
     };
 
@@ -241,8 +241,14 @@ __global__ void __launch_bounds__(NW * 32)
     // pieces c / c+1 / c / c+1, i.e. both k-halves of both token tiles.
     // V (transposed, B of O = P V): token rows 0-7 / 8-15 / 0-7 / 8-15 at
     // pieces c / c / c+1 / c+1, i.e. both token halves of two d tiles.
+    // Piece p (16 bytes, d = 8p..8p+7) of row t sits in unit t*U + p/8 at
+    // position (p % 8) ^ ((t*U + p/8) % 8).
     const int kt = (lane & 7) + ((lane >> 4) << 3), kc = (lane >> 3) & 1;
     const int vt = (lane & 7) + (((lane >> 3) & 1) << 3), vc = lane >> 4;
+    auto piece_off = [](int t, int piece) {
+        const int unit = t * U + (piece >> 3);
+        return unit * 128 + (((piece & 7) ^ (unit & 7)) << 4);
+    };
     const float qs = p.qk_scale_log2;
 
     int i = 0;
@@ -256,9 +262,7 @@ __global__ void __launch_bounds__(NW * 32)
         char *sv = sk + Cfg::kHalf;
         if (i == patch_i) { // warp-uniform
             if (lane < 2 * RV) {
-                const int piece = lane % RV, sl = piece >> 3, c = piece & 7;
-                char *dst = (lane >= RV ? sv : sk) + sl * SLB + patch_row * 128 +
-                            ((c ^ (patch_row & 7)) << 4);
+                char *dst = (lane >= RV ? sv : sk) + piece_off(patch_row, lane % RV);
                 *reinterpret_cast<uint4 *>(dst) = patch_val;
                 if (patch_dst)
                     *patch_dst = patch_val;
@@ -267,32 +271,33 @@ __global__ void __launch_bounds__(NW * 32)
             __syncwarp();
         }
         if (rows < CH) { // the partition's last chunk: zero the V rows past it
-            const int per_slab = (CH - rows) * 8;
-            for (int k = lane; k < Cfg::kSlabs * per_slab; k += 32) {
-                const int sl = k / per_slab, rem = k % per_slab;
-                *reinterpret_cast<uint4 *>(sv + sl * SLB + (rows + (rem >> 3)) * 128 +
-                                           ((rem & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
-            }
+            for (int k = rows * (ROW / 16) + lane; k < CH * (ROW / 16); k += 32)
+                reinterpret_cast<uint4 *>(sv)[k] = make_uint4(0u, 0u, 0u, 0u);
             fence_proxy_async_smem();
             __syncwarp();
         }
 
-        // S = Q K^T for the chunk's 16 tokens.
+        // S = Q K^T for the chunk's 16 tokens, even and odd k-steps in
+        // separate accumulators (two shorter dependency chains per tile).
         const uint32_t kb = smem_addr(sk), vb = smem_addr(sv);
-        float sc[2][4];
+        float sc[2][4], sd[2][4];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                sc[j][e] = 0.f;
+                sc[j][e] = sd[j][e] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < KT; ++kk) {
-            const int c = ((2 * kk) & 7) + kc;
             uint32_t b[4];
-            ldsm_x4(kb + (kk >> 2) * SLB + kt * 128 + ((c ^ (kt & 7)) << 4), b);
-            mma_16816<kBf16>(sc[0], qa[kk], b[0], b[1]);
-            mma_16816<kBf16>(sc[1], qa[kk], b[2], b[3]);
+            ldsm_x4(kb + piece_off(kt, 2 * kk + kc), b);
+            mma_16816<kBf16>(kk & 1 ? sd[0] : sc[0], qa[kk], b[0], b[1]);
+            mma_16816<kBf16>(kk & 1 ? sd[1] : sc[1], qa[kk], b[2], b[3]);
         }
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                sc[j][e] += sd[j][e];
 
         // Online softmax (base 2). sc[j][e]: token 8j + q2 + (e & 1), row g0
         // for e < 2, g1 otherwise.
@@ -334,13 +339,15 @@ __global__ void __launch_bounds__(NW * 32)
             for (int j = 0; j < 2; ++j)
                 pr[j][2] = pr[j][3] = 0.f;
         }
+        if (__any_sync(FULL, c0 != 1.f || c1 != 1.f)) { // a running max moved
 #pragma unroll
-        for (int j = 0; j < 2 * KT; ++j) {
-            o[j][0] *= c0;
-            o[j][1] *= c0;
-            if constexpr (TWO) {
-                o[j][2] *= c1;
-                o[j][3] *= c1;
+            for (int j = 0; j < 2 * KT; ++j) {
+                o[j][0] *= c0;
+                o[j][1] *= c0;
+                if constexpr (TWO) {
+                    o[j][2] *= c1;
+                    o[j][3] *= c1;
+                }
             }
         }
 
@@ -364,9 +371,8 @@ __global__ void __launch_bounds__(NW * 32)
         // O += P V, two 8-wide d tiles per transposed ldmatrix.
 #pragma unroll
         for (int dp = 0; dp < KT; ++dp) {
-            const int c = ((2 * dp) & 7) + vc;
             uint32_t b[4];
-            ldsm_x4_trans(vb + (dp >> 2) * SLB + vt * 128 + ((c ^ (vt & 7)) << 4), b);
+            ldsm_x4_trans(vb + piece_off(vt, 2 * dp + vc), b);
             mma_16816<kBf16>(o[2 * dp], pa, b[0], b[1]);
             mma_16816<kBf16>(o[2 * dp + 1], pa, b[2], b[3]);
             if constexpr (kBf16) {

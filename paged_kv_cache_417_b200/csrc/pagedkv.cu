@@ -38,11 +38,20 @@ constexpr int kSplitStages = PA_SPLIT_STAGES;
 #ifndef PA_GROUP_KERNEL
 #define PA_GROUP_KERNEL 1
 #endif
-constexpr int kGroupWarps = 4;
+#ifndef PA_GROUP_WARPS
+#define PA_GROUP_WARPS 4
+#endif
+constexpr int kGroupWarps = PA_GROUP_WARPS;
 constexpr int kGroupStages = 2;
 constexpr int kTargetCtasPerSm = 12; // ~4 waves of 3 resident CTAs
 constexpr int kMinAutoPartition = 128;
 constexpr int kAutoPartition = 2048;
+// The grouped kernel streams best in long partitions (B200 sweeps of 128 to
+// 2048 tokens at 2, 4 and 8 K/V heads: 1024 was fastest in every case), so
+// its automatic choice is 1024, halved (down to 256) only while the grid
+// would have fewer CTAs than the GPU has SMs.
+constexpr int kGroupAutoPartition = 1024;
+constexpr int kGroupMinAutoPartition = 256;
 constexpr int kPartitionQuantum = 32;
 constexpr int kMaxDevices = 64;
 
@@ -115,24 +124,23 @@ bool use_group_kernel(const pa_cache_desc *c, int32_t num_heads)
            rows <= INT32_MAX;
 }
 
-// CTA rows of a decode grid per partition: one per (sequence, query head),
-// or per (sequence, K/V head) for the grouped kernel.
-int64_t decode_units(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c)
-{
-    return (int64_t)num_seqs * (use_group_kernel(c, num_heads) ? c->num_kv_heads : num_heads);
-}
-
 // Partition (tokens per work unit) for a decode; >= max_context_len means a
-// single pass. Automatic choice: 2048 tokens, halved (down to 128) while the
-// grid of `units` CTA rows would give fewer than about four waves of
-// resident CTAs.
-int choose_partition(int64_t units, int32_t max_ctx, int32_t requested, int sm_count)
+// single pass. Automatic choice for decode_split_kernel (one CTA row per
+// (sequence, query head)): 2048 tokens, halved (down to 128) while the grid
+// would give fewer than about four waves of resident CTAs. For
+// decode_group_kernel (one CTA row per (sequence, K/V head)): 1024, halved
+// (down to 256) while the grid has fewer CTAs than SMs.
+int choose_partition(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c,
+                     int32_t max_ctx, int32_t requested, int sm_count)
 {
     int P = requested;
     if (P == 0) {
-        P = kAutoPartition;
-        while (P > kMinAutoPartition &&
-               units * ((max_ctx + P - 1) / P) < (int64_t)kTargetCtasPerSm * sm_count)
+        const bool grouped = use_group_kernel(c, num_heads);
+        const int64_t units = (int64_t)num_seqs * (grouped ? c->num_kv_heads : num_heads);
+        const int floor_p = grouped ? kGroupMinAutoPartition : kMinAutoPartition;
+        const int64_t target = (int64_t)(grouped ? 1 : kTargetCtasPerSm) * sm_count;
+        P = grouped ? kGroupAutoPartition : kAutoPartition;
+        while (P > floor_p && units * ((max_ctx + P - 1) / P) < target)
             P /= 2;
     }
     if (max_ctx <= P) {
@@ -238,9 +246,10 @@ pa_status dispatch_bs(const DecodeParams &p, int bs, cudaStream_t st)
     return fail(PA_ERR_UNSUPPORTED, "block_size %d", bs);
 }
 
-// The 2-D row view of a 16-bit pool that decode_group_kernel copies from:
-// rows of head_dim elements, boxes of 64 elements x min(block_size, 16) rows,
-// 128-byte swizzle. The encoder is the driver's, looked up once.
+// The row view of a 16-bit pool that decode_group_kernel copies from: dims
+// (64 elements, head_dim/64 128-byte units, rows), boxes of min(block_size,
+// 16) whole rows, 128-byte swizzle. The encoder is the driver's, looked up
+// once.
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -270,12 +279,13 @@ pa_status encode_pool_rows(CUtensorMap *map, const void *pool, const pa_cache_de
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc)
         return fail(PA_ERR_CUDA, "the driver has no cuTensorMapEncodeTiled");
-    const cuuint64_t dims[2] = {(cuuint64_t)c->head_dim,
+    const cuuint32_t units = (cuuint32_t)c->head_dim / 64;
+    const cuuint64_t dims[3] = {64, units,
                                 (cuuint64_t)c->num_blocks * c->num_kv_heads * c->block_size};
-    const cuuint64_t strides[1] = {(cuuint64_t)c->head_dim * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)std::min<int32_t>(c->block_size, 16)};
-    const cuuint32_t elem_strides[2] = {1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(pool), dims,
+    const cuuint64_t strides[2] = {128, (cuuint64_t)c->head_dim * 2};
+    const cuuint32_t box[3] = {64, units, (cuuint32_t)std::min<int32_t>(c->block_size, 16)};
+    const cuuint32_t elem_strides[3] = {1, 1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(pool), dims,
                            strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -465,8 +475,7 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
         num_heads % cache->num_kv_heads != 0 || max_context_len < 0 ||
         check_partition_request(partition_size) != PA_OK)
         return -1;
-    return choose_partition(decode_units(num_seqs, num_heads, cache), max_context_len,
-                            partition_size,
+    return choose_partition(num_seqs, num_heads, cache, max_context_len, partition_size,
                             partition_size == 0 ? sm_count_of_current_device() : 148);
 }
 
@@ -515,7 +524,7 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
     if (cache->num_blocks == 0 && max_context_len > 0)
         return fail(PA_ERR_INVALID_ARG, "empty pool with max_context_len %d", max_context_len);
 
-    const int P = choose_partition(decode_units(num_seqs, num_heads, cache), max_context_len,
+    const int P = choose_partition(num_seqs, num_heads, cache, max_context_len,
                                    partition_size, sm_count_of_current_device());
     const int64_t parts = max_context_len > P ? (max_context_len + P - 1) / P : 1;
     if (parts > 65535)
@@ -793,7 +802,7 @@ extern "C" pa_status pa_decode_noalloc(void *out, pa_dtype out_dtype, const void
     if (num_heads % cache->num_kv_heads != 0)
         return fail(PA_ERR_UNSUPPORTED, "num_heads %d is not a multiple of num_kv_heads %d",
                     num_heads, cache->num_kv_heads);
-    const int P = choose_partition(decode_units(num_seqs, num_heads, cache), max_context_len,
+    const int P = choose_partition(num_seqs, num_heads, cache, max_context_len,
                                    partition_size, sm_count_of_current_device());
     const int64_t parts = max_context_len > P ? (max_context_len + P - 1) / P : 1;
     if (parts > 1) {

@@ -99,6 +99,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int 
         : "memory");
 }
 
+// The same for a 3-D tensor map, coordinates (x, y, z).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int x, int y, int z,
+                                            uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
 // Four 8x8 tiles of 16-bit elements; lanes 8i..8i+7 give the row addresses
 // of tile i, register i receives it (.trans: transposed).
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])

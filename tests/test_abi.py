@@ -133,11 +133,14 @@ def test_workspace_and_partition_sizes(lib):
     assert lib.decode_partition_size(1, 32, desc(32), 32768, 0) == 512
     assert lib.decode_partition_size(96, 32, desc(32), 2048, 1024) == 1024
     assert lib.decode_partition_size(1, 1, desc(1), 30000, 0) == 128
-    # Grouped heads (G = 4) on a 16-bit cache: one CTA row per K/V head, so
-    # 96 x 8 rows need 4 partitions of 512 for four waves; the fp8 cache
-    # stays on one CTA row per query head.
-    assert lib.decode_partition_size(96, 32, desc(8), 2048, 0) == 512
-    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_BF16), 2048, 0) == 512
+    # Grouped heads (G = 4) on a 16-bit cache: one CTA row per K/V head,
+    # 1024-token partitions while the grid has at least one CTA per SM; the
+    # fp8 cache stays on one CTA row per query head.
+    assert lib.decode_partition_size(96, 32, desc(8), 2048, 0) == 1024
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_BF16), 2048, 0) == 1024
+    assert lib.decode_partition_size(96, 32, desc(8), 1000, 0) == 1024  # single pass
+    assert lib.decode_partition_size(1, 32, desc(8), 32768, 0) == 1024  # 8 x 32 CTAs
+    assert lib.decode_partition_size(1, 32, desc(8), 4096, 0) == 256  # 8 x 16 CTAs
     assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3), 2048, 0) == 2048
     with pytest.raises(ValueError):
         lib.decode_partition_size(96, 32, desc(7), 2048, 0)  # 32 % 7 != 0
