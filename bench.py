@@ -6,7 +6,7 @@ bandwidth on B200.
 
 A step is one decode step of the whole hot path on one batch: copy-on-write
 block copies (when the workload has any), the K/V write of every sequence's
-new token, and decode attention (plus its reduce when the context is split),
+new token, and decode attention (split partitions merged inside the same kernel),
 for every layer of the workload. The default workload is the Llama-7B-shaped
 single layer: 96 sequences, 32 heads, head_dim 128, block size 16, context
 lengths uniform in [128, 2048], an 8192-block pool.
@@ -56,7 +56,7 @@ WORKLOADS = {
                       "ctx U[128,2048], 8192-block pool, write_kv + decode"),
     "long_context": (lambda seed, dt="f16": wl.long_context(seed=seed, dtype=dt),
                      "long_context: 8 seqs, 32 heads, head_dim 128, block_size 16, "
-                     "ctx U[16384,32768], 20000-block pool, split decode + reduce"),
+                     "ctx U[16384,32768], 20000-block pool, split decode (partitions merged in-kernel)"),
     "prefix_cow": (lambda seed, dt="f16": wl.prefix_cow(seed=seed, dtype=dt),
                    "prefix_cow: 64 seqs sharing a 1024-token prefix, suffix U[1,512], "
                    "32 heads, head_dim 128, copy_blocks + write_kv + decode"),
@@ -423,9 +423,13 @@ def main():
     P = pk.decode_partition_size(S, step.num_heads, d["key_caches"][0], step.max_context_len,
                                  args.partition)
     split = step.max_context_len > P
+    # Split partitions are merged by the last CTA of each sequence, unless
+    # the grid has more (sequence, head) slots than the workspace has
+    # arrival counters (then a separate reduce kernel runs).
+    reduce_launch = split and S * step.num_heads > 65536
     has_copy = step.copy_pairs.shape[0] > 0
     launches_per_step = (1 if has_copy else 0) + L * ((1 if args.fused else 2) +
-                                                       (1 if split else 0))
+                                                       (1 if reduce_launch else 0))
     # L2 flush by reading 256 MiB: the previous step's lines are evicted and
     # L2 is left holding clean lines, so no write-back lands on the next step.
     flush_buf = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
@@ -582,7 +586,7 @@ def main():
                 "frac": achieved / peak, "traffic": recorded_traffic(traffic_key(args)),
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
-                "kernel": "pa_decode (decode kernel + reduce kernel when split)",
+                "kernel": "pa_decode (one decode kernel; split partitions merged in-kernel)",
                 "algorithmic_bytes_per_launch": ab["total"],
                 "kv_bytes_per_launch": ab["kv"],
                 "decode_us": dec_avg_s * 1e6,

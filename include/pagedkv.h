@@ -139,12 +139,16 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
  * partition_size  0 = automatic; else tokens per work unit, a positive
  *               multiple of 32 up to 8192. A sequence longer than it is split
  *               into partitions whose partial results (running max, sum and
- *               unnormalised output, fp32) go to the workspace and are merged
- *               by a second kernel with the log-sum-exp rule.
+ *               unnormalised output, fp32) go to the workspace; the last CTA
+ *               of a sequence to finish merges them with the log-sum-exp
+ *               rule (when num_seqs * num_heads > 65536, a second kernel).
  * workspace     device, >= pa_decode_workspace_size(...) bytes when that is
- *               non-zero (may be NULL otherwise). Its contents on entry do
- *               not matter; two calls sharing one workspace on different
- *               streams race.
+ *               non-zero (may be NULL otherwise). Its first 256 KiB hold
+ *               arrival counters that must be zero before the first call
+ *               that uses the workspace; every call leaves them zero
+ *               (zero-fill a new workspace once and keep it for this
+ *               library). The rest is scratch. Two calls sharing one
+ *               workspace on different streams race.
  * Accumulation is fp32 throughout. A block id outside the pool sets
  * PA_DEVERR_BLOCK_ID and makes that sequence's output NaN.
  */

@@ -225,8 +225,10 @@ def decode_partition_size(num_seqs, num_heads, cache, max_context_len, partition
 
 def alloc_workspace(num_seqs, num_heads, head_dim, max_context_len, partition_size=0,
                     device="cuda"):
+    """A decode workspace, zero-filled (its counter region must start at
+    zero; every call leaves it so)."""
     n = decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len, partition_size)
-    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
 
 
 def decode(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len,

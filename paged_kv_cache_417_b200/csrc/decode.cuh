@@ -8,8 +8,9 @@
 // A work unit is (sequence s, head h, partition p) = tokens
 // [p*P, min((p+1)*P, ctx)) of one (sequence, head). A sequence that fits one
 // partition is finished in place; a longer one leaves (running max, running
-// sum, unnormalised output) per partition in the workspace and
-// reduce_kernel merges them with the log-sum-exp rule.
+// sum, unnormalised output) per partition in the workspace, and the last of
+// its CTAs to finish merges them with the log-sum-exp rule (merge_if_last;
+// reduce_kernel does it when the workspace has no arrival counters).
 //
 // The K/V of a unit stream through shared memory in chunks of 4 KiB of K
 // rows (16 tokens at head_dim 128, 32 at 64) plus the matching V rows. Each
@@ -52,6 +53,7 @@ namespace pagedkv {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull; // 1 s: far above any copy latency
 constexpr int kMaxPartition = 8192;              // tokens per work unit, upper bound
+constexpr int kSplitCounters = 65536;            // arrival counters in a split workspace
 
 struct DecodeParams {
     void *out;
@@ -62,6 +64,10 @@ struct DecodeParams {
     const int32_t *context_lens;
     float *ws_acc; // [S][H][num_parts][D]
     float *ws_ml;  // [S][H][num_parts][2] = (max, sum), base-2 domain
+    // Arrival counters of split units, zero between calls: the last CTA of
+    // a split (sequence, head slot) merges its partitions. NULL: a separate
+    // reduce_kernel merges instead.
+    int32_t *ws_count;
     int32_t *dev_err;
     int32_t num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq, max_context_len;
     int32_t partition_size, num_parts;
@@ -591,6 +597,145 @@ template <typename T, typename QT, int D, int BS, int NS> struct WarpStream {
     }
 };
 
+// Merge partitions of query head h of sequence s (unit0 = its first
+// partial): M = max_p m_p, L = sum_p l_p 2^(m_p - M), out = sum_p o_p 2^(m_p
+// - M) / L. Loads bypass L1 (the partials were written by other CTAs).
+template <int D>
+__device__ __forceinline__ void merge_partitions(const DecodeParams &p, int s, int h, int d,
+                                                 int num_parts)
+{
+    const size_t unit0 = ((size_t)s * p.num_heads + h) * p.num_parts;
+    float M = -INFINITY;
+    for (int i = 0; i < num_parts; ++i)
+        M = fmaxf(M, __ldcg(&p.ws_ml[(unit0 + i) * 2]));
+    float L = 0.f, O = 0.f;
+    for (int i = 0; i < num_parts; ++i) {
+        const float f = exp2f(__ldcg(&p.ws_ml[(unit0 + i) * 2]) - M);
+        L = fmaf(__ldcg(&p.ws_ml[(unit0 + i) * 2 + 1]), f, L);
+        O = fmaf(__ldcg(&p.ws_acc[(unit0 + i) * D + d]), f, O);
+    }
+    store_out(p.out, p.out_dtype, ((size_t)s * p.num_heads + h) * D + d, O / L);
+}
+
+// Most output elements a thread merges in merge_if_last (16 heads x D 128
+// over 128 threads).
+constexpr int kMergeOutPerThread = 16;
+
+// Arrival on a split counter: an atomic add with acquire-release semantics
+// at GPU scope. Release publishes every write the CTA ordered before it
+// (its barrier); acquire lets the last arriver see all earlier arrivers'
+// writes.
+__device__ __forceinline__ int arrive_acq_rel(int32_t *counter)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
+                 : "=r"(old)
+                 : "l"(counter)
+                 : "memory");
+    return old;
+}
+
+// Called by every thread of a CTA that has just written the partials of
+// query heads h0 .. h0+nh-1 of sequence s: counts the CTA in on counter
+// `slot`; the CTA that completes the count (the last of the num_parts
+// partitions to finish) merges those heads into the output and resets the
+// counter to zero for the next call (the classic last-block pattern). The
+// merge turns each head's (m, l) pairs into normalised weights
+// 2^(m_p - M) / L in shared memory `wbuf` (nh * num_parts floats; one warp
+// per head, each lane holding up to kMergeLanePairs pairs, all heads' loads
+// issued before any reduction), then every thread sums its output elements
+// over the partitions with all loads of a partition issued together. The
+// host guarantees nh * num_parts <= the buffer and nh * D <=
+// kMergeOutPerThread * nthreads.
+constexpr int kMergeLanePairs = 4; // partitions per lane held in registers
+template <int D>
+__device__ __forceinline__ void merge_if_last(const DecodeParams &p, int s, int h0, int nh,
+                                              int slot, int num_parts, int tid, int nthreads,
+                                              int *flag, float *wbuf)
+{
+    __syncthreads();
+    if (tid == 0)
+        *flag = arrive_acq_rel(&p.ws_count[slot]) == num_parts - 1;
+    __syncthreads();
+    if (!*flag)
+        return;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads >> 5;
+    const float2 *ml0 = reinterpret_cast<const float2 *>(p.ws_ml) +
+                        ((size_t)s * p.num_heads + h0) * p.num_parts;
+    for (int g0 = warp; g0 < nh; g0 += nwarps * kMergeLanePairs) {
+        // Up to kMergeLanePairs heads per pass (g0, g0 + nwarps, ...), when
+        // every lane holds its partitions of them in registers; else one.
+        const bool fits = num_parts <= 32;
+        float2 v[kMergeLanePairs];
+#pragma unroll
+        for (int j = 0; j < kMergeLanePairs; ++j) {
+            const int g = g0 + j * nwarps;
+            v[j] = make_float2(-INFINITY, 0.f);
+            if (fits && g < nh && lane < num_parts)
+                v[j] = __ldcg(ml0 + (size_t)g * p.num_parts + lane);
+        }
+#pragma unroll
+        for (int j = 0; j < kMergeLanePairs; ++j) {
+            const int g = g0 + j * nwarps;
+            if (g >= nh || (!fits && j > 0))
+                continue; // warp-uniform
+            const float2 *ml = ml0 + (size_t)g * p.num_parts;
+            float M = v[j].x;
+            if (!fits)
+                for (int i = lane; i < num_parts; i += 32)
+                    M = fmaxf(M, __ldcg(ml + i).x);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            float L = lane < num_parts && fits ? v[j].y * exp2f(v[j].x - M) : 0.f;
+            if (!fits)
+                for (int i = lane; i < num_parts; i += 32) {
+                    const float2 q = __ldcg(ml + i);
+                    L = fmaf(q.y, exp2f(q.x - M), L);
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                L += __shfl_xor_sync(0xffffffffu, L, o);
+            if (fits) {
+                if (lane < num_parts)
+                    wbuf[g * num_parts + lane] = exp2f(v[j].x - M) / L;
+            } else {
+                for (int i = lane; i < num_parts; i += 32)
+                    wbuf[g * num_parts + i] = exp2f(__ldcg(ml + i).x - M) / L;
+            }
+        }
+        if (!fits)
+            g0 -= nwarps * (kMergeLanePairs - 1); // advance by one head per warp
+    }
+    __syncthreads();
+    float O[kMergeOutPerThread];
+#pragma unroll
+    for (int k = 0; k < kMergeOutPerThread; ++k)
+        O[k] = 0.f;
+    const float *acc0 = p.ws_acc + ((size_t)s * p.num_heads + h0) * p.num_parts * D;
+    for (int i = 0; i < num_parts; ++i) {
+#pragma unroll
+        for (int k = 0; k < kMergeOutPerThread; ++k) {
+            const int idx = tid + k * nthreads;
+            if (idx < nh * D) {
+                const int g = idx / D, d = idx - g * D;
+                O[k] = fmaf(__ldcg(acc0 + ((size_t)g * p.num_parts + i) * D + d),
+                            wbuf[g * num_parts + i], O[k]);
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kMergeOutPerThread; ++k) {
+        const int idx = tid + k * nthreads;
+        if (idx < nh * D) {
+            const int g = idx / D, d = idx - g * D;
+            store_out(p.out, p.out_dtype, ((size_t)s * p.num_heads + h0 + g) * D + d, O[k]);
+        }
+    }
+    if (tid == 0)
+        p.ws_count[slot] = 0;
+}
+
 // Shared prologue: read the context length and the partition's slice of the
 // block table at the same time (one global latency). Returns false when the
 // partition is past the sequence (the whole CTA returns).
@@ -784,10 +929,13 @@ __global__ void __launch_bounds__(NW * 32)
             }
         }
     }
+    if (u.num_parts > 1 && p.ws_count)
+        merge_if_last<D>(p, s, h, 1, s * H + h, u.num_parts, tid, NW * 32, &cta_flags,
+                         reinterpret_cast<float *>(rings));
 }
 
-// Merge the partitions of every split sequence:
-// M = max_p m_p, L = sum_p l_p 2^(m_p - M), out = sum_p o_p 2^(m_p - M) / L.
+// Separate merge kernel, for grids with more (sequence, head) slots than a
+// workspace holds counters: one CTA per (head, sequence).
 template <int D>
 __global__ void __launch_bounds__(D) reduce_kernel(const __grid_constant__ DecodeParams p,
                                                    int block_size)
@@ -799,17 +947,7 @@ __global__ void __launch_bounds__(D) reduce_kernel(const __grid_constant__ Decod
     const int num_parts = ctx > 0 ? (ctx + P - 1) / P : 1;
     if (num_parts <= 1)
         return;
-    const size_t unit0 = ((size_t)s * p.num_heads + h) * p.num_parts;
-    float M = -INFINITY;
-    for (int i = 0; i < num_parts; ++i)
-        M = fmaxf(M, p.ws_ml[(unit0 + i) * 2]);
-    float L = 0.f, O = 0.f;
-    for (int i = 0; i < num_parts; ++i) {
-        const float f = exp2f(p.ws_ml[(unit0 + i) * 2] - M);
-        L = fmaf(p.ws_ml[(unit0 + i) * 2 + 1], f, L);
-        O = fmaf(p.ws_acc[(unit0 + i) * D + d], f, O);
-    }
-    store_out(p.out, p.out_dtype, ((size_t)s * p.num_heads + h) * D + d, O / L);
+    merge_partitions<D>(p, s, h, d, num_parts);
 }
 
 } // namespace pagedkv

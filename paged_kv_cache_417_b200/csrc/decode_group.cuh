@@ -5,7 +5,9 @@
 // the unit (K/V head kvh, sequence s, partition p) for the whole group, so
 // each K/V byte crosses HBM once per group instead of once per query head,
 // and the G query rows share every staged tile. The outputs, the split
-// workspace and the reduce are those of decode_split_kernel (per query head).
+// workspace and the merge of partitions are those of decode_split_kernel
+// (per query head; the last CTA of a (K/V head, sequence) merges its G
+// heads).
 //
 // Staging: each pool is viewed as a tensor of rows (row = one token of one
 // (block, head) tile, D 16-bit elements; row index (block*Hkv + kvh)*bs +
@@ -465,6 +467,9 @@ __global__ void __launch_bounds__(NW * 32)
             }
         }
     }
+    if (u.num_parts > 1 && p.ws_count)
+        merge_if_last<D>(p, s, kvh * G, G, s * HK + kvh, u.num_parts, tid, NW * 32, &cta_flags,
+                         reinterpret_cast<float *>(rings));
 }
 
 } // namespace pagedkv

@@ -161,11 +161,21 @@ pa_status check_partition_request(int32_t partition_size)
     return PA_OK;
 }
 
+// Split workspace: [arrival counters, kSplitCounters int32][partial sums
+// acc, units*parts*D fp32, padded to 256 B][(max, sum) pairs]. The counter
+// region comes first and is used for nothing else, so it stays zero from
+// call to call whatever the shapes; it must be zero before the first call.
+constexpr size_t kCounterBytes = (size_t)kSplitCounters * sizeof(int32_t);
+// Floats of shared memory the merging CTA may use for weights: the smallest
+// ring area of any decode instantiation (fp8, head_dim 64: 8704 floats;
+// grouped, head_dim 64: 8192).
+constexpr int64_t kMergeWeights = 8192;
+
 size_t workspace_bytes_for(int64_t units, int64_t num_parts, int head_dim)
 {
     const size_t acc = (size_t)(units * num_parts * head_dim) * sizeof(float);
     const size_t acc_padded = (acc + 255) / 256 * 256;
-    return acc_padded + (size_t)(units * num_parts * 2) * sizeof(float);
+    return kCounterBytes + acc_padded + (size_t)(units * num_parts * 2) * sizeof(float);
 }
 
 // Raise a kernel's dynamic shared-memory limit once per device. `done` must
@@ -226,7 +236,7 @@ pa_status launch_decode(const DecodeParams &p, cudaStream_t stream)
                    Cfg::smem_bytes(p.partition_size), stream, p);
     if (e != cudaSuccess)
         return cuda_fail(e, "decode launch");
-    if (p.num_parts > 1) {
+    if (p.num_parts > 1 && !p.ws_count) {
         e = launch_pdl(reduce_kernel<D>, dim3(p.num_heads, p.num_seqs, 1), dim3(D), 0, stream, p,
                        (int)BS);
         if (e != cudaSuccess)
@@ -308,7 +318,7 @@ pa_status launch_group(const GroupParams &gp, cudaStream_t stream)
                    dim3(kGroupWarps * 32), Cfg::smem_bytes(p.partition_size), stream, gp);
     if (e != cudaSuccess)
         return cuda_fail(e, "group decode launch");
-    if (p.num_parts > 1) {
+    if (p.num_parts > 1 && !p.ws_count) {
         e = launch_pdl(reduce_kernel<D>, dim3(p.num_heads, p.num_seqs, 1), dim3(D), 0, stream, p,
                        (int)BS);
         if (e != cudaSuccess)
@@ -558,8 +568,17 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
         if (!aligned16(workspace))
             return fail(PA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
         const size_t acc = (size_t)(units * parts * cache->head_dim) * sizeof(float);
-        p.ws_acc = static_cast<float *>(workspace);
-        p.ws_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) + (acc + 255) / 256 * 256);
+        char *w = static_cast<char *>(workspace);
+        // Counter slots: (sequence, query head) for decode_split_kernel,
+        // (sequence, K/V head) for the grouped kernel; both < S * H. The
+        // merging CTA keeps one weight per (head, partition) in its ring
+        // memory (at least kMergeWeights floats in every instantiation).
+        const int64_t heads_per_cta =
+            use_group_kernel(cache, num_heads) ? num_heads / cache->num_kv_heads : 1;
+        const bool in_kernel = units <= kSplitCounters && heads_per_cta * parts <= kMergeWeights;
+        p.ws_count = in_kernel ? reinterpret_cast<int32_t *>(w) : nullptr;
+        p.ws_acc = reinterpret_cast<float *>(w + kCounterBytes);
+        p.ws_ml = reinterpret_cast<float *>(w + kCounterBytes + (acc + 255) / 256 * 256);
     }
     return dispatch_decode(p, cache, static_cast<cudaStream_t>(stream));
 }

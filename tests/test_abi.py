@@ -112,11 +112,12 @@ def test_workspace_and_partition_sizes(lib):
     # single pass: no workspace
     assert lib.decode_workspace_size(4, 4, 64, 100, 0) == 0
     assert lib.decode_workspace_size(4, 4, 64, 512, 512) == 0
-    # explicit partitions: acc [S,H,P,D] fp32 padded to 256 B, then (m, l) pairs
+    # explicit partitions: 65536 int32 arrival counters, acc [S,H,P,D] fp32
+    # padded to 256 B, then (m, l) pairs
     S, H, D, ctx, P = 3, 5, 128, 1000, 256
     parts = -(-ctx // P)
     acc = S * H * parts * D * 4
-    want = -(-acc // 256) * 256 + S * H * parts * 2 * 4
+    want = 65536 * 4 + -(-acc // 256) * 256 + S * H * parts * 2 * 4
     assert lib.decode_workspace_size(S, H, D, ctx, P) == want
     # automatic: a bound that covers the smallest automatic partition (128)
     assert lib.decode_workspace_size(S, H, D, ctx, 0) >= lib.decode_workspace_size(S, H, D, ctx,
