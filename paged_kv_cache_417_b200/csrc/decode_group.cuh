@@ -1,5 +1,7 @@
-// decode_group.cuh - paged decode attention for grouped query heads
-// (num_heads = G * num_kv_heads, 2 <= G <= 16, 16-bit caches) on sm_100a.
+// decode_group.cuh - paged decode attention on warp-level tensor-core tiles
+// for grouped query heads (num_heads = G * num_kv_heads, G <= 16) on
+// sm_100a: 16-bit caches, and fp8 (e4m3) caches with f16 rows and head_dim
+// 128 (2 <= G <= 16 for both; the kernel itself also handles G = 1).
 //
 // Query heads kvh*G .. kvh*G+G-1 all attend over K/V head kvh. A CTA takes
 // the unit (K/V head kvh, sequence s, partition p) for the whole group, so
@@ -9,41 +11,56 @@
 // (per query head; the last CTA of a (K/V head, sequence) merges its G
 // heads).
 //
-// Staging: each pool is viewed as a tensor of rows (row = one token of one
-// (block, head) tile, D 16-bit elements; row index (block*Hkv + kvh)*bs +
-// offset), each row split into D/64 128-byte units: dims (64 elements,
-// D/64 units, rows). A warp's stage receives 16 tokens of K and of V
-// through tiled TMA copies (cp.async.bulk.tensor) of min(bs, 16) whole rows
-// per box, contiguous in global memory, with the 128-byte swizzle: 16-byte
-// piece c of 128-byte unit u of the stage lands at piece c ^ (u % 8) of that
-// unit. A stage is [K | V] x [16 rows x D*2 bytes], each half starting on a
-// 1024-byte boundary; row t's unit h is unit t*D/64 + h, so the 8 rows of an
-// 8x8 ldmatrix tile hit 8 distinct bank groups at D = 64 and 4 (2-way) at
-// D = 128.
+// Staging: each pool is viewed as a 3-D tensor for the TMA unit. 16-bit
+// pools: (64 elements, D/64 128-byte units, rows), row = one token of one
+// (block, head) tile, row index (block*Hkv + kvh)*bs + offset. fp8 pools:
+// (D code bytes, bs rows, tiles), tile index block*Hkv + kvh, which steps
+// over the tile's row scales. A warp's stage receives CH tokens of K and of
+// V (16 at 16 bits, 32 at fp8: 8 KiB either way) through tiled copies
+// (cp.async.bulk.tensor) of min(bs, 16) whole rows per box with the 128-byte
+// swizzle: 16-byte piece c of 128-byte unit u of the stage lands at piece
+// c ^ (u % 8). fp8 row scales follow by 1-D bulk copies into a small
+// per-warp area. Every code area starts on a 1024-byte boundary; the 8 rows
+// of an 8x8 ldmatrix tile hit 8 distinct bank groups when a row is one unit
+// (fp8, 16-bit at D = 64) and 4 when it is two (2-way at D = 128).
 //
-// Math per 16-token chunk in one warp, on tensor-core tiles (mma.sync
-// m16n8k16, fp32 accumulation); the G query heads are the M rows, padded to
-// 16 with zeros (G <= 8 uses rows 0-7 only):
+// Math per 16-token step in one warp, on tensor-core tiles (mma.sync
+// m16n8k16, f16/bf16 operands, fp32 accumulation); the G query heads are the
+// M rows, padded to 16 with zeros (G <= 8 uses rows 0-7 only):
 //   S = Q K^T      2 column tiles of 8 tokens x D/16 k-steps, K tiles by
-//                  ldmatrix straight from the swizzled stage;
+//                  ldmatrix straight from the swizzled stage. fp8: a tile
+//                  register holds 4 consecutive codes of one token; they are
+//                  widened with the e4m3x2 -> f16x2 conversion into the two
+//                  halves of the B fragment, and the query's k order is
+//                  permuted the same way (any k order gives the same sum).
+//                  The token's K scale multiplies its score.
 //   online softmax in base 2 on the accumulator fragments: the 16 scores of
 //                  a row live in one quad of lanes (2 shuffles per max);
 //   O += P V       P goes from the S fragments into the A operand without
-//                  leaving registers; V tiles by ldmatrix.trans.
-// P is rounded to the cache's type for the product (the running sum keeps
+//                  leaving registers. 16-bit V tiles by ldmatrix.trans. fp8
+//                  V: ldmatrix cannot transpose bytes, so each 8x8 tile of
+//                  widened codes is transposed in registers (movmatrix); the
+//                  d columns then come out as {0,1,4,5,8,9,12,13} and
+//                  {2,3,6,7,10,11,14,15} of each 16, i.e. lane quad q holds
+//                  d = 16c + 4q .. 4q+3 of piece c. The token's V scale is
+//                  folded into P relative to the largest V scale met so far
+//                  (R): P' = p * s_v / R <= 1, so an f16 P' keeps its
+//                  precision however small the scales; O is rescaled when R
+//                  grows and multiplied by R at the end.
+// P is rounded to the operand type for the product (the running sum keeps
 // the fp32 weights). bf16 carries only 8 significant bits, so a bf16 P is
 // split into a bf16 head and a bf16 remainder and multiplied twice, which
 // keeps about 16 bits.
 //
-// Rows past the context: their scores are set to -inf (never computed from
-// the stale bytes), and the V rows of a partial last chunk are zeroed in
-// shared memory before the product, so a weight of 0 meets a finite value
-// (0 * NaN would otherwise reach the sum).
+// Rows past the context: their scores are set to -inf and their P' to 0
+// by selection (never computed from the stale bytes), and the V rows of a
+// partial last chunk are zeroed in shared memory before the product, so a
+// weight of 0 meets a finite value (0 * NaN would otherwise reach the sum).
 //
 // These tiles are warp-sized on purpose: the group is at most 16 rows,
 // below the 64-row minimum of a tcgen05 MMA, and the kernel is bound by HBM
-// bandwidth, so the tensor cores only have to remove the per-element FMA
-// and shuffle work of decode_split_kernel.
+// bandwidth, so the tensor cores only have to remove the per-element FMA,
+// conversion and shuffle work of decode_split_kernel.
 #pragma once
 
 #include <cuda.h> // CUtensorMap (type only; maps are encoded on the host)
@@ -55,28 +72,33 @@ namespace pagedkv {
 constexpr int kGroupMaxHeads = 16;
 
 struct GroupParams {
-    CUtensorMap tk; // key pool: dims (64, D/64, NB*Hkv*bs), box (64, D/64, min(bs, 16)), 128B swizzle
+    CUtensorMap tk; // key pool (see the staging note above), 128B swizzle
     CUtensorMap tv; // value pool, same geometry
     DecodeParams p;
 };
 
-template <int D, int BS, int NW, int NS> struct GroupCfg {
+template <typename T, int D, int BS, int NW, int NS> struct GroupCfg {
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
-    static constexpr int kChunk = 16;                      // tokens per warp step
-    static constexpr int kUnits = D / 64;                  // 128-byte units per row
-    static constexpr int kRow = D * 2;                     // bytes per row
-    static constexpr int kHalf = kChunk * kRow;            // the K (or V) rows of a stage
+    static constexpr bool kFp8 = std::is_same<T, E4M3>::value;
+    static_assert(!kFp8 || D == 128, "fp8 rows of 128 bytes");
+    static constexpr int kRow = D * (kFp8 ? 1 : 2);        // bytes per cached row
+    static constexpr int kUnits = kRow / 128;              // 128-byte units per row
+    static constexpr int kChunk = kFp8 ? 32 : 16;          // tokens per stage
+    static constexpr int kHalf = kChunk * kRow;            // the K (or V) codes of a stage
     static constexpr int kStage = 2 * kHalf;
     static constexpr int kRing = NS * kStage;              // one warp's stages
-    static constexpr int kSeg = BS < kChunk ? BS : kChunk; // rows per TMA box
+    static constexpr int kSeg = BS < 16 ? BS : 16;         // rows per TMA box
     static constexpr int kRingsBytes = NW * kRing;
     static constexpr int kBarBytes = NW * NS * 8;
-    static constexpr int kFixedBytes = kRingsBytes + kBarBytes;
+    // fp8 row scales: per warp, [stage][K | V][kChunk] floats.
+    static constexpr int kScaleBytes = kFp8 ? NW * NS * 2 * kChunk * 4 : 0;
+    static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kScaleBytes;
     // After its last chunk a warp leaves (O, m, l) of its rows in its ring.
     static constexpr int kMergeStride = D + 2;
     static_assert(kGroupMaxHeads * kMergeStride * 4 <= kRing, "merge area fits a ring");
     static_assert(kHalf % 1024 == 0 && (kSeg * kRow) % 1024 == 0, "swizzle atoms");
+    static_assert(kChunk % kSeg == 0 && kChunk % 16 == 0, "chunk geometry");
     // 1 KiB of slack to align the rings to 1024 bytes.
     static size_t smem_bytes(int partition)
     {
@@ -102,14 +124,33 @@ __device__ __forceinline__ float2 unpack_bf2(uint32_t u)
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-// T: __half or __nv_bfloat16 (cache, query and new-row type). TWO: G > 8
-// (fragment rows 8-15 are live).
+// Two e4m3 codes (low byte first) widened to an f16 pair (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two_codes)
+{
+    const __half2_raw h =
+        __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// Transpose of an 8x8 tile of 16-bit elements held as one register per lane
+// (lane l holds row l/4, columns 2(l%4), 2(l%4)+1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// T: __half, __nv_bfloat16 (cache, query and new-row type) or E4M3 (codes;
+// query and new rows are f16). TWO: G > 8 (fragment rows 8-15 are live).
 template <typename T, int D, int BS, int NW, int NS, bool TWO>
 __global__ void __launch_bounds__(NW * 32)
     decode_group_kernel(const __grid_constant__ GroupParams gp)
 {
+    using Cfg = GroupCfg<T, D, BS, NW, NS>;
+    constexpr bool kFp8 = Cfg::kFp8;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-    using Cfg = GroupCfg<D, BS, NW, NS>;
+    using QT = typename std::conditional<kFp8, __half, T>::type; // operand / row type
     constexpr int CH = Cfg::kChunk, SEG = Cfg::kSeg, ROW = Cfg::kRow, U = Cfg::kUnits;
     constexpr int KT = D / 16; // k-steps of q.k = pairs of 8-wide d tiles of O
     constexpr int MS = Cfg::kMergeStride;
@@ -120,6 +161,7 @@ __global__ void __launch_bounds__(NW * 32)
     unsigned char *smem = group_smem + ((1024u - (smem_addr(group_smem) & 1023u)) & 1023u);
     char *rings = reinterpret_cast<char *>(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kRingsBytes);
+    float *scales = reinterpret_cast<float *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes);
     int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
     __shared__ int cta_flags;
 
@@ -137,23 +179,26 @@ __global__ void __launch_bounds__(NW * 32)
     pdl_wait_prior_grid(); // every input may come from the previous kernel
 
     // Fragment coordinates: this lane holds rows g0 and g1 = g0 + 8 and, in
-    // every 8-wide column tile, columns q2 and q2 + 1.
-    const int g0 = lane >> 2, g1 = g0 + 8, q2 = 2 * (lane & 3);
+    // every 8-wide column tile, columns q2 and q2 + 1 (q = lane % 4).
+    const int g0 = lane >> 2, g1 = g0 + 8, q = lane & 3, q2 = 2 * q;
 
     // Q as the A operand, one 16x16 tile per k-step; rows >= G are zero.
+    // k-slots (2q, 2q+1) / (2q+8, 2q+9) hold d = 16kk + 2q (+1) / + 8 (+1);
+    // fp8: d = 16kk + 4q (+1) / + 2 (+1), matching the widened K codes.
     // Loaded before the block table so that the two reads overlap.
     uint32_t qa[KT][4];
     {
-        const uint32_t *q = static_cast<const uint32_t *>(p.query); // element pairs
+        const uint32_t *qp = static_cast<const uint32_t *>(p.query); // element pairs
         const size_t r0 = ((size_t)s * H + (size_t)kvh * G + g0) * (D / 2);
         const size_t r1 = r0 + (size_t)8 * (D / 2);
 #pragma unroll
         for (int kk = 0; kk < KT; ++kk) {
-            const int c = (16 * kk + q2) / 2;
-            qa[kk][0] = g0 < G ? q[r0 + c] : 0u;
-            qa[kk][1] = TWO && g1 < G ? q[r1 + c] : 0u;
-            qa[kk][2] = g0 < G ? q[r0 + c + 4] : 0u;
-            qa[kk][3] = TWO && g1 < G ? q[r1 + c + 4] : 0u;
+            const int c = kFp8 ? (16 * kk + 4 * q) / 2 : (16 * kk + q2) / 2;
+            const int c2 = kFp8 ? c + 1 : c + 4;
+            qa[kk][0] = g0 < G ? qp[r0 + c] : 0u;
+            qa[kk][1] = TWO && g1 < G ? qp[r1 + c] : 0u;
+            qa[kk][2] = g0 < G ? qp[r0 + c2] : 0u;
+            qa[kk][3] = TWO && g1 < G ? qp[r1 + c2] : 0u;
         }
     }
 
@@ -164,54 +209,97 @@ __global__ void __launch_bounds__(NW * 32)
         return; // uniform across the CTA
     __syncthreads();
 
-    float o[2 * KT][4]; // 8-wide d tile j: d = 8j + q2 (+1); rows g0 (0, 1), g1 (2, 3)
+    // O tile j covers 8 d: 16-bit d = 8j + q2 (+1); fp8 d = 16(j/2) +
+    // 4q + 2(j%2) (+1). Elements 0, 1: row g0; 2, 3: row g1.
+    auto dcol = [&](int j) { return kFp8 ? 16 * (j >> 1) + 4 * q + 2 * (j & 1) : 8 * j + q2; };
+    float o[2 * KT][4];
 #pragma unroll
     for (int j = 0; j < 2 * KT; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             o[j][e] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float vref = 1.17549435e-38f; // fp8: largest V scale so far (R), floored at FLT_MIN
 
     const int n_chunks = (u.n_tok + CH - 1) / CH;
     const int my_chunks = n_chunks <= warp ? 0 : (n_chunks - warp + NW - 1) / NW;
     char *ring = rings + (size_t)warp * Cfg::kRing;
     const uint32_t ring_s = smem_addr(ring);
     const uint32_t bar0 = smem_addr(&bars[warp * NS]);
+    float *wscales = scales + (size_t)warp * NS * 2 * CH; // fp8: [stage][K | V][CH]
 
     // Fused append: the warp owning the chunk of the sequence's last token
     // puts the new K/V row into that chunk once it has landed, and into the
-    // cache. Lanes [0, D/8) carry 16 bytes of the K row each, the next D/8
-    // lanes the V row.
-    constexpr int RV = D / 8;
+    // cache. Lanes [0, RV) carry 16 bytes of the stored K row each, the next
+    // RV lanes the V row (fp8: 16 codes quantised from 16 inputs, with the
+    // row scale amax / 448 on every lane of the half).
+    constexpr int RV = ROW / 16;
     int patch_i = -1, patch_row = 0;
     uint4 patch_val = make_uint4(0u, 0u, 0u, 0u);
+    float patch_scale = 0.f;
     uint4 *patch_dst = nullptr;
+    float *patch_sdst = nullptr;
     if (p.new_key != nullptr && part == u.num_parts - 1 && u.n_tok > 0) {
         const int c_last = (u.n_tok - 1) / CH;
         if (c_last % NW == warp) { // warp-uniform
             patch_i = c_last / NW;
             patch_row = (u.n_tok - 1) - c_last * CH;
+            const bool isv = lane >= RV;
+            const int piece = lane % RV;
+            constexpr int EPL = kFp8 ? 16 : 8; // inputs per lane
+            const QT *src = static_cast<const QT *>(isv ? p.new_value : p.new_key) +
+                            ((size_t)s * HK + kvh) * D + (size_t)piece * EPL;
+            if constexpr (kFp8) {
+                // codes = e4m3(x * (448 / amax)), scale = amax / 448.
+                float x[16];
+                float amax = 0.f;
+                if (lane < 2 * RV) {
+                    unpack8_to<QT>(*reinterpret_cast<const uint4 *>(src), x);
+                    unpack8_to<QT>(*reinterpret_cast<const uint4 *>(src + 8), x + 8);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        amax = fmaxf(amax, fabsf(x[e]));
+                }
+#pragma unroll
+                for (int o2 = 1; o2 < RV; o2 <<= 1)
+                    amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o2));
+                if (lane < 2 * RV) {
+                    const float inv = amax > 0.f ? 448.f / amax : 0.f;
+                    patch_val = quantize16_e4m3(x, inv);
+                    patch_scale = amax / 448.f;
+                }
+            } else {
+                if (lane < 2 * RV)
+                    patch_val = *reinterpret_cast<const uint4 *>(src);
+            }
             if (lane < 2 * RV) {
-                const bool isv = lane >= RV;
-                const int piece = lane % RV;
-                const T *src = static_cast<const T *>(isv ? p.new_value : p.new_key) +
-                               ((size_t)s * HK + kvh) * D + (size_t)piece * 8;
-                patch_val = *reinterpret_cast<const uint4 *>(src);
                 const int b = table[(u.n_tok - 1) / BS];
                 if (b >= 0 && b < p.num_blocks) {
                     char *cache = const_cast<char *>(
                         static_cast<const char *>(isv ? p.value_cache : p.key_cache));
-                    const size_t row = ((size_t)b * HK + kvh) * BS + (u.n_tok - 1) % BS;
-                    patch_dst = reinterpret_cast<uint4 *>(cache + row * (D * 2)) + piece;
+                    const size_t tile = (size_t)b * HK + kvh;
+                    const int off = (u.n_tok - 1) % BS;
+                    if constexpr (kFp8) {
+                        char *t0 = cache + tile * (size_t)(BS * (D + 4));
+                        patch_dst = reinterpret_cast<uint4 *>(t0 + (size_t)off * D) + piece;
+                        if (piece == 0)
+                            patch_sdst = reinterpret_cast<float *>(t0 + BS * D) + off;
+                    } else {
+                        patch_dst = reinterpret_cast<uint4 *>(
+                                        cache + (tile * BS + off) * (size_t)(D * 2)) +
+                                    piece;
+                    }
                 }
             }
         }
     }
 
-    // Lane 0: the TMA boxes of local chunk i (global chunk warp + i*NW).
-    // Boxes that start past the context are not fetched; a block id outside
-    // the pool is replaced by block 0 and recorded.
+    // Lane 0: the copies of local chunk i (global chunk warp + i*NW). Boxes
+    // that start past the context are not fetched; a block id outside the
+    // pool is replaced by block 0 and recorded.
     int bad_id = 0;
+    const char *kpool = static_cast<const char *>(p.key_cache);
+    const char *vpool = static_cast<const char *>(p.value_cache);
     auto issue = [&](int i) {
         const int tok0 = (warp + i * NW) * CH;
         const int rows = min(CH, u.n_tok - tok0);
@@ -219,7 +307,7 @@ __global__ void __launch_bounds__(NW * 32)
         const int st = i % NS;
         const uint32_t dk = ring_s + st * Cfg::kStage, dv = dk + Cfg::kHalf;
         const uint32_t bar = bar0 + st * 8;
-        mbar_arrive_expect_tx(bar, (uint32_t)(nseg * SEG * ROW * 2));
+        mbar_arrive_expect_tx(bar, (uint32_t)(nseg * SEG * (ROW + (kFp8 ? 4 : 0)) * 2));
         for (int sg = 0; sg < nseg; ++sg) {
             const int tok = tok0 + sg * SEG;
             int b = table[tok / BS];
@@ -227,9 +315,20 @@ __global__ void __launch_bounds__(NW * 32)
                 bad_id = 1;
                 b = 0;
             }
-            const int y = (b * HK + kvh) * BS + tok % BS;
-            tma_load_3d(dk + sg * SEG * ROW, &gp.tk, 0, 0, y, bar);
-            tma_load_3d(dv + sg * SEG * ROW, &gp.tv, 0, 0, y, bar);
+            const int tile = b * HK + kvh;
+            if constexpr (kFp8) {
+                const int off = tok % BS;
+                tma_load_3d(dk + sg * SEG * ROW, &gp.tk, 0, off, tile, bar);
+                tma_load_3d(dv + sg * SEG * ROW, &gp.tv, 0, off, tile, bar);
+                const size_t sofs = (size_t)tile * (BS * (D + 4)) + BS * D + (size_t)off * 4;
+                float *sk = wscales + (st * 2) * CH + sg * SEG;
+                bulk_g2s(smem_addr(sk), kpool + sofs, SEG * 4, bar);
+                bulk_g2s(smem_addr(sk + CH), vpool + sofs, SEG * 4, bar);
+            } else {
+                const int y = tile * BS + tok % BS;
+                tma_load_3d(dk + sg * SEG * ROW, &gp.tk, 0, 0, y, bar);
+                tma_load_3d(dv + sg * SEG * ROW, &gp.tv, 0, 0, y, bar);
+            }
         }
     };
 
@@ -238,14 +337,16 @@ __global__ void __launch_bounds__(NW * 32)
             issue(i);
     int issued = min(NS, my_chunks);
 
-    // ldmatrix row addresses. K (non-transposed, B of S = Q K^T): lanes
-    // 0-7 / 8-15 / 16-23 / 24-31 give token rows 0-7 / 0-7 / 8-15 / 8-15 at
-    // pieces c / c+1 / c / c+1, i.e. both k-halves of both token tiles.
-    // V (transposed, B of O = P V): token rows 0-7 / 8-15 / 0-7 / 8-15 at
-    // pieces c / c / c+1 / c+1, i.e. both token halves of two d tiles.
-    // Piece p (16 bytes, d = 8p..8p+7) of row t sits in unit t*U + p/8 at
-    // position (p % 8) ^ ((t*U + p/8) % 8).
-    const int kt = (lane & 7) + ((lane >> 4) << 3), kc = (lane >> 3) & 1;
+    // ldmatrix row addresses (rows within a 16-token step). 16-bit K
+    // (non-transposed, B of S = Q K^T): lanes 0-7 / 8-15 / 16-23 / 24-31
+    // give token rows 0-7 / 0-7 / 8-15 / 8-15 at pieces c / c+1 / c / c+1.
+    // 16-bit V (transposed, B of O = P V): rows 0-7 / 8-15 / 0-7 / 8-15 at
+    // pieces c / c / c+1 / c+1. fp8 K and V (non-transposed): rows 0-7 /
+    // 8-15 / 0-7 / 8-15 at pieces c / c / c+1 / c+1, register = (token tile,
+    // piece). Piece p (16 bytes) of row t sits in unit t*U + p/8 at position
+    // (p % 8) ^ ((t*U + p/8) % 8).
+    const int kt = kFp8 ? (lane & 7) + (((lane >> 3) & 1) << 3) : (lane & 7) + ((lane >> 4) << 3);
+    const int kc = kFp8 ? lane >> 4 : (lane >> 3) & 1;
     const int vt = (lane & 7) + (((lane >> 3) & 1) << 3), vc = lane >> 4;
     auto piece_off = [](int t, int piece) {
         const int unit = t * U + (piece >> 3);
@@ -262,13 +363,23 @@ __global__ void __launch_bounds__(NW * 32)
         const int rows = min(CH, u.n_tok - (warp + i * NW) * CH);
         char *sk = ring + st * Cfg::kStage;
         char *sv = sk + Cfg::kHalf;
+        const float *ksc = wscales + (st * 2) * CH; // fp8 scales of the stage
+        const float *vsc = ksc + CH;
         if (i == patch_i) { // warp-uniform
             if (lane < 2 * RV) {
-                char *dst = (lane >= RV ? sv : sk) + piece_off(patch_row, lane % RV);
+                const bool isv = lane >= RV;
+                char *dst = (isv ? sv : sk) + piece_off(patch_row, lane % RV);
                 *reinterpret_cast<uint4 *>(dst) = patch_val;
                 if (patch_dst)
                     *patch_dst = patch_val;
-                fence_proxy_async_smem();
+                if constexpr (kFp8) {
+                    if (lane % RV == 0) {
+                        const_cast<float *>(isv ? vsc : ksc)[patch_row] = patch_scale;
+                        if (patch_sdst)
+                            *patch_sdst = patch_scale;
+                    }
+                }
+                fence_proxy_async_smem(); // before the stage is refilled by a copy
             }
             __syncwarp();
         }
@@ -279,107 +390,188 @@ __global__ void __launch_bounds__(NW * 32)
             __syncwarp();
         }
 
-        // S = Q K^T for the chunk's 16 tokens, even and odd k-steps in
-        // separate accumulators (two shorter dependency chains per tile).
-        const uint32_t kb = smem_addr(sk), vb = smem_addr(sv);
-        float sc[2][4], sd[2][4];
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                sc[j][e] = sd[j][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < KT; ++kk) {
-            uint32_t b[4];
-            ldsm_x4(kb + piece_off(kt, 2 * kk + kc), b);
-            mma_16816<kBf16>(kk & 1 ? sd[0] : sc[0], qa[kk], b[0], b[1]);
-            mma_16816<kBf16>(kk & 1 ? sd[1] : sc[1], qa[kk], b[2], b[3]);
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                sc[j][e] += sd[j][e];
+        for (int sub = 0; sub < CH / 16; ++sub) {
+            const int srows = rows - 16 * sub; // valid tokens of this step
+            if (srows <= 0)
+                break; // warp-uniform
+            const int t0 = 16 * sub;
 
-        // Online softmax (base 2). sc[j][e]: token 8j + q2 + (e & 1), row g0
-        // for e < 2, g1 otherwise.
-        float x[2][4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                x[j][e] = 8 * j + q2 + (e & 1) < rows ? sc[j][e] * qs : -INFINITY;
-        float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 2));
-        const float mn0 = fmaxf(m0, mx0); // finite: token 0 of a chunk is always valid
-        const float c0 = exp2f(m0 - mn0);
-        m0 = mn0;
-        float pr[2][4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            pr[j][0] = exp2f(x[j][0] - mn0);
-            pr[j][1] = exp2f(x[j][1] - mn0);
-        }
-        l0 = fmaf(l0, c0, (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
-        float c1 = 1.f;
-        if constexpr (TWO) {
-            float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
-            const float mn1 = fmaxf(m1, mx1);
-            c1 = exp2f(m1 - mn1);
-            m1 = mn1;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                pr[j][2] = exp2f(x[j][2] - mn1);
-                pr[j][3] = exp2f(x[j][3] - mn1);
-            }
-            l1 = fmaf(l1, c1, (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]));
-        } else {
+            // S = Q K^T for the step's 16 tokens, even and odd k-steps in
+            // separate accumulators (two shorter dependency chains per tile).
+            const uint32_t kb = smem_addr(sk), vb = smem_addr(sv);
+            float sc[2][4], sd[2][4];
 #pragma unroll
             for (int j = 0; j < 2; ++j)
-                pr[j][2] = pr[j][3] = 0.f;
-        }
-        if (__any_sync(FULL, c0 != 1.f || c1 != 1.f)) { // a running max moved
 #pragma unroll
-            for (int j = 0; j < 2 * KT; ++j) {
-                o[j][0] *= c0;
-                o[j][1] *= c0;
-                if constexpr (TWO) {
-                    o[j][2] *= c1;
-                    o[j][3] *= c1;
+                for (int e = 0; e < 4; ++e)
+                    sc[j][e] = sd[j][e] = 0.f;
+            if constexpr (kFp8) {
+#pragma unroll
+                for (int kp = 0; kp < KT / 2; ++kp) { // pieces 2kp, 2kp+1
+                    uint32_t r[4];
+                    ldsm_x4(kb + piece_off(t0 + kt, 2 * kp + kc), r);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int kk = 2 * kp + h;
+                        float(&acc0)[4] = h ? sd[0] : sc[0];
+                        float(&acc1)[4] = h ? sd[1] : sc[1];
+                        mma_16816<false>(acc0, qa[kk], e4m3x2_to_h2(r[2 * h]),
+                                         e4m3x2_to_h2(r[2 * h] >> 16));
+                        mma_16816<false>(acc1, qa[kk], e4m3x2_to_h2(r[2 * h + 1]),
+                                         e4m3x2_to_h2(r[2 * h + 1] >> 16));
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < KT; ++kk) {
+                    uint32_t b[4];
+                    ldsm_x4(kb + piece_off(t0 + kt, 2 * kk + kc), b);
+                    mma_16816<kBf16>(kk & 1 ? sd[0] : sc[0], qa[kk], b[0], b[1]);
+                    mma_16816<kBf16>(kk & 1 ? sd[1] : sc[1], qa[kk], b[2], b[3]);
                 }
             }
-        }
-
-        // P as the A operand (16 rows x 16 tokens): the S fragment layout of
-        // the two token tiles is exactly the A fragment layout.
-        uint32_t pa[4];
-        pa[0] = pack2<T>(pr[0][0], pr[0][1]);
-        pa[1] = pack2<T>(pr[0][2], pr[0][3]);
-        pa[2] = pack2<T>(pr[1][0], pr[1][1]);
-        pa[3] = pack2<T>(pr[1][2], pr[1][3]);
-        uint32_t pl[4]; // bf16: the remainder P - bf16(P)
-        if constexpr (kBf16) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int j = k >> 1, e = (k & 1) * 2;
-                const float2 h = unpack_bf2(pa[k]);
-                pl[k] = pack2<T>(pr[j][e] - h.x, pr[j][e + 1] - h.y);
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    sc[j][e] += sd[j][e];
+
+            // Online softmax (base 2). sc[j][e]: token t0 + 8j + q2 + (e & 1),
+            // row g0 for e < 2, g1 otherwise.
+            float x[2][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float2 ks = make_float2(qs, qs);
+                if constexpr (kFp8) {
+                    const float2 k2 = *reinterpret_cast<const float2 *>(ksc + t0 + 8 * j + q2);
+                    ks = make_float2(k2.x * qs, k2.y * qs);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    x[j][e] = 8 * j + q2 + (e & 1) < srows ? sc[j][e] * ((e & 1) ? ks.y : ks.x)
+                                                            : -INFINITY;
             }
-        }
-
-        // O += P V, two 8-wide d tiles per transposed ldmatrix.
+            float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 2));
+            const float mn0 = fmaxf(m0, mx0); // finite: token 0 of a step is always valid
+            const float c0 = exp2f(m0 - mn0);
+            m0 = mn0;
+            float pr[2][4];
 #pragma unroll
-        for (int dp = 0; dp < KT; ++dp) {
-            uint32_t b[4];
-            ldsm_x4_trans(vb + piece_off(vt, 2 * dp + vc), b);
-            mma_16816<kBf16>(o[2 * dp], pa, b[0], b[1]);
-            mma_16816<kBf16>(o[2 * dp + 1], pa, b[2], b[3]);
+            for (int j = 0; j < 2; ++j) {
+                pr[j][0] = exp2f(x[j][0] - mn0);
+                pr[j][1] = exp2f(x[j][1] - mn0);
+            }
+            l0 = fmaf(l0, c0, (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
+            float c1 = 1.f;
+            if constexpr (TWO) {
+                float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
+                const float mn1 = fmaxf(m1, mx1);
+                c1 = exp2f(m1 - mn1);
+                m1 = mn1;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    pr[j][2] = exp2f(x[j][2] - mn1);
+                    pr[j][3] = exp2f(x[j][3] - mn1);
+                }
+                l1 = fmaf(l1, c1, (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]));
+            } else {
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+                    pr[j][2] = pr[j][3] = 0.f;
+            }
+            float cr = 1.f; // fp8: R_old / R_new
+            if constexpr (kFp8) {
+                // Fold the V scales into P relative to R (tokens past the
+                // context get P' = 0 by selection).
+                float vs[2][2];
+                float vmax = 0.f;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float2 v2 = *reinterpret_cast<const float2 *>(vsc + t0 + 8 * j + q2);
+                    vs[j][0] = 8 * j + q2 < srows ? v2.x : 0.f;
+                    vs[j][1] = 8 * j + q2 + 1 < srows ? v2.y : 0.f;
+                    vmax = fmaxf(vmax, fmaxf(vs[j][0], vs[j][1]));
+                }
+                vmax = fmaxf(vmax, __shfl_xor_sync(FULL, vmax, 1));
+                vmax = fmaxf(vmax, __shfl_xor_sync(FULL, vmax, 2));
+                const float rn = fmaxf(vref, vmax);
+                cr = vref / rn;
+                vref = rn;
+                const float inv = 1.f / rn;
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        pr[j][e] = 8 * j + q2 + (e & 1) < srows ? pr[j][e] * (vs[j][e & 1] * inv)
+                                                                : 0.f;
+            }
+            if (__any_sync(FULL, c0 != 1.f || c1 != 1.f || cr != 1.f)) { // a max moved
+                const float f0 = c0 * cr, f1 = c1 * cr;
+#pragma unroll
+                for (int j = 0; j < 2 * KT; ++j) {
+                    o[j][0] *= f0;
+                    o[j][1] *= f0;
+                    if constexpr (TWO) {
+                        o[j][2] *= f1;
+                        o[j][3] *= f1;
+                    }
+                }
+            }
+
+            // P as the A operand (16 rows x 16 tokens): the S fragment layout
+            // of the two token tiles is exactly the A fragment layout.
+            uint32_t pa[4];
+            pa[0] = pack2<QT>(pr[0][0], pr[0][1]);
+            pa[1] = pack2<QT>(pr[0][2], pr[0][3]);
+            pa[2] = pack2<QT>(pr[1][0], pr[1][1]);
+            pa[3] = pack2<QT>(pr[1][2], pr[1][3]);
+            uint32_t pl[4]; // bf16: the remainder P - bf16(P)
             if constexpr (kBf16) {
-                mma_16816<kBf16>(o[2 * dp], pl, b[0], b[1]);
-                mma_16816<kBf16>(o[2 * dp + 1], pl, b[2], b[3]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int j = k >> 1, e = (k & 1) * 2;
+                    const float2 hh = unpack_bf2(pa[k]);
+                    pl[k] = pack2<T>(pr[j][e] - hh.x, pr[j][e + 1] - hh.y);
+                }
+            }
+
+            if constexpr (kFp8) {
+                // O += P V: per pair of pieces, widen the codes and transpose
+                // each 8x8 half-tile in registers. r[0] / r[1]: token tiles
+                // 0 / 1 of piece 2kp, r[2] / r[3]: of piece 2kp + 1.
+#pragma unroll
+                for (int kp = 0; kp < KT / 2; ++kp) {
+                    uint32_t r[4];
+                    ldsm_x4(vb + piece_off(t0 + vt, 2 * kp + vc), r);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int c = 2 * kp + h; // piece: d = 16c .. 16c + 15
+                        const uint32_t lo0 = movmatrix_trans(e4m3x2_to_h2(r[2 * h]));
+                        const uint32_t lo1 = movmatrix_trans(e4m3x2_to_h2(r[2 * h + 1]));
+                        const uint32_t hi0 = movmatrix_trans(e4m3x2_to_h2(r[2 * h] >> 16));
+                        const uint32_t hi1 = movmatrix_trans(e4m3x2_to_h2(r[2 * h + 1] >> 16));
+                        mma_16816<false>(o[2 * c], pa, lo0, lo1);
+                        mma_16816<false>(o[2 * c + 1], pa, hi0, hi1);
+                    }
+                }
+            } else {
+                // O += P V, two 8-wide d tiles per transposed ldmatrix.
+#pragma unroll
+                for (int dp = 0; dp < KT; ++dp) {
+                    uint32_t b[4];
+                    ldsm_x4_trans(vb + piece_off(t0 + vt, 2 * dp + vc), b);
+                    mma_16816<kBf16>(o[2 * dp], pa, b[0], b[1]);
+                    mma_16816<kBf16>(o[2 * dp + 1], pa, b[2], b[3]);
+                    if constexpr (kBf16) {
+                        mma_16816<kBf16>(o[2 * dp], pl, b[0], b[1]);
+                        mma_16816<kBf16>(o[2 * dp + 1], pl, b[2], b[3]);
+                    }
+                }
             }
         }
         __syncwarp();
@@ -404,17 +596,20 @@ __global__ void __launch_bounds__(NW * 32)
             atomicOr(&cta_flags, 1);
     }
 
-    // Row sums over the quad; then this warp's (O, m, l) into its ring.
+    // Row sums over the quad; then this warp's (O, m, l) into its ring (fp8:
+    // O back in the scale of the codes' values, times R).
     l0 += __shfl_xor_sync(FULL, l0, 1);
     l0 += __shfl_xor_sync(FULL, l0, 2);
     l1 += __shfl_xor_sync(FULL, l1, 1);
     l1 += __shfl_xor_sync(FULL, l1, 2);
+    const float oscale = kFp8 ? vref : 1.f;
     __syncwarp();
     float *mw = reinterpret_cast<float *>(ring);
     if (g0 < G) {
 #pragma unroll
         for (int j = 0; j < 2 * KT; ++j)
-            *reinterpret_cast<float2 *>(mw + g0 * MS + 8 * j + q2) = make_float2(o[j][0], o[j][1]);
+            *reinterpret_cast<float2 *>(mw + g0 * MS + dcol(j)) =
+                make_float2(o[j][0] * oscale, o[j][1] * oscale);
         if ((lane & 3) == 0) {
             mw[g0 * MS + D] = m0;
             mw[g0 * MS + D + 1] = l0;
@@ -424,8 +619,8 @@ __global__ void __launch_bounds__(NW * 32)
         if (g1 < G) {
 #pragma unroll
             for (int j = 0; j < 2 * KT; ++j)
-                *reinterpret_cast<float2 *>(mw + g1 * MS + 8 * j + q2) =
-                    make_float2(o[j][2], o[j][3]);
+                *reinterpret_cast<float2 *>(mw + g1 * MS + dcol(j)) =
+                    make_float2(o[j][2] * oscale, o[j][3] * oscale);
             if ((lane & 3) == 0) {
                 mw[g1 * MS + D] = m1;
                 mw[g1 * MS + D + 1] = l1;

@@ -124,9 +124,8 @@ def test_workspace_and_partition_sizes(lib):
                                                                                    128)
     with pytest.raises(ValueError):
         lib.decode_workspace_size(S, H, D, ctx, 40)
-    def desc(hkv, dtype=lib.PA_F16, nb=8192, d=128, bs=16):
-        return lib.CacheDesc(nb, bs, hkv, d, dtype, dtype if dtype != lib.PA_FP8_E4M3
-                             else lib.PA_F16)
+    def desc(hkv, dtype=lib.PA_F16, nb=8192, d=128, bs=16, io=lib.PA_F16):
+        return lib.CacheDesc(nb, bs, hkv, d, dtype, dtype if dtype != lib.PA_FP8_E4M3 else io)
 
     assert lib.decode_partition_size(S, H, desc(H, d=D), 100, 0) == 128  # single, rounded to 32
     assert lib.decode_partition_size(96, 32, desc(32), 2048, 0) == 2048  # single pass
@@ -134,15 +133,21 @@ def test_workspace_and_partition_sizes(lib):
     assert lib.decode_partition_size(1, 32, desc(32), 32768, 0) == 512
     assert lib.decode_partition_size(96, 32, desc(32), 2048, 1024) == 1024
     assert lib.decode_partition_size(1, 1, desc(1), 30000, 0) == 128
-    # Grouped heads (G = 4) on a 16-bit cache: one CTA row per K/V head,
-    # 1024-token partitions while the grid has at least one CTA per SM; the
-    # fp8 cache stays on one CTA row per query head.
+    # Grouped heads (2 <= G <= 16) on a 16-bit cache, or on an fp8 cache with
+    # f16 rows and head_dim 128: the tensor-core kernel, one CTA row per K/V
+    # head, 1024-token partitions while the grid has at least one CTA per SM.
+    # fp8 without grouping, with bf16 rows or head_dim 64 stays on one CTA
+    # row per query head.
     assert lib.decode_partition_size(96, 32, desc(8), 2048, 0) == 1024
     assert lib.decode_partition_size(96, 32, desc(8, lib.PA_BF16), 2048, 0) == 1024
     assert lib.decode_partition_size(96, 32, desc(8), 1000, 0) == 1024  # single pass
     assert lib.decode_partition_size(1, 32, desc(8), 32768, 0) == 1024  # 8 x 32 CTAs
     assert lib.decode_partition_size(1, 32, desc(8), 4096, 0) == 256  # 8 x 16 CTAs
-    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3), 2048, 0) == 2048
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3), 2048, 0) == 1024
+    assert lib.decode_partition_size(96, 32, desc(32, lib.PA_FP8_E4M3), 2048, 0) == 2048
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3, io=lib.PA_BF16),
+                                      2048, 0) == 2048
+    assert lib.decode_partition_size(96, 32, desc(32, lib.PA_FP8_E4M3, d=64), 2048, 0) == 2048
     with pytest.raises(ValueError):
         lib.decode_partition_size(96, 32, desc(7), 2048, 0)  # 32 % 7 != 0
     assert lib.decode_partition_size(96, 32, desc(1), 2048, 0) == 2048  # G = 32 > 16

@@ -184,3 +184,50 @@ def test_group_kernel_full_size_sampled():
     sub = wl.subset(st, ids)
     ref, _, _ = oracle.run_step(sub, 0)
     assert max_err(outs[0][torch.as_tensor(ids, device="cuda")], ref) <= TOL
+
+
+# ------------------------------------------- fp8 cache on the grouped kernel
+# fp8 (e4m3 + row scales) caches with f16 rows and head_dim 128 and
+# 2 <= G <= 16 take the grouped tensor-core kernel (K codes widened into the
+# B fragments, V tiles transposed in registers, V scales folded into P).
+
+@pytest.mark.parametrize("G,bs", [(2, 16), (3, 8), (4, 32), (8, 8), (12, 16), (16, 32)])
+@pytest.mark.parametrize("partition", [0, 64])
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_group_kernel_fp8_matches_oracle(G, bs, partition, fused):
+    st = wl.llama_layer(num_seqs=6, num_blocks=1500, num_heads=2 * G, num_kv_heads=2,
+                        block_size=bs, dtype="fp8", ctx_range=(1, 700))
+    run = run_step_fused if fused else run_step
+    outs, d, err = run(st, partition_size=partition)
+    assert err == 0
+    ref, kref, vref = oracle.run_step(st, 0)
+    assert max_err(outs[0], ref) <= TOL
+    assert np.array_equal(to_bits(d["key_caches"][0]), kref)
+    assert np.array_equal(to_bits(d["value_caches"][0]), vref)
+
+
+def test_group_kernel_fp8_fused_equals_separate_and_split_matches_single():
+    st = wl.llama_layer(num_seqs=8, num_blocks=2000, num_heads=32, num_kv_heads=4,
+                        dtype="fp8", ctx_range=(900, 3000))
+    a, da, _ = run_step(st)
+    b, db, _ = run_step_fused(st)
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+    assert torch.equal(da["key_caches"][0].data, db["key_caches"][0].data)
+    ref, _, _ = oracle.run_step(st, 0)
+    single, _, e1 = run_step(st, partition_size=4096, out_dtype=torch.float32)
+    split, _, e2 = run_step(st, partition_size=256, out_dtype=torch.float32)
+    assert e1 == 0 and e2 == 0
+    assert max_err(single[0], ref) <= TOL and max_err(split[0], ref) <= TOL
+    assert float((split[0] - single[0]).abs().max()) <= TOL
+
+
+def test_group_kernel_fp8_full_size_sampled():
+    st = wl.llama_layer(num_kv_heads=8, dtype="fp8")
+    outs, d, err = run_step_fused(st)
+    assert err == 0
+    ctx = st.context_lens
+    rng = np.random.default_rng(66)
+    ids = sorted(set([int(np.argmin(ctx)), int(np.argmax(ctx))] +
+                     rng.choice(st.num_seqs, 4, replace=False).tolist()))
+    ref, _, _ = oracle.run_step(wl.subset(st, ids), 0)
+    assert max_err(outs[0][torch.as_tensor(ids, device="cuda")], ref) <= TOL
