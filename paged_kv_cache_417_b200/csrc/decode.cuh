@@ -115,16 +115,38 @@ __device__ __forceinline__ void unpack8(const uint4 &raw, float (&f)[8])
 // Storage tag of an fp8 cache: OCP e4m3 codes, one fp32 scale per row.
 struct E4M3 {};
 
-// Four e4m3 codes (little-endian bytes of u) to floats, through the
-// hardware fp8x2 -> f16x2 conversion.
+// Four e4m3 codes (little-endian bytes of u) to two f16 pairs (codes 0, 1
+// in lo; 2, 3 in hi; exact), with the hardware e4m3x2 -> f16x2 conversion
+// applied to the register's two 16-bit halves directly.
+__device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t u, uint32_t &lo, uint32_t &hi)
+{
+    asm("{\n\t.reg .b16 a, b;\n\t"
+        "mov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(u));
+}
+
+// An f16 pair (low half first) to two floats.
+__device__ __forceinline__ float2 h2_to_float2(uint32_t h)
+{
+    float2 f;
+    asm("{\n\t.reg .b16 a, b;\n\t"
+        "mov.b32 {a, b}, %2;\n\t"
+        "cvt.f32.f16 %0, a;\n\t"
+        "cvt.f32.f16 %1, b;\n\t}"
+        : "=f"(f.x), "=f"(f.y)
+        : "r"(h));
+    return f;
+}
+
+// Four e4m3 codes (little-endian bytes of u) to floats (exact).
 __device__ __forceinline__ void e4m3x4_to_float(uint32_t u, float *f)
 {
-    __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(u & 0xffffu), __NV_E4M3);
-    __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(u >> 16), __NV_E4M3);
-    __half2 a, b;
-    memcpy(&a, &lo, 4);
-    memcpy(&b, &hi, 4);
-    float2 fa = __half22float2(a), fb = __half22float2(b);
+    uint32_t lo, hi;
+    e4m3x4_to_h2x2(u, lo, hi);
+    const float2 fa = h2_to_float2(lo), fb = h2_to_float2(hi);
     f[0] = fa.x; f[1] = fa.y; f[2] = fb.x; f[3] = fb.y;
 }
 
@@ -204,14 +226,8 @@ template <> struct Store<E4M3> {
     {
         const uint32_t c[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            __half2_raw lo =
-                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(c[k] & 0xffffu), __NV_E4M3);
-            __half2_raw hi =
-                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(c[k] >> 16), __NV_E4M3);
-            w[2 * k] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
-            w[2 * k + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
-        }
+        for (int k = 0; k < 4; ++k)
+            e4m3x4_to_h2x2(c[k], w[2 * k], w[2 * k + 1]);
     }
 };
 

@@ -124,14 +124,6 @@ __device__ __forceinline__ float2 unpack_bf2(uint32_t u)
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-// Two e4m3 codes (low byte first) widened to an f16 pair (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two_codes)
-{
-    const __half2_raw h =
-        __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
 // Transpose of an 8x8 tile of 16-bit elements held as one register per lane
 // (lane l holds row l/4, columns 2(l%4), 2(l%4)+1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
@@ -416,10 +408,11 @@ __global__ void __launch_bounds__(NW * 32)
                         const int kk = 2 * kp + h;
                         float(&acc0)[4] = h ? sd[0] : sc[0];
                         float(&acc1)[4] = h ? sd[1] : sc[1];
-                        mma_16816<false>(acc0, qa[kk], e4m3x2_to_h2(r[2 * h]),
-                                         e4m3x2_to_h2(r[2 * h] >> 16));
-                        mma_16816<false>(acc1, qa[kk], e4m3x2_to_h2(r[2 * h + 1]),
-                                         e4m3x2_to_h2(r[2 * h + 1] >> 16));
+                        uint32_t b0l, b0h, b1l, b1h;
+                        e4m3x4_to_h2x2(r[2 * h], b0l, b0h);
+                        e4m3x4_to_h2x2(r[2 * h + 1], b1l, b1h);
+                        mma_16816<false>(acc0, qa[kk], b0l, b0h);
+                        mma_16816<false>(acc1, qa[kk], b1l, b1h);
                     }
                 }
             } else {
@@ -551,10 +544,13 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int c = 2 * kp + h; // piece: d = 16c .. 16c + 15
-                        const uint32_t lo0 = movmatrix_trans(e4m3x2_to_h2(r[2 * h]));
-                        const uint32_t lo1 = movmatrix_trans(e4m3x2_to_h2(r[2 * h + 1]));
-                        const uint32_t hi0 = movmatrix_trans(e4m3x2_to_h2(r[2 * h] >> 16));
-                        const uint32_t hi1 = movmatrix_trans(e4m3x2_to_h2(r[2 * h + 1] >> 16));
+                        uint32_t w0l, w0h, w1l, w1h;
+                        e4m3x4_to_h2x2(r[2 * h], w0l, w0h);
+                        e4m3x4_to_h2x2(r[2 * h + 1], w1l, w1h);
+                        const uint32_t lo0 = movmatrix_trans(w0l);
+                        const uint32_t lo1 = movmatrix_trans(w1l);
+                        const uint32_t hi0 = movmatrix_trans(w0h);
+                        const uint32_t hi1 = movmatrix_trans(w1h);
                         mma_16816<false>(o[2 * c], pa, lo0, lo1);
                         mma_16816<false>(o[2 * c + 1], pa, hi0, hi1);
                     }
