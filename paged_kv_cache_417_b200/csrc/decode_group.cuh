@@ -52,10 +52,11 @@
 // split into a bf16 head and a bf16 remainder and multiplied twice, which
 // keeps about 16 bits.
 //
-// Rows past the context: their scores are set to -inf and their P' to 0
-// by selection (never computed from the stale bytes), and the V rows of a
-// partial last chunk are zeroed in shared memory before the product, so a
-// weight of 0 meets a finite value (0 * NaN would otherwise reach the sum).
+// Rows past the context (only in a partition's last step): their scores are
+// set to -inf and their fp8 V scales to 0 by selection (never computed from
+// the stale bytes), and the V rows of a partial last chunk are zeroed in
+// shared memory before the product, so a weight of 0 meets a finite value
+// (0 * NaN would otherwise reach the sum).
 //
 // These tiles are warp-sized on purpose: the group is at most 16 rows,
 // below the 64-row minimum of a tcgen05 MMA, and the kernel is bound by HBM
@@ -432,6 +433,8 @@ __global__ void __launch_bounds__(NW * 32)
 
             // Online softmax (base 2). sc[j][e]: token t0 + 8j + q2 + (e & 1),
             // row g0 for e < 2, g1 otherwise.
+            // Only a partition's last step can be partial (warp-uniform).
+            const bool partial = srows < 16;
             float x[2][4];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -442,8 +445,15 @@ __global__ void __launch_bounds__(NW * 32)
                 }
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    x[j][e] = 8 * j + q2 + (e & 1) < srows ? sc[j][e] * ((e & 1) ? ks.y : ks.x)
-                                                            : -INFINITY;
+                    x[j][e] = sc[j][e] * ((e & 1) ? ks.y : ks.x);
+            }
+            if (partial) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (8 * j + q2 + (e & 1) >= srows)
+                            x[j][e] = -INFINITY;
             }
             float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
             mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 1));
@@ -486,8 +496,14 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const float2 v2 = *reinterpret_cast<const float2 *>(vsc + t0 + 8 * j + q2);
-                    vs[j][0] = 8 * j + q2 < srows ? v2.x : 0.f;
-                    vs[j][1] = 8 * j + q2 + 1 < srows ? v2.y : 0.f;
+                    vs[j][0] = v2.x;
+                    vs[j][1] = v2.y;
+                    if (partial) { // stale scales past the context must not reach P'
+                        if (8 * j + q2 >= srows)
+                            vs[j][0] = 0.f;
+                        if (8 * j + q2 + 1 >= srows)
+                            vs[j][1] = 0.f;
+                    }
                     vmax = fmaxf(vmax, fmaxf(vs[j][0], vs[j][1]));
                 }
                 vmax = fmaxf(vmax, __shfl_xor_sync(FULL, vmax, 1));
@@ -496,12 +512,12 @@ __global__ void __launch_bounds__(NW * 32)
                 cr = vref / rn;
                 vref = rn;
                 const float inv = 1.f / rn;
+                // Tokens past the context have p = 0 and a zeroed scale.
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        pr[j][e] = 8 * j + q2 + (e & 1) < srows ? pr[j][e] * (vs[j][e & 1] * inv)
-                                                                : 0.f;
+                        pr[j][e] *= vs[j][e & 1] * inv;
             }
             if (__any_sync(FULL, c0 != 1.f || c1 != 1.f || cr != 1.f)) { // a max moved
                 const float f0 = c0 * cr, f1 = c1 * cr;
