@@ -46,11 +46,15 @@ constexpr int kGroupStages = 2;
 constexpr int kTargetCtasPerSm = 12; // ~4 waves of 3 resident CTAs
 constexpr int kMinAutoPartition = 128;
 constexpr int kAutoPartition = 2048;
-// The grouped kernel streams best in long partitions (B200 sweeps of 128 to
-// 2048 tokens at 2, 4 and 8 K/V heads: 1024 was fastest in every case), so
-// its automatic choice is 1024, halved (down to 256) only while the grid
-// would have fewer CTAs than the GPU has SMs.
-constexpr int kGroupAutoPartition = 1024;
+// The grouped kernel streams best in long partitions. When it hands out the
+// longest sequences first (batches of up to kRankMaxSeqs), its automatic
+// choice is 2048 tokens, halved (down to 256) while the grid would have
+// fewer than 2 CTAs per SM (B200, Llama-7B layer: 8 K/V heads 73 us at 2048
+// vs 81 us at 1024; 4 K/V heads 49 us at either; 2 K/V heads 37 us at 1024
+// vs 43 us at 2048). In natural order (larger batches) long last units drain
+// slowly, so it starts from 1024 and halves while there are fewer CTAs than
+// SMs (256 sequences x 32 layers: 74 us per layer at 1024, single pass
+// slower).
 constexpr int kGroupMinAutoPartition = 256;
 constexpr int kPartitionQuantum = 32;
 constexpr int kMaxDevices = 64;
@@ -136,18 +140,20 @@ bool use_group_kernel(const pa_cache_desc *c, int32_t num_heads)
 // single pass. Automatic choice for decode_split_kernel (one CTA row per
 // (sequence, query head)): 2048 tokens, halved (down to 128) while the grid
 // would give fewer than about four waves of resident CTAs. For
-// decode_group_kernel (one CTA row per (sequence, K/V head)): 1024, halved
-// (down to 256) while the grid has fewer CTAs than SMs.
+// decode_group_kernel (one CTA row per (sequence, K/V head)): 2048, halved
+// (down to 256) while the grid has fewer than 2 CTAs per SM.
 int choose_partition(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c,
                      int32_t max_ctx, int32_t requested, int sm_count)
 {
     int P = requested;
     if (P == 0) {
         const bool grouped = use_group_kernel(c, num_heads);
+        const bool ranked = grouped && PA_GROUP_RANK && num_seqs <= kRankMaxSeqs;
         const int64_t units = (int64_t)num_seqs * (grouped ? c->num_kv_heads : num_heads);
         const int floor_p = grouped ? kGroupMinAutoPartition : kMinAutoPartition;
-        const int64_t target = (int64_t)(grouped ? 1 : kTargetCtasPerSm) * sm_count;
-        P = grouped ? kGroupAutoPartition : kAutoPartition;
+        const int64_t target =
+            (int64_t)(!grouped ? kTargetCtasPerSm : ranked ? 2 : 1) * sm_count;
+        P = !grouped ? kAutoPartition : ranked ? 2048 : 1024;
         while (P > floor_p && units * ((max_ctx + P - 1) / P) < target)
             P /= 2;
     }

@@ -135,15 +135,19 @@ def test_workspace_and_partition_sizes(lib):
     assert lib.decode_partition_size(1, 1, desc(1), 30000, 0) == 128
     # Grouped heads (2 <= G <= 16) on a 16-bit cache, or on an fp8 cache with
     # f16 rows and head_dim 128: the tensor-core kernel, one CTA row per K/V
-    # head, 1024-token partitions while the grid has at least one CTA per SM.
+    # head. Batches of up to 128 sequences (handed out longest first):
+    # 2048-token partitions halved while the grid has fewer than 2 CTAs per
+    # SM; larger batches: 1024 halved while it has fewer CTAs than SMs.
     # fp8 without grouping, with bf16 rows or head_dim 64 stays on one CTA
     # row per query head.
-    assert lib.decode_partition_size(96, 32, desc(8), 2048, 0) == 1024
-    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_BF16), 2048, 0) == 1024
+    assert lib.decode_partition_size(96, 32, desc(8), 2048, 0) == 2048  # single pass
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_BF16), 4096, 0) == 2048
+    assert lib.decode_partition_size(96, 32, desc(2), 2048, 0) == 1024  # 192 x 2 CTAs
     assert lib.decode_partition_size(96, 32, desc(8), 1000, 0) == 1024  # single pass
-    assert lib.decode_partition_size(1, 32, desc(8), 32768, 0) == 1024  # 8 x 32 CTAs
+    assert lib.decode_partition_size(1, 32, desc(8), 32768, 0) == 512  # 8 x 64 CTAs
     assert lib.decode_partition_size(1, 32, desc(8), 4096, 0) == 256  # 8 x 16 CTAs
-    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3), 2048, 0) == 1024
+    assert lib.decode_partition_size(256, 32, desc(8), 2048, 0) == 1024  # natural order
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3), 4096, 0) == 2048
     assert lib.decode_partition_size(96, 32, desc(32, lib.PA_FP8_E4M3), 2048, 0) == 2048
     assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3, io=lib.PA_BF16),
                                       2048, 0) == 2048
