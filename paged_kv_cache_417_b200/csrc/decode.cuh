@@ -71,6 +71,7 @@ struct DecodeParams {
     int32_t *dev_err;
     int32_t num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq, max_context_len;
     int32_t partition_size, num_parts;
+    int32_t rank_seqs; // 1: grid row y takes the sequence of rank y (ranked_sequence)
     int32_t out_dtype; // 0 f16, 1 bf16, 2 f32
     float qk_scale_log2;
     // Fused append (pa_write_kv_decode): the new token of sequence s, at
@@ -752,6 +753,38 @@ __device__ __forceinline__ void merge_if_last(const DecodeParams &p, int s, int 
         p.ws_count[slot] = 0;
 }
 
+// Longest sequences first: when DecodeParams::rank_seqs is set (batches of
+// up to kRankMaxSeqs sequences; the host decides per launch), a CTA on grid
+// row y works on the sequence of rank y by (context length descending,
+// index ascending), so the hardware hands out the longest units first and a
+// launch ends on short ones (a per-CTA timeline of the grouped kernel on the
+// Llama-7B layer showed a ~12 us drain of long last CTAs). Any order gives
+// the same outputs. The ranking costs each CTA a dependent round trip for
+// all context lengths and O(S^2 / threads) compares.
+constexpr int kRankMaxSeqs = 128;
+
+// Every thread of the CTA calls it (two barriers): the sequence of rank y.
+// ctx_buf: kRankMaxSeqs ints of shared memory; out: one shared int.
+__device__ __forceinline__ int ranked_sequence(const int32_t *context_lens, int S, int y,
+                                               int tid, int nthreads, int32_t *ctx_buf, int *out)
+{
+    for (int k = tid; k < S; k += nthreads)
+        ctx_buf[k] = context_lens[k];
+    __syncthreads();
+    for (int k = tid; k < S; k += nthreads) {
+        const int c = ctx_buf[k];
+        int r = 0;
+        for (int j = 0; j < S; ++j) {
+            const int cj = ctx_buf[j];
+            r += (cj > c) | ((cj == c) & (j < k));
+        }
+        if (r == y)
+            *out = k; // ranks are a permutation: exactly one writer
+    }
+    __syncthreads();
+    return *out;
+}
+
 // Shared prologue: read the context length and the partition's slice of the
 // block table at the same time (one global latency). Returns false when the
 // partition is past the sequence (the whole CTA returns).
@@ -785,7 +818,8 @@ template <typename T, int D, int BS, int NW, int NS> struct SplitCfg {
     static constexpr int kRingsBytes = NW * C::kRingBytes;
     static constexpr int kBarBytes = NW * NS * 8;
     static constexpr int kMergeBytes = NW * (D + 2) * 4;
-    static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kMergeBytes;
+    static constexpr int kRankBytes = kRankMaxSeqs * 4;
+    static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kMergeBytes + kRankBytes;
     static size_t smem_bytes(int partition)
     {
         return kFixedBytes + ((partition / BS) * 4 + 15) / 16 * 16;
@@ -806,13 +840,16 @@ __global__ void __launch_bounds__(NW * 32)
     char *rings = reinterpret_cast<char *>(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kRingsBytes);
     float *merge = reinterpret_cast<float *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes);
+    int32_t *rank_ctx = reinterpret_cast<int32_t *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes +
+                                                    Cfg::kMergeBytes);
     int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
-    __shared__ int cta_flags;
+    __shared__ int cta_flags, ranked_seq;
 
     // Dependent kernels (the reduce, the next layer's write) may launch now;
     // each of them waits for this grid before it touches data.
     pdl_launch_dependents();
-    const int h = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
+    const int h = blockIdx.x, part = blockIdx.z;
+    int s = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads, HK = p.num_kv_heads;
     const int group = H / HK;  // query heads per K/V head
@@ -825,6 +862,9 @@ __global__ void __launch_bounds__(NW * 32)
             mbar_init(smem_addr(&bars[warp * NS + k]), 1);
     fence_mbar_init();
     pdl_wait_prior_grid(); // every input may come from the previous kernel
+    if (p.rank_seqs)
+        s = ranked_sequence(p.context_lens, p.num_seqs, blockIdx.y, tid, NW * 32, rank_ctx,
+                            &ranked_seq);
     UnitInfo u;
     const bool live = load_unit<BS>(p, s, part, tid, NW * 32, tid == 0 && h == 0 && part == 0,
                                     table, u);

@@ -72,19 +72,6 @@ namespace pagedkv {
 
 constexpr int kGroupMaxHeads = 16;
 
-// Longest sequences first: for batches of up to kRankMaxSeqs sequences,
-// grid row y takes the sequence of rank y by (context length descending,
-// index ascending), so the hardware hands out the longest units first and
-// the launch ends on short ones (a per-CTA timeline of the Llama-7B layer
-// with 8 K/V heads showed a ~12 us drain of long last CTAs). Any order gives
-// the same outputs. Every CTA ranks the whole batch (O(S^2 / threads)
-// compares), so larger batches keep the natural order: at 256 sequences the
-// ranking cost more than the shorter drain saved. PA_GROUP_RANK=0 builds
-// the natural order for comparisons.
-#ifndef PA_GROUP_RANK
-#define PA_GROUP_RANK 1
-#endif
-constexpr int kRankMaxSeqs = 128;
 
 struct GroupParams {
     CUtensorMap tk; // key pool (see the staging note above), 128B swizzle
@@ -108,7 +95,7 @@ template <typename T, int D, int BS, int NW, int NS> struct GroupCfg {
     static constexpr int kBarBytes = NW * NS * 8;
     // fp8 row scales: per warp, [stage][K | V][kChunk] floats.
     static constexpr int kScaleBytes = kFp8 ? NW * NS * 2 * kChunk * 4 : 0;
-    static constexpr int kRankBytes = PA_GROUP_RANK ? kRankMaxSeqs * 4 : 0; // context lengths
+    static constexpr int kRankBytes = kRankMaxSeqs * 4; // context lengths for ranking
     static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kScaleBytes + kRankBytes;
     // After its last chunk a warp leaves (O, m, l) of its rows in its ring.
     static constexpr int kMergeStride = D + 2;
@@ -188,24 +175,9 @@ __global__ void __launch_bounds__(NW * 32)
             mbar_init(smem_addr(&bars[warp * NS + k]), 1);
     fence_mbar_init();
     pdl_wait_prior_grid(); // every input may come from the previous kernel
-    if (PA_GROUP_RANK && p.num_seqs <= kRankMaxSeqs) {
-        const int S = p.num_seqs;
-        for (int k = tid; k < S; k += NW * 32)
-            rank_ctx[k] = p.context_lens[k];
-        __syncthreads();
-        for (int k = tid; k < S; k += NW * 32) {
-            const int c = rank_ctx[k];
-            int r = 0;
-            for (int j = 0; j < S; ++j) {
-                const int cj = rank_ctx[j];
-                r += (cj > c) | ((cj == c) & (j < k));
-            }
-            if (r == (int)blockIdx.y)
-                ranked_seq = k; // ranks are a permutation: exactly one writer
-        }
-        __syncthreads();
-        s = ranked_seq;
-    }
+    if (p.rank_seqs) // longest sequences first (ranked_sequence)
+        s = ranked_sequence(p.context_lens, p.num_seqs, blockIdx.y, tid, NW * 32, rank_ctx,
+                            &ranked_seq);
 
     // Fragment coordinates: this lane holds rows g0 and g1 = g0 + 8 and, in
     // every 8-wide column tile, columns q2 and q2 + 1 (q = lane % 4).

@@ -136,6 +136,28 @@ bool use_group_kernel(const pa_cache_desc *c, int32_t num_heads)
     return G >= 2;
 }
 
+// Whether a launch hands out its sequences longest first (ranked_sequence).
+// Each CTA pays a dependent round trip for it, so it is worth it only when
+// the drain of long last units dominates: the grouped kernel for batches of
+// up to kRankMaxSeqs; decode_split_kernel only for grids of at least six
+// waves of units of at least 1024 tokens (B200: Llama-7B layer 256.7 ->
+// 252.0 us, fp8 183.3 -> 174.4 us; with shorter or fewer units - the
+// prefix-sharing batch, 8-sequence batches - it was 8-12 % slower).
+constexpr int kRankMinWaves = 6;
+constexpr int kRankMinPartition = 1024;
+constexpr int kResidentCtasPerSm = 3;
+bool rank_sequences(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c, int P,
+                    int64_t parts)
+{
+    if (num_seqs > kRankMaxSeqs)
+        return false;
+    if (use_group_kernel(c, num_heads))
+        return true;
+    const int64_t ctas = (int64_t)num_seqs * num_heads * parts;
+    return P >= kRankMinPartition &&
+           ctas >= (int64_t)kRankMinWaves * kResidentCtasPerSm * sm_count_of_current_device();
+}
+
 // Partition (tokens per work unit) for a decode; >= max_context_len means a
 // single pass. Automatic choice for decode_split_kernel (one CTA row per
 // (sequence, query head)): 2048 tokens, halved (down to 128) while the grid
@@ -148,7 +170,7 @@ int choose_partition(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c
     int P = requested;
     if (P == 0) {
         const bool grouped = use_group_kernel(c, num_heads);
-        const bool ranked = grouped && PA_GROUP_RANK && num_seqs <= kRankMaxSeqs;
+        const bool ranked = grouped && num_seqs <= kRankMaxSeqs;
         const int64_t units = (int64_t)num_seqs * (grouped ? c->num_kv_heads : num_heads);
         const int floor_p = grouped ? kGroupMinAutoPartition : kMinAutoPartition;
         const int64_t target =
@@ -588,6 +610,7 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
     p.max_context_len = max_context_len;
     p.partition_size = P;
     p.num_parts = (int32_t)parts;
+    p.rank_seqs = rank_sequences(num_seqs, num_heads, cache, P, parts) ? 1 : 0;
     p.out_dtype = (int32_t)out_dtype;
     p.qk_scale_log2 = scale * 1.4426950408889634f;
     p.new_key = new_key;
