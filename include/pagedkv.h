@@ -110,10 +110,11 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t hea
                                 int32_t max_context_len, int32_t partition_size);
 
 /* The partition size pa_decode uses for these arguments (tokens per CTA
- * work unit); >= max_context_len means a single pass without a reduce. The
- * cache descriptor decides the kernel and so the work units: one CTA row per
- * (sequence, query head), or per (sequence, K/V head) when grouped query
- * heads take the grouped kernel (16-bit cache, 2 <= G <= 16). Returns -1 on
+ * work unit); >= max_context_len means a single pass without partitions to
+ * merge. The cache descriptor decides the kernel and so the work units: one
+ * CTA row per (sequence, query head), or per (sequence, K/V head) when
+ * grouped query heads take the grouped kernel (2 <= G <= 16 with a 16-bit
+ * cache, or with an fp8 cache of f16 rows and head_dim 128). Returns -1 on
  * invalid arguments. */
 int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
                                  const pa_cache_desc *cache, int32_t max_context_len,
