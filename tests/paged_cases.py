@@ -389,5 +389,34 @@ def pin_grouped_heads(orc, seed=19):
             assert np.max(np.abs(got[s] - ref)) <= 1e-12, "grouped heads vs dense"
 
 
-ALL_PINS = [pin_grouped_heads, pin_dense, pin_bruteforce, pin_closed_forms, pin_permutation, pin_write_kv,
+def pin_grouped_heads_fp8(orc, seed=20):
+    """Grouped heads on an fp8 cache: the decode equals the decode of the
+    same cache with each K/V head's tiles repeated G times (one K/V head per
+    query head), whose fp8 path pin_fp8 ties to dense attention."""
+    rng = np.random.default_rng(seed)
+    for Hk, G, D, bs in [(2, 3, 64, 16), (1, 4, 128, 8)]:
+        ctxs = [1, 20, 47]
+        nb = sum(-(-c // bs) for c in ctxs) + 2
+        tb = bs * D + 4 * bs
+        kc = np.full((nb, Hk, tb), 0x7F, dtype=np.uint8)
+        vc = kc.copy()
+        bt = np.full((3, max(-(-c // bs) for c in ctxs)), -1, dtype=np.int32)
+        perm, nxt = rng.permutation(nb), 0
+        for s, c in enumerate(ctxs):
+            blocks = perm[nxt: nxt + -(-c // bs)]
+            nxt += len(blocks)
+            bt[s, : len(blocks)] = blocks
+            k = to_storage_bits(rng.standard_normal((c, Hk, D), dtype=np.float32), "f16")
+            v = to_storage_bits(rng.standard_normal((c, Hk, D), dtype=np.float32), "f16")
+            slots = np.array([blocks[t // bs] * bs + t % bs for t in range(c)], dtype=np.int64)
+            orc.write_kv_fp8(k, v, slots, kc, vc, bs)
+        q = to_storage_bits(rng.standard_normal((3, Hk * G, D), dtype=np.float32), "f16")
+        ctx = np.array(ctxs, dtype=np.int32)
+        got = orc.decode_fp8(q, kc, vc, bt, ctx, np.float32(0.1), bs)
+        ref = orc.decode_fp8(q, np.repeat(kc, G, axis=1), np.repeat(vc, G, axis=1), bt, ctx,
+                             np.float32(0.1), bs)
+        assert np.max(np.abs(got - ref)) <= 1e-12, "fp8 grouped heads vs repeated heads"
+
+
+ALL_PINS = [pin_grouped_heads, pin_grouped_heads_fp8, pin_dense, pin_bruteforce, pin_closed_forms, pin_permutation, pin_write_kv,
             pin_copy_blocks, pin_swap_blocks, pin_fp8]

@@ -157,7 +157,9 @@ MUTANTS = [
     ("swap_wrong_dst", "memcpy(dst_k[l] + b * block_elems, src_k[l] + a * block_elems,",
      "memcpy(dst_k[l] + a % dst_blocks * block_elems, src_k[l] + a * block_elems,"),
     ("gqa_head_map", "context_lens[s], h / group, scale);",
-     "context_lens[s], h % num_kv_heads, scale);"),
+     "context_lens[s], h % num_kv_heads, scale);", 0),
+    ("fp8_gqa_head_map", "context_lens[s], h / group, scale);",
+     "context_lens[s], h % num_kv_heads, scale);", 1),
     ("f16_exponent_bias", "v = ldexp((double)(f | 0x400), e - 25);",
      "v = ldexp((double)(f | 0x400), e - 24);"),
 ]
