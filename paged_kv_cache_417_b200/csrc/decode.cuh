@@ -189,7 +189,7 @@ __device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, 
 
 // Which arithmetic the stream uses. The macros exist for tuning sweeps.
 #ifndef PA_QK_MIXED
-#define PA_QK_MIXED 1 // q.k with fma.rn.f32.f16 for f16 caches with f16 queries
+#define PA_QK_MIXED 1 // q.k with fma.rn.f32.f16 for f16 queries on f16 or fp8 caches
 #endif
 #ifndef PA_FFMA2
 #define PA_FFMA2 1 // packed fp32 FMAs on the fp32 (non-mixed) paths
@@ -309,10 +309,12 @@ template <typename T, typename QT, int D, int BS, int NS> struct WarpStream {
     static constexpr int STEPS = C::kSteps, E = C::kE, J = C::kJ, ROW = C::kRow;
     static constexpr int DATA = C::kData, SCL = C::kScales, STAGE = C::kStage;
     static constexpr unsigned FULL = 0xffffffffu;
-    // q.k on raw f16 query pairs with mixed FMAs, the scale applied per row;
-    // else on fp32 copies of the query pre-scaled by scale*log2(e).
+    // q.k on raw f16 query pairs with mixed FMAs (f16 caches, and fp8 codes
+    // widened to exact f16 pairs), the scale applied per row; else on fp32
+    // copies of the query pre-scaled by scale*log2(e).
     static constexpr bool kQKMixed =
-        PA_QK_MIXED && std::is_same<QT, __half>::value && std::is_same<T, __half>::value;
+        PA_QK_MIXED && std::is_same<QT, __half>::value &&
+        (std::is_same<T, __half>::value || std::is_same<T, E4M3>::value);
     static constexpr bool kPVMixed = PA_PV_MIXED && std::is_same<T, __half>::value;
 
     float qf[kQKMixed ? 1 : J][kQKMixed ? 1 : E];
