@@ -155,3 +155,44 @@ def test_workspace_and_partition_sizes(lib):
     with pytest.raises(ValueError):
         lib.decode_partition_size(96, 32, desc(7), 2048, 0)  # 32 % 7 != 0
     assert lib.decode_partition_size(96, 32, desc(1), 2048, 0) == 2048  # G = 32 > 16
+
+
+def test_newer_entry_points_reject_bad_arguments_on_host(lib):
+    """Checks that return before any CUDA call (fake pointers are never
+    dereferenced)."""
+    L = lib._lib
+    fake = ctypes.c_void_p(0x1000)
+    # An empty pool with a positive max_context_len cannot be decoded.
+    empty = _desc(lib, nb=0)
+    st = L.pa_decode(fake, 0, fake, 1, 2, fake, fake, ctypes.byref(empty), fake, 1, fake, 16,
+                     0.125, 0, None, 0, None, None)
+    assert st == lib.PA_ERR_INVALID_ARG and b"empty pool" in L.pa_last_error()
+    # The fused call needs both new rows.
+    desc = _desc(lib)
+    st = L.pa_write_kv_decode(fake, 0, fake, None, fake, 1, 2, fake, fake, ctypes.byref(desc),
+                              fake, 1, fake, 16, 0.125, 0, None, 0, None, None)
+    assert st == lib.PA_ERR_INVALID_ARG
+    # pa_decode_noalloc refuses work whose partials exceed its built-in
+    # scratch (64 sequences x 64 heads x 256 partitions of 32 tokens).
+    big = _desc(lib, h=64, d=128)
+    st = L.pa_decode_noalloc(fake, 0, fake, 64, 64, fake, fake, ctypes.byref(big), fake, 256,
+                             fake, 8192, 0.125, 32, None, None)
+    assert st == lib.PA_ERR_WORKSPACE and b"scratch" in L.pa_last_error()
+    # Self-test of the bounded wait: device flag required, limit in (0, 1 s].
+    assert L.pa_selftest_wait_timeout(None, 10, None) == lib.PA_ERR_INVALID_ARG
+    assert L.pa_selftest_wait_timeout(fake, 0, None) == lib.PA_ERR_INVALID_ARG
+    assert L.pa_selftest_wait_timeout(fake, 1000001, None) == lib.PA_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="would launch on fake pointers where a GPU exists")
+def test_grouped_decode_without_a_gpu_fails_cleanly(lib):
+    """With no GPU, a call that passes the host checks reports a CUDA error
+    (no CPU fallback computes anything)."""
+    L = lib._lib
+    fake = ctypes.c_void_p(0x1000)
+    for dt in (0, 3):  # f16, and fp8 with f16 rows (both take the grouped kernel)
+        desc = lib.CacheDesc(16, 16, 2, 128, dt, 0)
+        st = L.pa_decode(fake, 0, fake, 1, 8, fake, fake, ctypes.byref(desc), fake, 1, fake,
+                         16, 0.125, 0, None, 0, None, None)
+        assert st == lib.PA_ERR_CUDA, L.pa_last_error()
