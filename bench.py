@@ -577,7 +577,8 @@ def main():
     total_ms = max_over_ranks(step_ms, dist, dev)
     value = job_throughput(world, S, args.steps, total_ms)
 
-    # Roofline of the dominant kernel (the decode call: decode + its reduce).
+    # Roofline of the dominant kernel (the decode call; split partitions are
+    # merged inside it).
     ab = algorithmic_bytes(step)
     dec_avg_s = statistics.mean(dec_ms) / 1e3
     achieved = ab["total"] / dec_avg_s / 1e9
