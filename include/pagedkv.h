@@ -150,8 +150,16 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
  *               (zero-fill a new workspace once and keep it for this
  *               library). The rest is scratch. Two calls sharing one
  *               workspace on different streams race.
- * Accumulation is fp32 throughout. A block id outside the pool sets
- * PA_DEVERR_BLOCK_ID and makes that sequence's output NaN.
+ * Precision: q.k products and sums, the softmax (running max, exponentials,
+ * running sum) and the P.V sums are fp32. The softmax weight p of the P.V
+ * products is rounded to the operand type first in three cases: to f16 with
+ * f16 rows (a product of two f16 values is exact in fp32); to a bf16 head
+ * plus a bf16 remainder (about 16 significant bits) with bf16 rows on the
+ * grouped-heads kernel; and, with fp8 caches on the grouped-heads kernel,
+ * p times the row's V scale over the largest V scale seen so far, to f16.
+ * Otherwise (bf16 rows, and fp8 caches, with one CTA per query head) p
+ * stays fp32. The output is rounded once, to out_dtype. A block id outside
+ * the pool sets PA_DEVERR_BLOCK_ID and makes that sequence's output NaN.
  */
 pa_status pa_decode(void *out, pa_dtype out_dtype, const void *query, int32_t num_seqs,
                     int32_t num_heads, const void *key_cache, const void *value_cache,
@@ -204,14 +212,24 @@ pa_status pa_write_kv_decode(void *out, pa_dtype out_dtype, const void *query, c
  * - Limit: if the partial results need more than PA_NOALLOC_SCRATCH_BYTES
  *   (see pa_decode_workspace_size with the partition size actually used,
  *   pa_decode_partition_size), the call returns PA_ERR_WORKSPACE and
- *   launches nothing; a larger partition_size needs less scratch.
- * - Set-up: the first call on each device looks up that device's address of
- *   the array (with the device current); make that first call before any
- *   stream capture.
+ *   launches nothing; a larger partition_size needs less scratch. Argument
+ *   checks run in the same order as pa_decode's, so both calls return the
+ *   same status for the same arguments wherever the workspace is not the
+ *   cause.
+ * - Set-up: the call looks up the array's device address with the device
+ *   current, once per device and CUDA context (again after a device reset,
+ *   which gives the device a new context); make the first call on each
+ *   device before any stream capture.
  * - Sharing: every call in the process on a device uses the same array and
- *   leaves its contents behind. Nothing in it has to start at zero (each call
- *   writes every value it reads), but calls whose kernels overlap on the GPU
- *   (different streams or host threads) race on it: serialise them.
+ *   leaves its contents behind. The array's first 256 KiB are the split
+ *   arrival counters, which must be zero when a split call's kernel starts:
+ *   each split call clears the ones it uses with a cudaMemsetAsync on
+ *   `stream` before its kernel (one extra operation in the stream; nothing
+ *   is allocated). The rest is scratch that every call writes before it
+ *   reads. Calls whose kernels overlap on the GPU (different streams or host
+ *   threads) race on the array and give wrong output for the overlapping
+ *   calls, with no error reported: serialise them. Since every call clears
+ *   its counters first, a race does not reach later, serialised calls.
  * Everything else (arguments, errors, dev_err) is as for pa_decode.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (32u << 20)

@@ -306,9 +306,12 @@ def decode_noalloc(out, query, key_cache, value_cache, block_tables, context_len
     """Like :func:`decode`, for callers that must not allocate device memory
     while decoding (for example an engine that has handed almost all device
     memory to its KV block pool): partial results of split contexts go to a
-    fixed 32 MiB array inside the library instead of a workspace. Calls that
-    overlap on the GPU share that array and race; the first call on a device
-    looks up its address and should come before any stream capture."""
+    fixed 32 MiB array inside the library instead of a workspace. A split
+    call first clears the array's arrival counters on the current stream.
+    Calls that overlap on the GPU share the array and race (their outputs are
+    wrong, with no error); serialised calls are unaffected. The first call on
+    a device looks up the array's address and should come before any stream
+    capture."""
     _need_cache(key_cache, "key_cache")
     _need_cache(value_cache, "value_cache", key_cache)
     _need(query, "query", io_dtype(key_cache))

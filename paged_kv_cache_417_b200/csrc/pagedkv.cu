@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "pagedkv.h"
 
@@ -548,14 +549,83 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
 
 namespace {
 
-// pa_decode, and pa_write_kv_decode when new_key/new_value are given.
+// ---------------------------------------------------------------------------
+// The built-in split workspace of pa_decode_noalloc: a fixed array of device
+// memory compiled into the library, for callers that cannot allocate.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current()
+{
+    static std::atomic<CtxGetCurrentFn> cached{nullptr};
+    CtxGetCurrentFn f = cached.load(std::memory_order_acquire);
+    if (f)
+        return f;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    f = reinterpret_cast<CtxGetCurrentFn>(fn);
+    cached.store(f, std::memory_order_release);
+    return f;
+}
+
+// In host code g_noalloc_scratch names a host-side stand-in, not device
+// memory: its device address is looked up with the device current, once per
+// device and context (a device reset creates a new context whose copy of the
+// array may sit elsewhere), and handed to the kernels.
+pa_status noalloc_scratch(void **out)
+{
+    struct Entry {
+        CUcontext ctx;
+        void *addr;
+    };
+    static std::mutex mu;
+    static Entry cache[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(PA_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+    // The context current on this thread (none yet on a thread that has not
+    // used the runtime: then the look-up below sets it up).
+    CtxGetCurrentFn get = ctx_get_current();
+    CUcontext ctx = nullptr;
+    if (!get || get(&ctx) != CUDA_SUCCESS)
+        ctx = nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ctx || cache[dev].ctx != ctx || !cache[dev].addr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        if (!get || get(&ctx) != CUDA_SUCCESS)
+            ctx = nullptr;
+        cache[dev].ctx = ctx;
+        cache[dev].addr = p;
+    }
+    *out = cache[dev].addr;
+    return PA_OK;
+}
+
+// pa_decode, and pa_write_kv_decode when new_key/new_value are given. With
+// builtin_scratch (pa_decode_noalloc) the split workspace is the library's
+// own array instead of the caller's.
 pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_t num_seqs,
                         int32_t num_heads, const void *key_cache, const void *value_cache,
                         const pa_cache_desc *cache, const int32_t *block_tables,
                         int32_t max_blocks_per_seq, const int32_t *context_lens,
                         int32_t max_context_len, float scale, int32_t partition_size,
                         void *workspace, size_t workspace_bytes, int32_t *dev_err,
-                        void *stream, const void *new_key, const void *new_value)
+                        void *stream, const void *new_key, const void *new_value,
+                        bool builtin_scratch = false)
 {
     pa_status s = check_cache(cache);
     if (s != PA_OK)
@@ -618,6 +688,24 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
     if (parts > 1) {
         const int64_t units = (int64_t)num_seqs * num_heads;
         const size_t need = workspace_bytes_for(units, parts, cache->head_dim);
+        if (builtin_scratch) {
+            if (need > PA_NOALLOC_SCRATCH_BYTES)
+                return fail(PA_ERR_WORKSPACE,
+                            "split decode needs %zu bytes of scratch (partition %d); the "
+                            "built-in scratch holds %u: use a larger partition_size or pa_decode",
+                            need, P, (unsigned)PA_NOALLOC_SCRATCH_BYTES);
+            if ((s = noalloc_scratch(&workspace)) != PA_OK)
+                return s;
+            workspace_bytes = PA_NOALLOC_SCRATCH_BYTES;
+            // The array keeps whatever the last call left: clear the arrival
+            // counters this call can use (the first S * H of them), in stream
+            // order before the kernel.
+            const size_t counters = (size_t)std::min<int64_t>(units, kSplitCounters) * 4;
+            const cudaError_t e =
+                cudaMemsetAsync(workspace, 0, counters, static_cast<cudaStream_t>(stream));
+            if (e != cudaSuccess)
+                return cuda_fail(e, "clearing the built-in scratch counters");
+        }
         if (!workspace || workspace_bytes < need)
             return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes, need %zu", workspace_bytes,
                         need);
@@ -824,39 +912,6 @@ pa_status pa_swap_blocks(void *const *src_key_caches, void *const *src_value_cac
 
 } // extern "C"
 
-// ---------------------------------------------------------------------------
-// pa_decode_noalloc: pa_decode with the workspace taken from a fixed array of
-// device memory compiled into the library, for callers that cannot allocate.
-// ---------------------------------------------------------------------------
-namespace {
-
-static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
-
-// In host code g_noalloc_scratch names a host-side stand-in, not device
-// memory: its device address must be looked up, once per device, with that
-// device current.
-pa_status noalloc_scratch(void **out)
-{
-    static std::atomic<void *> addr[kMaxDevices];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= kMaxDevices)
-        return fail(PA_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
-    void *p = addr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || !p)
-            return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-        addr[dev].store(p, std::memory_order_release);
-    }
-    *out = p;
-    return PA_OK;
-}
-
-} // namespace
-
 extern "C" pa_status pa_decode_noalloc(void *out, pa_dtype out_dtype, const void *query,
                                        int32_t num_seqs, int32_t num_heads,
                                        const void *key_cache, const void *value_cache,
@@ -865,34 +920,8 @@ extern "C" pa_status pa_decode_noalloc(void *out, pa_dtype out_dtype, const void
                                        int32_t max_context_len, float scale,
                                        int32_t partition_size, int32_t *dev_err, void *stream)
 {
-    pa_status s = check_cache(cache);
-    if (s != PA_OK)
-        return s;
-    if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0)
-        return fail(PA_ERR_INVALID_ARG, "negative size argument");
-    if ((s = check_partition_request(partition_size)) != PA_OK)
-        return s;
-    if (num_seqs == 0)
-        return ok();
-    if (num_heads % cache->num_kv_heads != 0)
-        return fail(PA_ERR_UNSUPPORTED, "num_heads %d is not a multiple of num_kv_heads %d",
-                    num_heads, cache->num_kv_heads);
-    const int P = choose_partition(num_seqs, num_heads, cache, max_context_len,
-                                   partition_size, sm_count_of_current_device());
-    const int64_t parts = max_context_len > P ? (max_context_len + P - 1) / P : 1;
-    if (parts > 1) {
-        const size_t need =
-            workspace_bytes_for((int64_t)num_seqs * num_heads, parts, cache->head_dim);
-        if (need > PA_NOALLOC_SCRATCH_BYTES)
-            return fail(PA_ERR_WORKSPACE,
-                        "split decode needs %zu bytes of scratch (partition %d); the built-in "
-                        "scratch holds %u: use a larger partition_size or pa_decode",
-                        need, P, (unsigned)PA_NOALLOC_SCRATCH_BYTES);
-    }
-    void *scratch = nullptr;
-    if ((s = noalloc_scratch(&scratch)) != PA_OK)
-        return s;
-    return pa_decode(out, out_dtype, query, num_seqs, num_heads, key_cache, value_cache, cache,
-                     block_tables, max_blocks_per_seq, context_lens, max_context_len, scale,
-                     partition_size, scratch, PA_NOALLOC_SCRATCH_BYTES, dev_err, stream);
+    return decode_common(out, out_dtype, query, num_seqs, num_heads, key_cache, value_cache,
+                         cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                         scale, partition_size, nullptr, 0, dev_err, stream, nullptr, nullptr,
+                         true);
 }

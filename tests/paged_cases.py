@@ -234,6 +234,58 @@ def pin_write_kv(orc, seed=15):
     assert np.max(np.abs(got[0] - ref)) <= 1e-12, "write_kv round trip"
 
 
+def pin_write_kv_batched(orc, seed=21):
+    """Many tokens in one write call, padding slots among them (a batch of
+    sequences appending at once, "vLLM基础", §2.2 steps 4-6): row t of the
+    input lands at its own slot and nowhere else, checked against direct
+    numpy placement; the fp8 write stores each row's codes and scale as the
+    brute-force nearest-value encoding of that same row."""
+    rng = np.random.default_rng(seed)
+    H, D, bs, NB = 3, 64, 8, 10
+    T = 13
+    slots = rng.permutation(NB * bs)[:T].astype(np.int64)
+    slots[[2, 7, 11]] = -1                      # padding rows
+    nan = nan_bits("f16")
+    keys = to_storage_bits(rng.standard_normal((T, H, D), dtype=np.float32), "f16")
+    vals = to_storage_bits(rng.standard_normal((T, H, D), dtype=np.float32), "f16")
+    kc = np.full((NB, H, bs, D), nan, dtype=np.uint16)
+    vc = kc.copy()
+    orc.write_kv(keys, vals, slots, kc, vc, bs)
+    want_k = np.full_like(kc, nan)
+    want_v = np.full_like(vc, nan)
+    for t in range(T):
+        if slots[t] >= 0:
+            want_k[slots[t] // bs, :, slots[t] % bs, :] = keys[t]
+            want_v[slots[t] // bs, :, slots[t] % bs, :] = vals[t]
+    assert np.array_equal(kc, want_k), "batched K write differs from direct placement"
+    assert np.array_equal(vc, want_v), "batched V write differs from direct placement"
+    # The same batch into an fp8 pool.
+    table = e4m3_table()
+    tb = bs * D + 4 * bs
+    kq = np.full((NB, H, tb), 0x7F, dtype=np.uint8)
+    vq = kq.copy()
+    orc.write_kv_fp8(keys, vals, slots, kq, vq, bs)
+    written = np.zeros((NB, bs), dtype=bool)
+    for t in range(T):
+        if slots[t] < 0:
+            continue
+        b, o = slots[t] // bs, slots[t] % bs
+        written[b, o] = True
+        for h in range(H):
+            for pool, raw in ((kq, keys), (vq, vals)):
+                x = raw[t, h].view(np.float16).astype(np.float32)
+                amax = np.float32(np.max(np.abs(x)))
+                sc = pool[b, h, bs * D + 4 * o: bs * D + 4 * o + 4].view(np.float32)[0]
+                assert sc == amax / np.float32(448.0), "batched fp8 row scale"
+                codes = pool[b, h, o * D:(o + 1) * D]
+                assert np.array_equal(codes, e4m3_nearest(x * (np.float32(448.0) / amax))), \
+                    "batched fp8 row codes"
+                assert np.all(np.isfinite(table[codes]))
+    for pool in (kq, vq):
+        codes = pool[:, :, : bs * D].reshape(NB, H, bs, D)
+        assert np.all(codes.transpose(0, 2, 1, 3)[~written] == 0x7F), "fp8 wrote elsewhere"
+
+
 def pin_copy_blocks(orc, seed=16):
     rng = np.random.default_rng(seed)
     L, NB, H, bs, D = 3, 10, 2, 16, 64
@@ -418,5 +470,6 @@ def pin_grouped_heads_fp8(orc, seed=20):
         assert np.max(np.abs(got - ref)) <= 1e-12, "fp8 grouped heads vs repeated heads"
 
 
-ALL_PINS = [pin_grouped_heads, pin_grouped_heads_fp8, pin_dense, pin_bruteforce, pin_closed_forms, pin_permutation, pin_write_kv,
-            pin_copy_blocks, pin_swap_blocks, pin_fp8]
+ALL_PINS = [pin_grouped_heads, pin_grouped_heads_fp8, pin_dense, pin_bruteforce, pin_closed_forms,
+            pin_permutation, pin_write_kv, pin_write_kv_batched, pin_copy_blocks,
+            pin_swap_blocks, pin_fp8]

@@ -184,6 +184,40 @@ def test_newer_entry_points_reject_bad_arguments_on_host(lib):
     assert L.pa_selftest_wait_timeout(fake, 1000001, None) == lib.PA_ERR_INVALID_ARG
 
 
+def test_noalloc_checks_arguments_like_decode(lib):
+    """pa_decode_noalloc runs pa_decode's argument checks in the same order:
+    for arguments that fail before the workspace matters, both calls return
+    the same status (fake pointers are never dereferenced)."""
+    L = lib._lib
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1008)  # not 16-byte aligned
+    ok = _desc(lib, h=2)
+    # (num_seqs, num_heads, desc, max_blocks, max_ctx, partition, out_dtype, query, scale)
+    cases = [
+        (0, 3, ok, 1, 16, 0, 0, fake, 0.1),          # heads not a multiple, empty batch
+        (4, 3, ok, 1, 16, 0, 0, fake, 0.1),          # heads not a multiple
+        (0, 2, _desc(lib, d=96), 1, 16, 0, 0, fake, 0.1),
+        (0, 2, ok, 1, 16, 0, 7, fake, 0.1),          # out_dtype
+        (0, 2, ok, 1, 16, 48, 0, fake, 0.1),         # partition not a multiple of 32
+        (2, 2, ok, -1, 16, 0, 0, fake, 0.1),         # negative max_blocks_per_seq
+        (2, 2, ok, 1, -5, 0, 0, fake, 0.1),          # negative max_context_len
+        (70000, 2, ok, 1, 16, 0, 0, fake, 0.1),      # too many sequences
+        (2, 2, ok, 1, 16, 0, 0, None, 0.1),          # NULL query
+        (2, 2, ok, 1, 16, 0, 0, odd, 0.1),           # misaligned query
+        (2, 2, ok, 1, 16, 0, 0, fake, float("nan")),  # NaN scale
+        (2, 2, _desc(lib, nb=0), 1, 16, 0, 0, fake, 0.1),  # empty pool
+        (0, 2, ok, 1, 16, 0, 0, fake, 0.1),          # valid, empty batch: PA_OK
+    ]
+    for S, H, desc, mb, mcl, part, odt, q, scale in cases:
+        a = L.pa_decode(fake, odt, q, S, H, fake, fake, ctypes.byref(desc), fake, mb, fake, mcl,
+                        scale, part, None, 0, None, None)
+        b = L.pa_decode_noalloc(fake, odt, q, S, H, fake, fake, ctypes.byref(desc), fake, mb,
+                                fake, mcl, scale, part, None, None)
+        assert a == b, (S, H, mb, mcl, part, odt, a, b)
+    assert L.pa_decode(fake, 0, fake, 0, 3, fake, fake, ctypes.byref(ok), fake, 1, fake, 16,
+                       0.1, 0, None, 0, None, None) == lib.PA_ERR_UNSUPPORTED
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(),
                     reason="would launch on fake pointers where a GPU exists")
 def test_grouped_decode_without_a_gpu_fails_cleanly(lib):

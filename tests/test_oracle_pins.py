@@ -148,6 +148,11 @@ MUTANTS = [
     ("fp8_row_scale", "*scale = amax / 448.0f;", "*scale = amax / 440.0f;"),
     ("fp8_no_saturation", "if (a >= 448.0)\n        return sign | 0x7e;",
      "if (a >= 480.0)\n        return sign | 0x7e;"),
+    ("write_source_row_ignores_token", "size_t src = (size_t)((t * num_heads + h) * head_dim);",
+     "size_t src = (size_t)((0 * num_heads + h) * head_dim);", 0),
+    ("fp8_write_source_row_ignores_token",
+     "size_t src = (size_t)((t * num_heads + h) * head_dim);",
+     "size_t src = (size_t)((0 * num_heads + h) * head_dim);", 1),
     ("write_value_from_key", "memcpy(value_cache + dst, value + src,",
      "memcpy(value_cache + dst, key + src,"),
     ("copy_value_from_key", "memcpy(value_caches[l] + dst * block_elems, value_caches[l] + src",

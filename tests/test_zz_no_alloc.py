@@ -49,23 +49,66 @@ def _call(pk, fn_name, t, c, partition, workspace=None):
     return out, err
 
 
+def _grouped_case(rng, ctxs, kv_heads, group, D, bs):
+    """A paged case with ``group`` query heads per K/V head."""
+    c = pc.paged_case(rng, ctxs, kv_heads, D, bs)
+    c["q"] = pc.to_storage_bits(
+        rng.standard_normal((len(ctxs), kv_heads * group, D), dtype=np.float32), "f16")
+    return c
+
+
+def _same_bits(a, b):
+    return torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_noalloc_matches_decode_on_consecutive_calls():
+    """Two calls in a row per case (and cases back to back on the same
+    array): each output is bit-identical to pa_decode's with a caller
+    workspace, since both run the same kernel with the same partitions and
+    merge them in the same order."""
     import paged_kv_cache_417_b200 as pk
     rng = np.random.default_rng(77)
-    cases = [  # split contexts (partials go through the scratch), then a second batch
+    cases = [  # split contexts (partials go through the scratch), then other batches
         (pc.paged_case(rng, [3000, 17, 1500, 4096, 1], 4, 128, 16), 256),
         (pc.paged_case(rng, [700, 2048, 33, 999], 8, 64, 32), 0),
+        (_grouped_case(rng, [5000, 40, 2600], 2, 4, 128, 16), 512),
     ]
     for c, partition in cases:
         t = _upload(c)
         S, H, D = c["q"].shape
         ws = pk.alloc_workspace(S, H, D, int(c["ctx"].max()), partition)
         ref, err_ref = _call(pk, "pa_decode", t, c, partition, ws)
-        got, err_got = _call(pk, "pa_decode_noalloc", t, c, partition)
+        first, err1 = _call(pk, "pa_decode_noalloc", t, c, partition)
+        second, err2 = _call(pk, "pa_decode_noalloc", t, c, partition)
         torch.cuda.synchronize()
-        assert int(err_ref.item()) == 0 and int(err_got.item()) == 0
-        assert bool(torch.isfinite(got).all())
-        assert float((got.float() - ref.float()).abs().max()) <= TOL
+        assert int(err_ref.item()) == 0 and int(err1.item()) == 0 and int(err2.item()) == 0
+        assert bool(torch.isfinite(first).all())
+        assert _same_bits(first, ref), "first call differs from pa_decode"
+        assert _same_bits(second, ref), "second call differs from pa_decode"
+        assert float((first.float() - ref.float()).abs().max()) <= TOL
+
+
+def test_noalloc_separate_merge_kernel_path():
+    """Grouped heads whose merge weights exceed the merging CTA's buffer
+    (8 heads x 1032 partitions of 32 tokens) take the separate merge kernel;
+    both calls match pa_decode bit for bit and the oracle within the
+    tolerance."""
+    import oracle
+    import paged_kv_cache_417_b200 as pk
+    rng = np.random.default_rng(78)
+    c = _grouped_case(rng, [33000, 700], 1, 8, 128, 16)
+    t = _upload(c)
+    S, H, D = c["q"].shape
+    ws = pk.alloc_workspace(S, H, D, int(c["ctx"].max()), 32)
+    assert ws.numel() <= pk.NOALLOC_SCRATCH_BYTES
+    ref, err_ref = _call(pk, "pa_decode", t, c, 32, ws)
+    got1, err1 = _call(pk, "pa_decode_noalloc", t, c, 32)
+    got2, err2 = _call(pk, "pa_decode_noalloc", t, c, 32)
+    torch.cuda.synchronize()
+    assert int(err_ref.item()) == 0 and int(err1.item()) == 0 and int(err2.item()) == 0
+    assert _same_bits(got1, ref) and _same_bits(got2, ref)
+    want = oracle.decode(c["q"], c["kpool"], c["vpool"], c["bt"], c["ctx"], c["scale"])
+    assert float(np.max(np.abs(got1.double().cpu().numpy() - want))) <= TOL
 
 
 def test_noalloc_rejects_work_beyond_its_scratch():
