@@ -206,14 +206,19 @@ def oracle_inputs(sub, layers):
     return [wl.host_pools(sub, li) for li in layers]
 
 
-def time_oracle(sub, layers, pools):
+def time_oracle(sub, layers, pools, results=None):
     """Seconds the oracle takes for the whole step of ``sub`` on ``layers``:
-    copy-on-write, K/V write, decode."""
+    copy-on-write, K/V write, decode. ``results`` (a list) receives the fp64
+    outputs of each layer."""
     import oracle
     t0 = time.perf_counter()
+    outs = []
     for li, (kc, vc) in zip(layers, pools):
-        oracle.default().step_on_pools(sub, li, kc, vc)
-    return time.perf_counter() - t0
+        outs.append(oracle.default().step_on_pools(sub, li, kc, vc))
+    secs = time.perf_counter() - t0
+    if results is not None:
+        results[:] = outs
+    return secs
 
 
 def oracle_sample(step, target_seconds):
@@ -233,23 +238,58 @@ def oracle_sample(step, target_seconds):
     return wl.subset(step, sorted(ids))
 
 
-def cpu_baseline(step, target_seconds=12.0):
+def accuracy(step, sub, layers, refs, gpu_outs):
+    """Max and mean |gpu - oracle| over every output element of the sampled
+    sequences and layers, the worst element, and whether all are within the
+    tolerance: 2e-3 for f16 outputs (fp8 caches have f16 rows), and
+    |o| * 2^-8 + 1e-3 for bf16 outputs (bf16 rounding alone can pass 2e-3)."""
+    ids = np.asarray(sub.meta["seq_ids"], dtype=np.int64)
+    worst, total, count, ok = (0.0, None), 0.0, 0, True
+    bf16 = step.io_dtype == "bf16"
+    for li, ref in zip(layers, refs):
+        got = gpu_outs[li][ids].double().cpu().numpy()
+        if not np.all(np.isfinite(got)):
+            return {"max_abs_err": float("inf"), "within_tolerance": False,
+                    "checked": "non-finite GPU output"}
+        err = np.abs(got - ref)
+        tol = np.abs(ref) * 2.0 ** -8 + 1e-3 if bf16 else 2e-3
+        ok = ok and bool(np.all(err <= tol))
+        k = int(np.argmax(err))
+        if err.flat[k] >= worst[0]:
+            s_, h_, d_ = np.unravel_index(k, err.shape)
+            worst = (float(err.flat[k]), {"layer": int(li), "seq": int(ids[s_]),
+                                          "head": int(h_), "dim": int(d_)})
+        total += float(err.sum())
+        count += err.size
+    return {"max_abs_err": worst[0], "mean_abs_err": total / max(count, 1),
+            "worst": worst[1], "within_tolerance": ok,
+            "tolerance": "|o|*2^-8 + 1e-3 (bf16 output)" if bf16 else 2e-3,
+            "checked": (f"{sub.num_seqs} of {step.num_seqs} sequences x layers "
+                        f"{list(layers)} of {step.num_layers}: outputs of the timed steps "
+                        f"vs the fp64 oracle outputs of the CPU-baseline sample")}
+
+
+def cpu_baseline(step, gpu_outs=None, target_seconds=12.0):
     """The oracle on this host's cores over a bounded sample of the workload,
-    repeated until about ``target_seconds`` of oracle work were timed."""
+    repeated until about ``target_seconds`` of oracle work were timed. With
+    ``gpu_outs`` (the outputs of the timed steps, per layer) the oracle's
+    outputs for the sample are also compared with them."""
     import oracle
     layers = [0] if step.num_layers == 1 else [0, step.num_layers - 1]
     sub = oracle_sample(step, target_seconds / len(layers))
     pools = oracle_inputs(sub, layers)
-    secs, reps = 0.0, 0
+    secs, reps, refs = 0.0, 0, []
     while reps == 0 or secs < 0.8 * target_seconds:
-        secs += time_oracle(sub, layers, pools)
+        secs += time_oracle(sub, layers, pools, refs)
         reps += 1
     value = sub.num_seqs * len(layers) * reps / (secs * step.num_layers)
-    return {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+    line = {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": (f"{sub.num_seqs} of {step.num_seqs} sequences x {len(layers)} of "
                        f"{step.num_layers} layers (copy-on-write, K/V write, decode), "
                        f"{reps} repetition(s), fp64 C + OpenMP, {secs:.1f} s; value scaled "
                        f"to whole decode steps")}
+    acc = accuracy(step, sub, layers, refs, gpu_outs) if gpu_outs is not None else None
+    return line, acc
 
 
 def block_manager_timing(step, reps=200):
@@ -303,7 +343,7 @@ def job_throughput(world, seqs_per_rank, steps, max_ms):
 
 
 def run_reference(args, config_desc):
-    step = WORKLOADS[args.config][0](SEEDS[args.config], args.kv_dtype)
+    step = make_step(args.config, 0, args.kv_dtype, args.kv_heads, args.seqs)
     sub = oracle_sample(step, 2.0)
     layers = [0]
     pools = oracle_inputs(sub, layers)
@@ -330,8 +370,291 @@ def run_reference(args, config_desc):
 
 
 # ----------------------------------------------------------------------------
-# The CUDA path.
+# The CUDA path: one step as the benchmark launches it (also driven by the
+# GPU tests of the benchmarked path).
 # ----------------------------------------------------------------------------
+
+def make_step(config, rank=0, kv_dtype="f16", kv_heads=0, seqs=0):
+    """The workload of ``config`` for replica ``rank`` (seed + 1000 * rank),
+    optionally with ``kv_heads`` K/V heads or ``seqs`` sequences."""
+    seed = SEEDS[config] + 1000 * rank
+    if seqs:
+        if config != "llama7b_layer":
+            raise ValueError("--seqs applies to llama7b_layer only")
+        return wl.llama_layer(seed=seed, num_seqs=seqs, num_blocks=max(256, 8192 * seqs // 96),
+                              dtype=kv_dtype)
+    if kv_heads:
+        if config == "llama7b_layer":
+            return wl.llama_layer(seed=seed, dtype=kv_dtype, num_kv_heads=kv_heads)
+        if config.startswith("full_step_bs"):
+            return wl.full_step(seed=seed, dtype=kv_dtype, num_kv_heads=kv_heads,
+                                block_size=int(config[len("full_step_bs"):]))
+        raise ValueError("--kv-heads applies to llama7b_layer and full_step_bs*")
+    return WORKLOADS[config][0](seed, kv_dtype)
+
+
+INTEGER_INPUTS = ("block_tables", "context_lens", "slot_mapping", "copy_pairs")
+
+
+def native_inputs(step):
+    """The step's integer inputs (block tables, context lengths, the new
+    tokens' slots, copy-on-write pairs) built by the library's C++ block
+    manager with pa_bm_prepare_decode, from the allocation history the
+    workload's Python allocator followed: the same free order, the shared
+    prefix forked to every sequence, each sequence's cached tokens, then one
+    appended token per sequence. Where the workload gives each partly filled
+    last block a second holder, the C++ side forks the whole sequence (a
+    parallel-sampling sibling) while the Python allocator adds a holder to
+    that block only: every block of such a sequence then counts one more
+    holder on the C++ side, and every decode input is the same. Returns a
+    dict of numpy arrays (plus the manager's reference counts under
+    "ref_count")."""
+    from paged_kv_cache_417_b200.block_manager import BlockManager
+    m = step.meta
+    S, bs = step.num_seqs, step.block_size
+    bm = BlockManager(step.num_blocks, bs, m["free_order"])
+    prefix = int(m["prefix_tokens"])
+    if prefix and S:
+        bm.add_sequence(0)
+        bm.allocate_tokens(0, prefix)
+        for s in range(1, S):
+            bm.fork(0, s)
+    else:
+        for s in range(S):
+            bm.add_sequence(s)
+    for s in range(S):
+        bm.allocate_tokens(s, int(m["pre_tokens"][s]))
+    if m["fork_partial_tail"]:
+        for s in range(S):
+            if bm.num_tokens(s) % bs:
+                bm.fork(s, S + s)
+    out = bm.prepare_decode(np.arange(S, dtype=np.int64), step.max_blocks_per_seq)
+    out["ref_count"] = bm.ref_counts()
+    return out
+
+
+def upload_step(step, dev, integer_inputs=None):
+    """All inputs of ``step`` on ``dev`` (fp8 pools wrapped for the binding).
+    ``integer_inputs`` (e.g. from :func:`native_inputs`) replaces the block
+    tables, context lengths, slots and copy-on-write pairs."""
+    import torch
+    import paged_kv_cache_417_b200 as pk
+    from workloads.device import device_step
+    d = device_step(step, dev)
+    if integer_inputs is not None:
+        for k in INTEGER_INPUTS:
+            d[k] = torch.from_numpy(np.ascontiguousarray(integer_inputs[k])).to(dev)
+    if step.dtype == "fp8":
+        for key in ("key_caches", "value_caches"):
+            d[key] = [pk.Fp8Cache(t, step.block_size, step.head_dim, torch.float16)
+                      for t in d[key]]
+    return d
+
+
+class StepLauncher:
+    """One decode step of the whole path for every layer of ``step``:
+    copy-on-write block copies (when the workload has any), then per layer
+    the fused K/V write + decode (``fused``) or pa_write_kv then pa_decode.
+    The caches in ``d`` are updated in place; outputs go to ``self.outs``
+    unless other output tensors are given. ``swap`` (swap-resume workload)
+    swaps the workload's host blocks in first."""
+
+    def __init__(self, step, d, dev, fused=True, partition=0, swap=None):
+        import torch
+        import paged_kv_cache_417_b200 as pk
+        self.pk, self.torch = pk, torch
+        self.step, self.d, self.dev = step, d, dev
+        self.fused, self.partition, self.swap = fused, partition, swap
+        self.outs = [torch.empty_like(q) for q in d["query"]]
+        S = step.num_seqs
+        self.ws = pk.alloc_workspace(S, step.num_heads, step.head_dim, step.max_context_len,
+                                     partition, dev)
+        self.P = pk.decode_partition_size(S, step.num_heads, d["key_caches"][0],
+                                          step.max_context_len, partition)
+        self.split = step.max_context_len > self.P
+        # Split partitions are merged by the last CTA of each sequence, unless
+        # the grid has more (sequence, head) slots than the workspace has
+        # arrival counters (then a separate reduce kernel runs).
+        self.reduce_launch = self.split and S * step.num_heads > 65536
+        self.has_copy = step.copy_pairs.shape[0] > 0
+
+    @property
+    def launches_per_step(self):
+        L = self.step.num_layers
+        n = (1 if self.has_copy else 0) + L * ((1 if self.fused else 2) +
+                                               (1 if self.reduce_launch else 0))
+        return n + (1 if self.swap is not None else 0)
+
+    def swap_in(self):
+        sw, d = self.swap, self.d
+        self.pk.swap_blocks(sw["host_k"], sw["host_v"], d["key_caches"], d["value_caches"],
+                            sw["map"])
+
+    def one_step(self, dec_events=None, inputs=None, out_list=None):
+        """Enqueue one step on the current stream; ``dec_events`` (two lists)
+        receive CUDA events around every decode call."""
+        pk, torch, step, d = self.pk, self.torch, self.step, self.d
+        src = inputs or d
+        dst = out_list or self.outs
+        stream = torch.cuda.current_stream(self.dev)
+        if self.swap is not None:
+            self.swap_in()
+        if self.has_copy:
+            pk.copy_blocks(d["key_caches"], d["value_caches"], src["copy_pairs"])
+        for li in range(step.num_layers):
+            kc, vc = d["key_caches"][li], d["value_caches"][li]
+            if not self.fused:
+                pk.write_kv(src["new_key"][li], src["new_value"][li], src["slot_mapping"], kc,
+                            vc)
+            if dec_events is not None:
+                dec_events[0].append(torch.cuda.Event(enable_timing=True))
+                dec_events[0][-1].record(stream)
+            if self.fused:
+                pk.write_kv_decode(dst[li], src["query"][li], src["new_key"][li],
+                                   src["new_value"][li], kc, vc, src["block_tables"],
+                                   src["context_lens"], step.max_context_len,
+                                   float(step.scale), partition_size=self.partition,
+                                   workspace=self.ws)
+            else:
+                pk.decode(dst[li], src["query"][li], kc, vc, src["block_tables"],
+                          src["context_lens"], step.max_context_len, float(step.scale),
+                          partition_size=self.partition, workspace=self.ws)
+            if dec_events is not None:
+                dec_events[1].append(torch.cuda.Event(enable_timing=True))
+                dec_events[1][-1].record(stream)
+
+    def capture(self, inputs=None, out_list=None):
+        """The whole step recorded once as a CUDA graph (the library only
+        enqueues kernels on the current stream, allocates nothing and never
+        synchronises, so it can be captured)."""
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.one_step(inputs=inputs, out_list=out_list)
+        torch.cuda.synchronize(self.dev)
+        return g
+
+
+def make_swap(step, d, dev):
+    """Swap-resume workload: a pinned host pool holds the blocks of every 4th
+    sequence; each step swaps them into their GPU blocks first."""
+    import torch
+    S, L = step.num_seqs, step.num_layers
+    blocks = sorted({int(b) for s_ in range(0, S, 4) for b in step.block_tables[s_] if b >= 0})
+    idx = torch.tensor(blocks, device=dev)
+    hk = [d["key_caches"][li][idx].cpu().pin_memory() for li in range(L)]
+    hv = [d["value_caches"][li][idx].cpu().pin_memory() for li in range(L)]
+    return {"host_k": hk, "host_v": hv, "blocks": len(blocks),
+            "map": torch.tensor([[i, b] for i, b in enumerate(blocks)], dtype=torch.int64,
+                                device=dev),
+            "bytes": 2 * L * len(blocks) * hk[0][0].numel() * hk[0].element_size()}
+
+
+class E2EPipeline:
+    """End to end through the public API with host buffers: every step copies
+    its inputs from pinned host memory to the device and its outputs back, as
+    one packed DMA each way. Two input/output buffer sets and a copy stream
+    each way pipeline the steps, so a step's copies overlap its neighbours'
+    compute on the copy engines. With ``graph`` every buffer set has its own
+    captured step."""
+
+    def __init__(self, launcher, graph=True):
+        import torch
+        self.torch, self.launcher, self.graph = torch, launcher, graph
+        d, dev, L = launcher.d, launcher.dev, launcher.step.num_layers
+        names = [(k, i) for k in ("query", "new_key", "new_value") for i in range(L)]
+        names += [(k, None) for k in ("slot_mapping", "block_tables", "context_lens")]
+        if launcher.has_copy:
+            names.append(("copy_pairs", None))
+
+        def tensor_of(name):
+            k, i = name
+            return d[k][i] if i is not None else d[k]
+
+        layout, off = [], 0
+        for nm in names:
+            t = tensor_of(nm)
+            nbytes = t.numel() * t.element_size()
+            layout.append((nm, off, nbytes, t.dtype, t.shape))
+            off = (off + nbytes + 255) // 256 * 256
+        self.h2d = off
+        self.host_in = torch.empty(self.h2d, dtype=torch.uint8, pin_memory=True)
+        for nm, o, nbytes, _, _ in layout:
+            self.host_in[o:o + nbytes].copy_(tensor_of(nm).reshape(-1).view(torch.uint8).cpu())
+        self.out_meta = [(o.dtype, o.shape, o.numel() * o.element_size())
+                         for o in launcher.outs]
+        self.d2h = sum(m[2] for m in self.out_meta)
+
+        def views(buf):
+            v = {"query": [None] * L, "new_key": [None] * L, "new_value": [None] * L,
+                 "copy_pairs": d["copy_pairs"]}
+            for (k, i), o, nbytes, dt, shape in layout:
+                t = buf[o:o + nbytes].view(dt).view(shape)
+                if i is None:
+                    v[k] = t
+                else:
+                    v[k][i] = t
+            return v
+
+        self.bufs = []
+        for _ in range(2):
+            dev_in = torch.empty(self.h2d, dtype=torch.uint8, device=dev)
+            dev_out = torch.empty(self.d2h, dtype=torch.uint8, device=dev)
+            bf = {"dev_in": dev_in, "in": views(dev_in), "dev_out": dev_out,
+                  "out": self._split(dev_out),
+                  "host_out": torch.empty(self.d2h, dtype=torch.uint8, pin_memory=True)}
+            if graph:
+                bf["graph"] = launcher.capture(inputs=bf["in"], out_list=bf["out"])
+            self.bufs.append(bf)
+        self.up, self.down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        self.ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("h2d", "step", "d2h")}
+
+    def _split(self, flat):
+        outs, o = [], 0
+        for dt, shape, nb in self.out_meta:
+            outs.append(flat[o:o + nb].view(dt).view(shape))
+            o += nb
+        return outs
+
+    def host_outputs(self, b):
+        """The outputs of the last step that ran on buffer set ``b``, as
+        copied to pinned host memory (call after synchronising)."""
+        return self._split(self.bufs[b]["host_out"])
+
+    def run(self, n, sleep_s=0.0):
+        """Enqueue ``n`` end-to-end steps; returns the (start, end) timing
+        events, recorded on the upload and download streams."""
+        torch, ev, up, down = self.torch, self.ev, self.up, self.down
+        stream = torch.cuda.current_stream(self.launcher.dev)
+        with torch.cuda.stream(up):
+            if sleep_s:
+                torch.cuda._sleep(int(sleep_s * 2.0e9))
+            t0 = torch.cuda.Event(enable_timing=True)
+            t0.record(up)
+        for k in range(n):
+            b = k % 2
+            bf = self.bufs[b]
+            with torch.cuda.stream(up):
+                if k >= 2:
+                    up.wait_event(ev["step"][b])  # step k-2 has read these inputs
+                bf["dev_in"].copy_(self.host_in, non_blocking=True)
+                ev["h2d"][b].record(up)
+            stream.wait_event(ev["h2d"][b])
+            if k >= 2:
+                stream.wait_event(ev["d2h"][b])  # outputs of step k-2 copied out
+            if self.graph:
+                bf["graph"].replay()
+            else:
+                self.launcher.one_step(inputs=bf["in"], out_list=bf["out"])
+            ev["step"][b].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(ev["step"][b])
+                bf["host_out"].copy_(bf["dev_out"], non_blocking=True)
+                ev["d2h"][b].record(down)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t1.record(down)
+        return t0, t1
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -353,6 +676,9 @@ def main():
                     help="pa_write_kv then pa_decode instead of the fused pa_write_kv_decode")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step from the host instead of replaying a CUDA graph")
+    ap.add_argument("--inputs", default="native", choices=["native", "python"],
+                    help="which block manager builds the step's integer inputs: the "
+                         "library's C++ one (default) or the Python allocator of workloads/")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -379,8 +705,6 @@ def main():
         return
 
     import torch
-    import paged_kv_cache_417_b200 as pk
-    from workloads.device import device_step
 
     dist = None
     if world > 1:
@@ -390,46 +714,34 @@ def main():
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
 
+    try:
+        step = make_step(args.config, rank, args.kv_dtype, args.kv_heads, args.seqs)
+    except ValueError as e:
+        ap.error(str(e))
     if args.seqs:
-        if args.config != "llama7b_layer":
-            ap.error("--seqs applies to llama7b_layer only")
-        step = wl.llama_layer(seed=SEEDS[args.config] + 1000 * rank, num_seqs=args.seqs,
-                              num_blocks=max(256, 8192 * args.seqs // 96), dtype=args.kv_dtype)
         config_desc["workload"] += f" (reduced to {args.seqs} seqs)"
     elif args.kv_heads:
-        seed = SEEDS[args.config] + 1000 * rank
-        if args.config == "llama7b_layer":
-            step = wl.llama_layer(seed=seed, dtype=args.kv_dtype, num_kv_heads=args.kv_heads)
-        elif args.config.startswith("full_step_bs"):
-            step = wl.full_step(seed=seed, dtype=args.kv_dtype, num_kv_heads=args.kv_heads,
-                                block_size=int(args.config[len("full_step_bs"):]))
-        else:
-            ap.error("--kv-heads applies to llama7b_layer and full_step_bs*")
         config_desc["workload"] += f" with {args.kv_heads} K/V heads (grouped query heads)"
-    else:
-        step = WORKLOADS[args.config][0](SEEDS[args.config] + 1000 * rank, args.kv_dtype)
     if args.kv_dtype != "f16":
         config_desc["kv_dtype"] = args.kv_dtype
-    d = device_step(step, dev)
-    if step.dtype == "fp8":
-        for key in ("key_caches", "value_caches"):
-            d[key] = [pk.Fp8Cache(t, step.block_size, step.head_dim, torch.float16)
-                      for t in d[key]]
-    L, S = step.num_layers, step.num_seqs
+    native = None
+    if args.inputs == "native":
+        native = native_inputs(step)
+        for k in INTEGER_INPUTS:
+            if not np.array_equal(native[k], getattr(step, k)):
+                raise SystemExit(f"C++ block manager's {k} differs from the workload's")
+        config_desc["inputs"] = ("block tables, context lengths, slots and copy-on-write pairs "
+                                 "from the C++ block manager (pa_bm_prepare_decode); equal to "
+                                 "the Python allocator's")
+    else:
+        config_desc["inputs"] = "integer inputs from the Python allocator of workloads/"
+    d = upload_step(step, dev, native)
+    S = step.num_seqs
     stream = torch.cuda.current_stream(dev)
-    outs = [torch.empty_like(q) for q in d["query"]]
-    ws = pk.alloc_workspace(S, step.num_heads, step.head_dim, step.max_context_len,
-                            args.partition, dev)
-    P = pk.decode_partition_size(S, step.num_heads, d["key_caches"][0], step.max_context_len,
-                                 args.partition)
-    split = step.max_context_len > P
-    # Split partitions are merged by the last CTA of each sequence, unless
-    # the grid has more (sequence, head) slots than the workspace has
-    # arrival counters (then a separate reduce kernel runs).
-    reduce_launch = split and S * step.num_heads > 65536
-    has_copy = step.copy_pairs.shape[0] > 0
-    launches_per_step = (1 if has_copy else 0) + L * ((1 if args.fused else 2) +
-                                                       (1 if reduce_launch else 0))
+    swap = make_swap(step, d, dev) if args.config == "swap_resume" else None
+    launcher = StepLauncher(step, d, dev, fused=args.fused, partition=args.partition, swap=swap)
+    outs, P, split = launcher.outs, launcher.P, launcher.split
+    one_step = launcher.one_step
     # L2 flush by reading 256 MiB: the previous step's lines are evicted and
     # L2 is left holding clean lines, so no write-back lands on the next step.
     flush_buf = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
@@ -437,55 +749,6 @@ def main():
     def flush_l2():
         if flush:
             flush_buf.sum()
-
-    # Swap-resume workload: a pinned host pool holds the blocks of every 4th
-    # sequence; each step swaps them into their GPU blocks first.
-    swap = None
-    if args.config == "swap_resume":
-        blocks = sorted({int(b) for s_ in range(0, S, 4) for b in step.block_tables[s_]
-                         if b >= 0})
-        hk = [d["key_caches"][li][torch.tensor(blocks, device=dev)].cpu().pin_memory()
-              for li in range(L)]
-        hv = [d["value_caches"][li][torch.tensor(blocks, device=dev)].cpu().pin_memory()
-              for li in range(L)]
-        swap = {"host_k": hk, "host_v": hv, "blocks": len(blocks),
-                "map": torch.tensor([[i, b] for i, b in enumerate(blocks)],
-                                    dtype=torch.int64, device=dev),
-                "bytes": 2 * L * len(blocks) * hk[0][0].numel() * hk[0].element_size()}
-        launches_per_step += 1
-
-    def swap_in():
-        pk.swap_blocks(swap["host_k"], swap["host_v"], d["key_caches"], d["value_caches"],
-                       swap["map"])
-
-    def one_step(dec_events=None, inputs=None, out_list=None):
-        src = inputs or d
-        dst = out_list or outs
-        if swap is not None:
-            swap_in()
-        if has_copy:
-            pk.copy_blocks(d["key_caches"], d["value_caches"], src["copy_pairs"])
-        for li in range(L):
-            kc, vc = d["key_caches"][li], d["value_caches"][li]
-            if not args.fused:
-                pk.write_kv(src["new_key"][li], src["new_value"][li], src["slot_mapping"], kc,
-                            vc)
-            if dec_events is not None:
-                dec_events[0].append(torch.cuda.Event(enable_timing=True))
-                dec_events[0][-1].record(stream)
-            if args.fused:
-                pk.write_kv_decode(dst[li], src["query"][li], src["new_key"][li],
-                                   src["new_value"][li], kc, vc, src["block_tables"],
-                                   src["context_lens"], step.max_context_len,
-                                   float(step.scale), partition_size=args.partition,
-                                   workspace=ws)
-            else:
-                pk.decode(dst[li], src["query"][li], kc, vc, src["block_tables"],
-                          src["context_lens"], step.max_context_len, float(step.scale),
-                          partition_size=args.partition, workspace=ws)
-            if dec_events is not None:
-                dec_events[1].append(torch.cuda.Event(enable_timing=True))
-                dec_events[1][-1].record(stream)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -516,19 +779,9 @@ def main():
         secs = min(1.0, 1.5 * args.steps * host_step_s + 0.002)
         torch.cuda._sleep(int(secs * 2.0e9))
 
-    def capture(inputs=None, out_list=None):
-        """The whole step recorded once as a CUDA graph (the library only
-        enqueues kernels on the current stream, allocates nothing and never
-        synchronises, so it can be captured)."""
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            one_step(inputs=inputs, out_list=out_list)
-        torch.cuda.synchronize(dev)
-        return g
-
     run_step = one_step
     if args.graph:
-        graph_main = capture()
+        graph_main = launcher.capture()
         run_step = lambda dec_events=None, inputs=None: graph_main.replay()  # noqa: E731
         for _ in range(args.warmup):
             flush_l2()
@@ -563,6 +816,9 @@ def main():
         run_step(dec_events)
         ends[k].record(stream)
     barrier()
+    # The outputs of the timed (graph-replayed) steps, kept for the accuracy
+    # check against the oracle's outputs in the CPU-baseline leg.
+    timed_outs = [o.clone() for o in outs]
     if args.graph:
         # Decode events cannot sit inside a replayed graph: time the decode
         # calls on the eager path, same steps, for the roofline.
@@ -601,7 +857,7 @@ def main():
         barrier()
         for k in range(args.steps):
             ev0[k].record(stream)
-            swap_in()
+            launcher.swap_in()
             ev1[k].record(stream)
         barrier()
         swap_s = statistics.mean(a.elapsed_time(b) for a, b in zip(ev0, ev1)) / 1e3
@@ -624,109 +880,31 @@ def main():
                       "pinned_memcpy_gbs": swap["bytes"] / ref_s / 1e9,
                       "frac_of_memcpy": ref_s / swap_s}
 
-    # End to end through the public API with host buffers: every step copies
-    # its inputs from pinned host memory to the device and its outputs back,
-    # as one packed DMA each way. Two input/output buffer sets and a copy
-    # stream pipeline the steps, so a step's copies overlap its neighbours'
-    # compute on the copy engines. No L2 flush here: every step reads more
-    # K/V than L2 holds.
+    # End to end through the public API with host buffers (E2EPipeline). No
+    # L2 flush here: every step reads more K/V than L2 holds.
     e2e = None
     if not args.no_e2e:
-        names = [(k, i) for k in ("query", "new_key", "new_value") for i in range(L)]
-        names += [(k, None) for k in ("slot_mapping", "block_tables", "context_lens")]
-        if has_copy:
-            names.append(("copy_pairs", None))
-
-        def tensor_of(name):
-            k, i = name
-            return d[k][i] if i is not None else d[k]
-
-        layout, off = [], 0
-        for nm in names:
-            t = tensor_of(nm)
-            nbytes = t.numel() * t.element_size()
-            layout.append((nm, off, nbytes, t.dtype, t.shape))
-            off = (off + nbytes + 255) // 256 * 256
-        h2d = off
-        host_in = torch.empty(h2d, dtype=torch.uint8, pin_memory=True)
-        for nm, o, nbytes, _, _ in layout:
-            host_in[o:o + nbytes].copy_(tensor_of(nm).reshape(-1).view(torch.uint8).cpu())
-        out_bytes = [o.numel() * o.element_size() for o in outs]
-        d2h = sum(out_bytes)
-
-        def views(buf):
-            v = {"query": [None] * L, "new_key": [None] * L, "new_value": [None] * L,
-                 "copy_pairs": d["copy_pairs"]}
-            for (k, i), o, nbytes, dt, shape in layout:
-                t = buf[o:o + nbytes].view(dt).view(shape)
-                if i is None:
-                    v[k] = t
-                else:
-                    v[k][i] = t
-            return v
-
-        bufs = []
-        for _ in range(2):
-            dev_in = torch.empty(h2d, dtype=torch.uint8, device=dev)
-            dev_out = torch.empty(d2h, dtype=torch.uint8, device=dev)
-            out_list, o = [], 0
-            for ref, nb in zip(outs, out_bytes):
-                out_list.append(dev_out[o:o + nb].view(ref.dtype).view(ref.shape))
-                o += nb
-            bf = {"dev_in": dev_in, "in": views(dev_in), "dev_out": dev_out, "out": out_list,
-                  "host_out": torch.empty(d2h, dtype=torch.uint8, pin_memory=True)}
-            if args.graph:
-                bf["graph"] = capture(inputs=bf["in"], out_list=bf["out"])
-            bufs.append(bf)
-        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)  # H2D and D2H copy streams
-        ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("h2d", "step", "d2h")}
-
-        def e2e_run(n, sleep_s=0.0):
-            with torch.cuda.stream(up):
-                if sleep_s:
-                    torch.cuda._sleep(int(sleep_s * 2.0e9))
-                t0 = torch.cuda.Event(enable_timing=True)
-                t0.record(up)
-            for k in range(n):
-                b = k % 2
-                bf = bufs[b]
-                with torch.cuda.stream(up):
-                    if k >= 2:
-                        up.wait_event(ev["step"][b])  # step k-2 has read these inputs
-                    bf["dev_in"].copy_(host_in, non_blocking=True)
-                    ev["h2d"][b].record(up)
-                stream.wait_event(ev["h2d"][b])
-                if k >= 2:
-                    stream.wait_event(ev["d2h"][b])  # outputs of step k-2 copied out
-                if args.graph:
-                    bf["graph"].replay()
-                else:
-                    one_step(inputs=bf["in"], out_list=bf["out"])
-                ev["step"][b].record(stream)
-                with torch.cuda.stream(down):
-                    down.wait_event(ev["step"][b])
-                    bf["host_out"].copy_(bf["dev_out"], non_blocking=True)
-                    ev["d2h"][b].record(down)
-            t1 = torch.cuda.Event(enable_timing=True)
-            t1.record(down)
-            return t0, t1
-
+        pipe = E2EPipeline(launcher, graph=args.graph)
         barrier()
         h0 = time.perf_counter()
-        e2e_run(args.warmup)
+        pipe.run(args.warmup)
         host_e2e_s = (time.perf_counter() - h0) / args.warmup
         barrier()
-        t0, t1 = e2e_run(args.steps, min(1.0, 1.5 * args.steps * host_e2e_s + 0.002))
+        t0, t1 = pipe.run(args.steps, min(1.0, 1.5 * args.steps * host_e2e_s + 0.002))
         barrier()
         e2e_ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
+        # What the host received must be what the device-timed steps computed.
+        same = all(torch.equal(h.to(dev).view(torch.uint8), o.view(torch.uint8))
+                   for b in range(2) for h, o in zip(pipe.host_outputs(b), timed_outs))
         e2e = {"value": job_throughput(world, S, args.steps, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "h2d_bytes_per_step": pipe.h2d, "d2h_bytes_per_step": pipe.d2h,
+               "outputs_equal_device_timed": bool(same),
                "how": "one packed pinned-host DMA each way per step, 2 buffer sets, "
                       "separate upload and download streams overlapping compute"}
 
-    cpu = None
+    cpu, acc = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(step)
+        cpu, acc = cpu_baseline(step, timed_outs)
     bm_timing = block_manager_timing(step) if rank == 0 else None
 
     if rank == 0:
@@ -737,7 +915,8 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": step.dtype,
             "accumulate": "f32", "data": "synthetic", "config": config_desc,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+            "max_abs_err": acc["max_abs_err"] if acc else None, "accuracy": acc,
+            "gpu_launches": launcher.launches_per_step * args.steps, "clocks": clocks,
             "host_paced_value": paced, "host_block_manager": bm_timing, "swap": swap_stats,
             "partition_size": P, "split": split,
         }

@@ -30,14 +30,11 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().double().numpy()
 
 
-def run_step(step, layers=None, partition_size=0, out_dtype=None, keep_pre=False):
+def run_step(step, layers=None, partition_size=0, out_dtype=None):
     """copy_blocks (all layers) -> per layer write_kv, decode. Returns
     (outs list, device dict, dev_err int)."""
     layers = list(range(step.num_layers)) if layers is None else list(layers)
     d = wrap_caches(step, device_step(step, "cuda", layers))
-    if keep_pre:
-        d["pre_key"] = [k.clone() for k in d["key_caches"]]
-        d["pre_value"] = [v.clone() for v in d["value_caches"]]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     if step.copy_pairs.shape[0]:
         pk.copy_blocks(d["key_caches"], d["value_caches"], d["copy_pairs"], dev_err=err)
@@ -52,6 +49,39 @@ def run_step(step, layers=None, partition_size=0, out_dtype=None, keep_pre=False
         outs.append(out)
     torch.cuda.synchronize()
     return outs, d, int(err.item())
+
+
+def err_report(gpu_out: torch.Tensor, ref: np.ndarray):
+    """(max |gpu - ref|, mean |gpu - ref|, worst index) over every element."""
+    got = to_f64(gpu_out)
+    assert got.shape == ref.shape
+    assert np.all(np.isfinite(got)), "non-finite output"
+    if not ref.size:
+        return 0.0, 0.0, ()
+    err = np.abs(got - ref)
+    k = int(np.argmax(err))
+    return float(err.flat[k]), float(err.mean()), tuple(int(i) for i in
+                                                         np.unravel_index(k, err.shape))
+
+
+def check_outputs_and_pools(step, outs, d, layers, tol=TOL, out_index=None):
+    """Every output element of ``layers`` against the oracle's full step
+    (copy-on-write, write, decode) on the same inputs, and both pools of
+    those layers byte for byte. ``out_index(li)`` gives the position of layer
+    ``li`` in ``outs`` and ``d`` (default: li)."""
+    import oracle
+    for li in layers:
+        i = li if out_index is None else out_index(li)
+        ref, kref, vref = oracle.run_step(step, li)
+        mx, mean, worst = err_report(outs[i], ref)
+        assert mx <= tol, (f"{step.name} layer {li}: max err {mx:.3e} at (s, h, d) = {worst}, "
+                           f"mean {mean:.3e}")
+        for pool, want in ((d["key_caches"][i], kref), (d["value_caches"][i], vref)):
+            got = to_bits(pool)
+            if not np.array_equal(got, want):
+                bad = np.argwhere(got != want)
+                raise AssertionError(f"{step.name} layer {li}: pool differs at {bad[:3].tolist()} "
+                                     f"({len(bad)} elements)")
 
 
 def max_err(gpu_out: torch.Tensor, ref: np.ndarray) -> float:

@@ -6,6 +6,7 @@ import pytest
 
 import paged_kv_cache_417_b200 as pk
 from paged_kv_cache_417_b200.block_manager import BlockManager
+import workloads as wl
 from workloads import (BlockAllocator, Sequence, allocate_tokens, append_token,
                        check_invariants, free_sequence)
 
@@ -164,3 +165,43 @@ def test_prefix_sharing_reading_of_the_workload():
     assert len(res["copy_pairs"]) == int(np.sum(suffix % bs != 0))
     assert not set(res["copy_pairs"][:, 0].tolist()) & set(prefix)
     assert all(cc.ref_count(b) == 16 for b in prefix)   # 8 sequences + 8 siblings
+
+
+NATIVE_CASES = [
+    ("tiny", lambda: wl.tiny()),
+    ("llama7b_layer", lambda: wl.llama_layer()),
+    ("long_context", lambda: wl.long_context()),
+    ("prefix_cow", lambda: wl.prefix_cow()),
+    ("full_step_bs8", lambda: wl.full_step(block_size=8, num_layers=1)),
+    ("full_step_bs16", lambda: wl.full_step(block_size=16, num_layers=1)),
+    ("full_step_bs32", lambda: wl.full_step(block_size=32, num_layers=1)),
+]
+
+
+@pytest.mark.parametrize("name,make", NATIVE_CASES, ids=[c[0] for c in NATIVE_CASES])
+def test_native_step_inputs_equal_python_allocator(name, make):
+    """The benchmark's default inputs: the C++ block manager, replaying each
+    workload's allocation history, produces the same block tables, context
+    lengths, slots and copy-on-write pairs as the Python allocator. Where the
+    workload forks a sibling for each partly filled last block, the C++
+    sibling holds the whole pre-step sequence (the Python one its last block
+    only): reference counts differ by exactly those extra holdings."""
+    import bench
+    st = make()
+    got = bench.native_inputs(st)
+    for k in bench.INTEGER_INPUTS:
+        assert np.array_equal(got[k], getattr(st, k)), k
+    extra = np.zeros(st.num_blocks, dtype=np.int64)
+    if st.meta["fork_partial_tail"]:
+        bs = st.block_size
+        pre = st.context_lens.astype(np.int64) - 1
+        for s in range(st.num_seqs):
+            if pre[s] % bs:
+                n_pre = -(-pre[s] // bs)
+                table = st.block_tables[s, :n_pre].copy()
+                if st.copy_pairs.shape[0]:
+                    moved = dict(st.copy_pairs.tolist())
+                    inv = {dst: src for src, dst in moved.items()}
+                    table[-1] = inv.get(int(table[-1]), table[-1])
+                extra[table[:-1]] += 1
+    assert np.array_equal(got["ref_count"], st.ref_count + extra)

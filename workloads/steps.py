@@ -223,7 +223,14 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
         valid_slots=valid, base=base, layers=layers,
         ref_count=alloc.ref_count.copy(),
         meta={"allocator": alloc, "seqs": seqs, "phantom_holders": phantom,
-              "prefix_tokens": prefix_tokens}, num_kv_heads=Hk)
+              "prefix_tokens": prefix_tokens,
+              # The allocation history, for replaying the same step on
+              # another block manager: free order, cached tokens per
+              # sequence (the suffix when there is a shared prefix), and
+              # whether each partly filled last block has a second holder.
+              "free_order": np.asarray(order, dtype=np.int64).copy(),
+              "pre_tokens": np.asarray(pre_tokens, dtype=np.int64).copy(),
+              "fork_partial_tail": bool(fork_partial_tail)}, num_kv_heads=Hk)
     return step
 
 
