@@ -382,7 +382,7 @@ def make_step(config, rank=0, kv_dtype="f16", kv_heads=0, seqs=0):
         if config != "llama7b_layer":
             raise ValueError("--seqs applies to llama7b_layer only")
         return wl.llama_layer(seed=seed, num_seqs=seqs, num_blocks=max(256, 8192 * seqs // 96),
-                              dtype=kv_dtype)
+                              dtype=kv_dtype, num_kv_heads=kv_heads or None)
     if kv_heads:
         if config == "llama7b_layer":
             return wl.llama_layer(seed=seed, dtype=kv_dtype, num_kv_heads=kv_heads)
@@ -471,11 +471,13 @@ class StepLauncher:
                                      partition, dev)
         self.P = pk.decode_partition_size(S, step.num_heads, d["key_caches"][0],
                                           step.max_context_len, partition)
-        self.split = step.max_context_len > self.P
+        # P == 0: grouped heads whose token ranges are balanced per launch
+        # (pieces of a split sequence merged inside the same kernel).
+        self.split = self.P == 0 or step.max_context_len > self.P
         # Split partitions are merged by the last CTA of each sequence, unless
         # the grid has more (sequence, head) slots than the workspace has
         # arrival counters (then a separate reduce kernel runs).
-        self.reduce_launch = self.split and S * step.num_heads > 65536
+        self.reduce_launch = self.P > 0 and self.split and S * step.num_heads > 65536
         self.has_copy = step.copy_pairs.shape[0] > 0
 
     @property
@@ -720,7 +722,7 @@ def main():
         ap.error(str(e))
     if args.seqs:
         config_desc["workload"] += f" (reduced to {args.seqs} seqs)"
-    elif args.kv_heads:
+    if args.kv_heads:
         config_desc["workload"] += f" with {args.kv_heads} K/V heads (grouped query heads)"
     if args.kv_dtype != "f16":
         config_desc["kv_dtype"] = args.kv_dtype
@@ -918,7 +920,7 @@ def main():
             "max_abs_err": acc["max_abs_err"] if acc else None, "accuracy": acc,
             "gpu_launches": launcher.launches_per_step * args.steps, "clocks": clocks,
             "host_paced_value": paced, "host_block_manager": bm_timing, "swap": swap_stats,
-            "partition_size": P, "split": split,
+            "partition_size": P if P else "balanced per launch", "split": split,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -3,13 +3,19 @@
 // sm_100a: 16-bit caches, and fp8 (e4m3) caches with f16 rows and head_dim
 // 128 (2 <= G <= 16 for both; the kernel itself also handles G = 1).
 //
-// Query heads kvh*G .. kvh*G+G-1 all attend over K/V head kvh. A CTA takes
-// the unit (K/V head kvh, sequence s, partition p) for the whole group, so
-// each K/V byte crosses HBM once per group instead of once per query head,
-// and the G query rows share every staged tile. The outputs, the split
-// workspace and the merge of partitions are those of decode_split_kernel
-// (per query head; the last CTA of a (K/V head, sequence) merges its G
-// heads).
+// Query heads kvh*G .. kvh*G+G-1 all attend over K/V head kvh. A CTA works
+// on (K/V head, sequence) units for the whole group, so each K/V byte
+// crosses HBM once per group instead of once per query head, and the G query
+// rows share every staged tile. Two kernels share the staging and the math
+// (GroupWarp):
+//   decode_group_kernel  one CTA per (K/V head kvh, sequence s, partition p)
+//                        of a fixed partition size; the outputs, the split
+//                        workspace and the merge of partitions are those of
+//                        decode_split_kernel (per query head; the last CTA
+//                        of a (K/V head, sequence) merges its G heads).
+//   decode_flat_kernel   a persistent launch in which every CTA streams an
+//                        equal share of all the launch's chunks, across
+//                        unit boundaries (described before it below).
 //
 // Staging: each pool is viewed as a 3-D tensor for the TMA unit. 16-bit
 // pools: (64 elements, D/64 128-byte units, rows), row = one token of one
@@ -72,36 +78,43 @@ namespace pagedkv {
 
 constexpr int kGroupMaxHeads = 16;
 
-
 struct GroupParams {
     CUtensorMap tk; // key pool (see the staging note above), 128B swizzle
     CUtensorMap tv; // value pool, same geometry
     DecodeParams p;
+    int32_t num_ctas; // decode_flat_kernel: CTAs of the launch (balanced ranges)
 };
 
-template <typename T, int D, int BS, int NW, int NS> struct GroupCfg {
+// Stage geometry of the grouped kernels (independent of the block size).
+template <typename T, int D> struct GroupGeom {
     static_assert(D == 64 || D == 128, "head_dim");
-    static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
     static constexpr bool kFp8 = std::is_same<T, E4M3>::value;
     static_assert(!kFp8 || D == 128, "fp8 rows of 128 bytes");
-    static constexpr int kRow = D * (kFp8 ? 1 : 2);        // bytes per cached row
-    static constexpr int kUnits = kRow / 128;              // 128-byte units per row
-    static constexpr int kChunk = kFp8 ? 32 : 16;          // tokens per stage
-    static constexpr int kHalf = kChunk * kRow;            // the K (or V) codes of a stage
+    static constexpr int kRow = D * (kFp8 ? 1 : 2);  // bytes per cached row
+    static constexpr int kUnits = kRow / 128;        // 128-byte units per row
+    static constexpr int kChunk = kFp8 ? 32 : 16;    // tokens per stage
+    static constexpr int kHalf = kChunk * kRow;      // the K (or V) codes of a stage
     static constexpr int kStage = 2 * kHalf;
-    static constexpr int kRing = NS * kStage;              // one warp's stages
+    static constexpr int kMergeStride = D + 2;       // a row's (O, m, l) in a merge area
+    static_assert(kHalf % 1024 == 0, "swizzle atoms");
+};
+
+template <typename T, int D, int BS, int NW, int NS> struct GroupCfg : GroupGeom<T, D> {
+    using Geo = GroupGeom<T, D>;
+    static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
+    static constexpr int kRing = NS * Geo::kStage;         // one warp's stages
     static constexpr int kSeg = BS < 16 ? BS : 16;         // rows per TMA box
     static constexpr int kRingsBytes = NW * kRing;
     static constexpr int kBarBytes = NW * NS * 8;
     // fp8 row scales: per warp, [stage][K | V][kChunk] floats.
-    static constexpr int kScaleBytes = kFp8 ? NW * NS * 2 * kChunk * 4 : 0;
+    static constexpr int kScaleBytes = Geo::kFp8 ? NW * NS * 2 * Geo::kChunk * 4 : 0;
     static constexpr int kRankBytes = kRankMaxSeqs * 4; // context lengths for ranking
     static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kScaleBytes + kRankBytes;
-    // After its last chunk a warp leaves (O, m, l) of its rows in its ring.
-    static constexpr int kMergeStride = D + 2;
-    static_assert(kGroupMaxHeads * kMergeStride * 4 <= kRing, "merge area fits a ring");
-    static_assert(kHalf % 1024 == 0 && (kSeg * kRow) % 1024 == 0, "swizzle atoms");
-    static_assert(kChunk % kSeg == 0 && kChunk % 16 == 0, "chunk geometry");
+    // After its last chunk a warp of decode_group_kernel leaves (O, m, l) of
+    // its rows in its ring.
+    static_assert(kGroupMaxHeads * Geo::kMergeStride * 4 <= kRing, "merge area fits a ring");
+    static_assert((kSeg * Geo::kRow) % 1024 == 0, "swizzle atoms");
+    static_assert(Geo::kChunk % kSeg == 0 && Geo::kChunk % 16 == 0, "chunk geometry");
     // 1 KiB of slack to align the rings to 1024 bytes.
     static size_t smem_bytes(int partition)
     {
@@ -136,61 +149,73 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
     return y;
 }
 
-// T: __half, __nv_bfloat16 (cache, query and new-row type) or E4M3 (codes;
-// query and new rows are f16). TWO: G > 8 (fragment rows 8-15 are live).
-template <typename T, int D, int BS, int NW, int NS, bool TWO>
-__global__ void __launch_bounds__(NW * 32)
-    decode_group_kernel(const __grid_constant__ GroupParams gp)
-{
-    using Cfg = GroupCfg<T, D, BS, NW, NS>;
-    constexpr bool kFp8 = Cfg::kFp8;
-    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+// One warp's share of a group: the G query rows of a (sequence, K/V head) as
+// the A operand, the output accumulator fragments and the online-softmax
+// state, and the math that consumes one staged chunk (the header comment
+// above describes it). T: __half, __nv_bfloat16 or E4M3; TWO: G > 8
+// (fragment rows 8-15 are live).
+template <typename T, int D, bool TWO> struct GroupWarp {
+    using Geo = GroupGeom<T, D>;
+    static constexpr bool kFp8 = Geo::kFp8;
+    static constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     using QT = typename std::conditional<kFp8, __half, T>::type; // operand / row type
-    constexpr int CH = Cfg::kChunk, SEG = Cfg::kSeg, ROW = Cfg::kRow, U = Cfg::kUnits;
-    constexpr int KT = D / 16; // k-steps of q.k = pairs of 8-wide d tiles of O
-    constexpr int MS = Cfg::kMergeStride;
-    constexpr unsigned FULL = 0xffffffffu;
-    const DecodeParams &p = gp.p;
-
-    extern __shared__ __align__(1024) unsigned char group_smem[];
-    unsigned char *smem = group_smem + ((1024u - (smem_addr(group_smem) & 1023u)) & 1023u);
-    char *rings = reinterpret_cast<char *>(smem);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kRingsBytes);
-    float *scales = reinterpret_cast<float *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes);
-    int32_t *rank_ctx =
-        reinterpret_cast<int32_t *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes + Cfg::kScaleBytes);
-    int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
-    __shared__ int cta_flags, ranked_seq;
-
-    pdl_launch_dependents();
-    const int kvh = blockIdx.x, part = blockIdx.z;
-    int s = blockIdx.y;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = p.num_heads, HK = p.num_kv_heads, G = H / HK;
-
-    if (tid == 0)
-        cta_flags = 0;
-    if (lane == 0)
-        for (int k = 0; k < NS; ++k)
-            mbar_init(smem_addr(&bars[warp * NS + k]), 1);
-    fence_mbar_init();
-    pdl_wait_prior_grid(); // every input may come from the previous kernel
-    if (p.rank_seqs) // longest sequences first (ranked_sequence)
-        s = ranked_sequence(p.context_lens, p.num_seqs, blockIdx.y, tid, NW * 32, rank_ctx,
-                            &ranked_seq);
+    static constexpr int CH = Geo::kChunk, ROW = Geo::kRow, U = Geo::kUnits;
+    static constexpr int KT = D / 16; // k-steps of q.k = pairs of 8-wide d tiles of O
+    static constexpr int MS = Geo::kMergeStride;
+    static constexpr unsigned FULL = 0xffffffffu;
 
     // Fragment coordinates: this lane holds rows g0 and g1 = g0 + 8 and, in
     // every 8-wide column tile, columns q2 and q2 + 1 (q = lane % 4).
-    const int g0 = lane >> 2, g1 = g0 + 8, q = lane & 3, q2 = 2 * q;
+    int lane, g0, g1, q, q2;
+    // ldmatrix row addresses (rows within a 16-token step). 16-bit K
+    // (non-transposed, B of S = Q K^T): lanes 0-7 / 8-15 / 16-23 / 24-31
+    // give token rows 0-7 / 0-7 / 8-15 / 8-15 at pieces c / c+1 / c / c+1.
+    // 16-bit V (transposed, B of O = P V): rows 0-7 / 8-15 / 0-7 / 8-15 at
+    // pieces c / c / c+1 / c+1. fp8 K and V (non-transposed): rows 0-7 /
+    // 8-15 / 0-7 / 8-15 at pieces c / c / c+1 / c+1, register = (token tile,
+    // piece).
+    int kt, kc, vt, vc;
+    uint32_t qa[KT][4]; // Q as the A operand, one 16x16 tile per k-step
+    float o[2 * KT][4];
+    float m0, m1, l0, l1;
+    float vref; // fp8: largest V scale so far (R), floored at FLT_MIN
 
-    // Q as the A operand, one 16x16 tile per k-step; rows >= G are zero.
-    // k-slots (2q, 2q+1) / (2q+8, 2q+9) hold d = 16kk + 2q (+1) / + 8 (+1);
-    // fp8: d = 16kk + 4q (+1) / + 2 (+1), matching the widened K codes.
-    // Loaded before the block table so that the two reads overlap.
-    uint32_t qa[KT][4];
+    // Piece p (16 bytes) of row t sits in unit t*U + p/8 at position
+    // (p % 8) ^ ((t*U + p/8) % 8) of a swizzled stage.
+    static __device__ __forceinline__ int piece_off(int t, int piece)
     {
-        const uint32_t *qp = static_cast<const uint32_t *>(p.query); // element pairs
-        const size_t r0 = ((size_t)s * H + (size_t)kvh * G + g0) * (D / 2);
+        const int unit = t * U + (piece >> 3);
+        return unit * 128 + (((piece & 7) ^ (unit & 7)) << 4);
+    }
+
+    // O tile j covers 8 d: 16-bit d = 8j + q2 (+1); fp8 d = 16(j/2) + 4q +
+    // 2(j%2) (+1). Elements 0, 1: row g0; 2, 3: row g1.
+    __device__ __forceinline__ int dcol(int j) const
+    {
+        return kFp8 ? 16 * (j >> 1) + 4 * q + 2 * (j & 1) : 8 * j + q2;
+    }
+
+    __device__ __forceinline__ void init(int lane_)
+    {
+        lane = lane_;
+        g0 = lane >> 2;
+        g1 = g0 + 8;
+        q = lane & 3;
+        q2 = 2 * q;
+        kt = kFp8 ? (lane & 7) + (((lane >> 3) & 1) << 3) : (lane & 7) + ((lane >> 4) << 3);
+        kc = kFp8 ? lane >> 4 : (lane >> 3) & 1;
+        vt = (lane & 7) + (((lane >> 3) & 1) << 3);
+        vc = lane >> 4;
+    }
+
+    // The query rows of heads row0 .. row0 + G - 1 (row0 counts rows of D
+    // elements); rows >= G are zero. k-slots (2q, 2q+1) / (2q+8, 2q+9) hold
+    // d = 16kk + 2q (+1) / + 8 (+1); fp8: d = 16kk + 4q (+1) / + 2 (+1),
+    // matching the widened K codes.
+    __device__ __forceinline__ void load_q(const void *query, size_t row0, int G)
+    {
+        const uint32_t *qp = static_cast<const uint32_t *>(query); // element pairs
+        const size_t r0 = (row0 + g0) * (D / 2);
         const size_t r1 = r0 + (size_t)8 * (D / 2);
 #pragma unroll
         for (int kk = 0; kk < KT; ++kk) {
@@ -203,194 +228,31 @@ __global__ void __launch_bounds__(NW * 32)
         }
     }
 
-    UnitInfo u;
-    const bool live = load_unit<BS>(p, s, part, tid, NW * 32, tid == 0 && kvh == 0 && part == 0,
-                                    table, u);
-    if (!live)
-        return; // uniform across the CTA
-    __syncthreads();
-
-    // O tile j covers 8 d: 16-bit d = 8j + q2 (+1); fp8 d = 16(j/2) +
-    // 4q + 2(j%2) (+1). Elements 0, 1: row g0; 2, 3: row g1.
-    auto dcol = [&](int j) { return kFp8 ? 16 * (j >> 1) + 4 * q + 2 * (j & 1) : 8 * j + q2; };
-    float o[2 * KT][4];
+    __device__ __forceinline__ void reset()
+    {
 #pragma unroll
-    for (int j = 0; j < 2 * KT; ++j)
+        for (int j = 0; j < 2 * KT; ++j)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o[j][e] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float vref = 1.17549435e-38f; // fp8: largest V scale so far (R), floored at FLT_MIN
-
-    const int n_chunks = (u.n_tok + CH - 1) / CH;
-    const int my_chunks = n_chunks <= warp ? 0 : (n_chunks - warp + NW - 1) / NW;
-    char *ring = rings + (size_t)warp * Cfg::kRing;
-    const uint32_t ring_s = smem_addr(ring);
-    const uint32_t bar0 = smem_addr(&bars[warp * NS]);
-    float *wscales = scales + (size_t)warp * NS * 2 * CH; // fp8: [stage][K | V][CH]
-
-    // Fused append: the warp owning the chunk of the sequence's last token
-    // puts the new K/V row into that chunk once it has landed, and into the
-    // cache. Lanes [0, RV) carry 16 bytes of the stored K row each, the next
-    // RV lanes the V row (fp8: 16 codes quantised from 16 inputs, with the
-    // row scale amax / 448 on every lane of the half).
-    constexpr int RV = ROW / 16;
-    int patch_i = -1, patch_row = 0;
-    uint4 patch_val = make_uint4(0u, 0u, 0u, 0u);
-    float patch_scale = 0.f;
-    uint4 *patch_dst = nullptr;
-    float *patch_sdst = nullptr;
-    if (p.new_key != nullptr && part == u.num_parts - 1 && u.n_tok > 0) {
-        const int c_last = (u.n_tok - 1) / CH;
-        if (c_last % NW == warp) { // warp-uniform
-            patch_i = c_last / NW;
-            patch_row = (u.n_tok - 1) - c_last * CH;
-            const bool isv = lane >= RV;
-            const int piece = lane % RV;
-            constexpr int EPL = kFp8 ? 16 : 8; // inputs per lane
-            const QT *src = static_cast<const QT *>(isv ? p.new_value : p.new_key) +
-                            ((size_t)s * HK + kvh) * D + (size_t)piece * EPL;
-            if constexpr (kFp8) {
-                // codes = e4m3(x * (448 / amax)), scale = amax / 448.
-                float x[16];
-                float amax = 0.f;
-                if (lane < 2 * RV) {
-                    unpack8_to<QT>(*reinterpret_cast<const uint4 *>(src), x);
-                    unpack8_to<QT>(*reinterpret_cast<const uint4 *>(src + 8), x + 8);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        amax = fmaxf(amax, fabsf(x[e]));
-                }
-#pragma unroll
-                for (int o2 = 1; o2 < RV; o2 <<= 1)
-                    amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o2));
-                if (lane < 2 * RV) {
-                    const float inv = amax > 0.f ? 448.f / amax : 0.f;
-                    patch_val = quantize16_e4m3(x, inv);
-                    patch_scale = amax / 448.f;
-                }
-            } else {
-                if (lane < 2 * RV)
-                    patch_val = *reinterpret_cast<const uint4 *>(src);
-            }
-            if (lane < 2 * RV) {
-                const int b = table[(u.n_tok - 1) / BS];
-                if (b >= 0 && b < p.num_blocks) {
-                    char *cache = const_cast<char *>(
-                        static_cast<const char *>(isv ? p.value_cache : p.key_cache));
-                    const size_t tile = (size_t)b * HK + kvh;
-                    const int off = (u.n_tok - 1) % BS;
-                    if constexpr (kFp8) {
-                        char *t0 = cache + tile * (size_t)(BS * (D + 4));
-                        patch_dst = reinterpret_cast<uint4 *>(t0 + (size_t)off * D) + piece;
-                        if (piece == 0)
-                            patch_sdst = reinterpret_cast<float *>(t0 + BS * D) + off;
-                    } else {
-                        patch_dst = reinterpret_cast<uint4 *>(
-                                        cache + (tile * BS + off) * (size_t)(D * 2)) +
-                                    piece;
-                    }
-                }
-            }
-        }
+            for (int e = 0; e < 4; ++e)
+                o[j][e] = 0.f;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+        vref = 1.17549435e-38f;
     }
 
-    // Lane 0: the copies of local chunk i (global chunk warp + i*NW). Boxes
-    // that start past the context are not fetched; a block id outside the
-    // pool is replaced by block 0 and recorded.
-    int bad_id = 0;
-    const char *kpool = static_cast<const char *>(p.key_cache);
-    const char *vpool = static_cast<const char *>(p.value_cache);
-    auto issue = [&](int i) {
-        const int tok0 = (warp + i * NW) * CH;
-        const int rows = min(CH, u.n_tok - tok0);
-        const int nseg = (rows + SEG - 1) / SEG;
-        const int st = i % NS;
-        const uint32_t dk = ring_s + st * Cfg::kStage, dv = dk + Cfg::kHalf;
-        const uint32_t bar = bar0 + st * 8;
-        mbar_arrive_expect_tx(bar, (uint32_t)(nseg * SEG * (ROW + (kFp8 ? 4 : 0)) * 2));
-        for (int sg = 0; sg < nseg; ++sg) {
-            const int tok = tok0 + sg * SEG;
-            int b = table[tok / BS];
-            if (b < 0 || b >= p.num_blocks) {
-                bad_id = 1;
-                b = 0;
-            }
-            const int tile = b * HK + kvh;
-            if constexpr (kFp8) {
-                const int off = tok % BS;
-                tma_load_3d(dk + sg * SEG * ROW, &gp.tk, 0, off, tile, bar);
-                tma_load_3d(dv + sg * SEG * ROW, &gp.tv, 0, off, tile, bar);
-                const size_t sofs = (size_t)tile * (BS * (D + 4)) + BS * D + (size_t)off * 4;
-                float *sk = wscales + (st * 2) * CH + sg * SEG;
-                bulk_g2s(smem_addr(sk), kpool + sofs, SEG * 4, bar);
-                bulk_g2s(smem_addr(sk + CH), vpool + sofs, SEG * 4, bar);
-            } else {
-                const int y = tile * BS + tok % BS;
-                tma_load_3d(dk + sg * SEG * ROW, &gp.tk, 0, 0, y, bar);
-                tma_load_3d(dv + sg * SEG * ROW, &gp.tv, 0, 0, y, bar);
-            }
-        }
-    };
-
-    if (lane == 0)
-        for (int i = 0; i < min(NS, my_chunks); ++i)
-            issue(i);
-    int issued = min(NS, my_chunks);
-
-    // ldmatrix row addresses (rows within a 16-token step). 16-bit K
-    // (non-transposed, B of S = Q K^T): lanes 0-7 / 8-15 / 16-23 / 24-31
-    // give token rows 0-7 / 0-7 / 8-15 / 8-15 at pieces c / c+1 / c / c+1.
-    // 16-bit V (transposed, B of O = P V): rows 0-7 / 8-15 / 0-7 / 8-15 at
-    // pieces c / c / c+1 / c+1. fp8 K and V (non-transposed): rows 0-7 /
-    // 8-15 / 0-7 / 8-15 at pieces c / c / c+1 / c+1, register = (token tile,
-    // piece). Piece p (16 bytes) of row t sits in unit t*U + p/8 at position
-    // (p % 8) ^ ((t*U + p/8) % 8).
-    const int kt = kFp8 ? (lane & 7) + (((lane >> 3) & 1) << 3) : (lane & 7) + ((lane >> 4) << 3);
-    const int kc = kFp8 ? lane >> 4 : (lane >> 3) & 1;
-    const int vt = (lane & 7) + (((lane >> 3) & 1) << 3), vc = lane >> 4;
-    auto piece_off = [](int t, int piece) {
-        const int unit = t * U + (piece >> 3);
-        return unit * 128 + (((piece & 7) ^ (unit & 7)) << 4);
-    };
-    const float qs = p.qk_scale_log2;
-
-    int i = 0;
-    for (; i < my_chunks; ++i) {
-        const int st = i % NS;
-        const bool ok = mbar_wait_bounded(bar0 + st * 8, (i / NS) & 1, kWaitLimitNs);
-        if (__any_sync(FULL, !ok))
-            break;
-        const int rows = min(CH, u.n_tok - (warp + i * NW) * CH);
-        char *sk = ring + st * Cfg::kStage;
-        char *sv = sk + Cfg::kHalf;
-        const float *ksc = wscales + (st * 2) * CH; // fp8 scales of the stage
-        const float *vsc = ksc + CH;
-        if (i == patch_i) { // warp-uniform
-            if (lane < 2 * RV) {
-                const bool isv = lane >= RV;
-                char *dst = (isv ? sv : sk) + piece_off(patch_row, lane % RV);
-                *reinterpret_cast<uint4 *>(dst) = patch_val;
-                if (patch_dst)
-                    *patch_dst = patch_val;
-                if constexpr (kFp8) {
-                    if (lane % RV == 0) {
-                        const_cast<float *>(isv ? vsc : ksc)[patch_row] = patch_scale;
-                        if (patch_sdst)
-                            *patch_sdst = patch_scale;
-                    }
-                }
-                fence_proxy_async_smem(); // before the stage is refilled by a copy
-            }
-            __syncwarp();
-        }
-        if (rows < CH) { // the partition's last chunk: zero the V rows past it
+    // One staged chunk: K codes at sk, V at sv (swizzled), fp8 row scales at
+    // ksc / vsc, `rows` valid tokens (1 .. CH; only a unit's last chunk can
+    // be partial), qs = scale * log2(e).
+    __device__ __forceinline__ void chunk(char *sk, char *sv, const float *ksc, const float *vsc,
+                                          int rows, float qs)
+    {
+        if (rows < CH) { // zero the V rows past the context
             for (int k = rows * (ROW / 16) + lane; k < CH * (ROW / 16); k += 32)
                 reinterpret_cast<uint4 *>(sv)[k] = make_uint4(0u, 0u, 0u, 0u);
-            fence_proxy_async_smem();
+            fence_proxy_async_smem(); // before the stage is refilled by a copy
             __syncwarp();
         }
-
+        const uint32_t kb = smem_addr(sk), vb = smem_addr(sv);
 #pragma unroll
         for (int sub = 0; sub < CH / 16; ++sub) {
             const int srows = rows - 16 * sub; // valid tokens of this step
@@ -400,7 +262,6 @@ __global__ void __launch_bounds__(NW * 32)
 
             // S = Q K^T for the step's 16 tokens, even and odd k-steps in
             // separate accumulators (two shorter dependency chains per tile).
-            const uint32_t kb = smem_addr(sk), vb = smem_addr(sv);
             float sc[2][4], sd[2][4];
 #pragma unroll
             for (int j = 0; j < 2; ++j)
@@ -441,8 +302,7 @@ __global__ void __launch_bounds__(NW * 32)
 
             // Online softmax (base 2). sc[j][e]: token t0 + 8j + q2 + (e & 1),
             // row g0 for e < 2, g1 otherwise.
-            // Only a partition's last step can be partial (warp-uniform).
-            const bool partial = srows < 16;
+            const bool partial = srows < 16; // warp-uniform
             float x[2][4];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -594,6 +454,269 @@ __global__ void __launch_bounds__(NW * 32)
                 }
             }
         }
+    }
+
+    // Row sums over each quad, then this warp's (O, m, l) of rows < G into
+    // mw (row stride MS; fp8: O back in the scale of the codes' values,
+    // times R).
+    __device__ __forceinline__ void store(float *mw, int G)
+    {
+        l0 += __shfl_xor_sync(FULL, l0, 1);
+        l0 += __shfl_xor_sync(FULL, l0, 2);
+        l1 += __shfl_xor_sync(FULL, l1, 1);
+        l1 += __shfl_xor_sync(FULL, l1, 2);
+        const float oscale = kFp8 ? vref : 1.f;
+        __syncwarp();
+        if (g0 < G) {
+#pragma unroll
+            for (int j = 0; j < 2 * KT; ++j)
+                *reinterpret_cast<float2 *>(mw + g0 * MS + dcol(j)) =
+                    make_float2(o[j][0] * oscale, o[j][1] * oscale);
+            if ((lane & 3) == 0) {
+                mw[g0 * MS + D] = m0;
+                mw[g0 * MS + D + 1] = l0;
+            }
+        }
+        if constexpr (TWO) {
+            if (g1 < G) {
+#pragma unroll
+                for (int j = 0; j < 2 * KT; ++j)
+                    *reinterpret_cast<float2 *>(mw + g1 * MS + dcol(j)) =
+                        make_float2(o[j][2] * oscale, o[j][3] * oscale);
+                if ((lane & 3) == 0) {
+                    mw[g1 * MS + D] = m1;
+                    mw[g1 * MS + D + 1] = l1;
+                }
+            }
+        }
+    }
+};
+
+// The new token's K and V rows for the fused append (pa_write_kv_decode),
+// one (sequence, K/V head) row per warp: lanes [0, RV) hold 16 bytes of the
+// stored K row each, the next RV lanes the V row (fp8: 16 codes quantised
+// from 16 inputs, with the row scale amax / 448 on every lane of the half).
+template <typename T, int D, int BS> struct NewRow {
+    using Geo = GroupGeom<T, D>;
+    using QT = typename std::conditional<Geo::kFp8, __half, T>::type;
+    static constexpr int RV = Geo::kRow / 16;
+    static constexpr size_t kTile =
+        Geo::kFp8 ? (size_t)BS * (D + 4) : (size_t)BS * D * 2; // one (block, head) tile
+    uint4 val;
+    float scale;
+
+    // Every lane calls it; src_row = s * num_kv_heads + kvh.
+    __device__ __forceinline__ void load(const DecodeParams &p, size_t src_row, int lane)
+    {
+        const bool isv = lane >= RV;
+        const int piece = lane % RV;
+        constexpr int EPL = Geo::kFp8 ? 16 : 8; // inputs per lane
+        const QT *src = static_cast<const QT *>(isv ? p.new_value : p.new_key) + src_row * D +
+                        (size_t)piece * EPL;
+        val = make_uint4(0u, 0u, 0u, 0u);
+        scale = 0.f;
+        if constexpr (Geo::kFp8) {
+            // codes = e4m3(x * (448 / amax)), scale = amax / 448.
+            float x[16];
+            float amax = 0.f;
+            if (lane < 2 * RV) {
+                unpack8_to<QT>(*reinterpret_cast<const uint4 *>(src), x);
+                unpack8_to<QT>(*reinterpret_cast<const uint4 *>(src + 8), x + 8);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    amax = fmaxf(amax, fabsf(x[e]));
+            }
+#pragma unroll
+            for (int o2 = 1; o2 < RV; o2 <<= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o2));
+            if (lane < 2 * RV) {
+                const float inv = amax > 0.f ? 448.f / amax : 0.f;
+                val = quantize16_e4m3(x, inv);
+                scale = amax / 448.f;
+            }
+        } else {
+            if (lane < 2 * RV)
+                val = *reinterpret_cast<const uint4 *>(src);
+        }
+    }
+
+    // Where this lane's 16 bytes (and, on the first lane of each half, the
+    // fp8 row scale) go in the cache: block b, K/V head kvh, slot offset off.
+    // NULL for lanes without a part and for a block id outside the pool.
+    __device__ __forceinline__ void locate(const DecodeParams &p, int b, int kvh, int off,
+                                           int lane, uint4 *&d, float *&sd) const
+    {
+        d = nullptr;
+        sd = nullptr;
+        if (lane >= 2 * RV || b < 0 || b >= p.num_blocks)
+            return;
+        const bool isv = lane >= RV;
+        const int piece = lane % RV;
+        char *cache =
+            const_cast<char *>(static_cast<const char *>(isv ? p.value_cache : p.key_cache));
+        char *tile = cache + ((size_t)b * p.num_kv_heads + kvh) * kTile;
+        d = reinterpret_cast<uint4 *>(tile + (size_t)off * Geo::kRow) + piece;
+        if (Geo::kFp8 && piece == 0)
+            sd = reinterpret_cast<float *>(tile + (size_t)BS * Geo::kRow) + off;
+    }
+};
+
+// decode_group_kernel: one CTA per (K/V head, sequence, partition) of a
+// fixed partition size; grid (num_kv_heads, num_seqs, num_parts).
+template <typename T, int D, int BS, int NW, int NS, bool TWO>
+__global__ void __launch_bounds__(NW * 32)
+    decode_group_kernel(const __grid_constant__ GroupParams gp)
+{
+    using Cfg = GroupCfg<T, D, BS, NW, NS>;
+    using Wp = GroupWarp<T, D, TWO>;
+    constexpr bool kFp8 = Cfg::kFp8;
+    constexpr int CH = Cfg::kChunk, SEG = Cfg::kSeg, ROW = Cfg::kRow;
+    constexpr int MS = Cfg::kMergeStride;
+    constexpr unsigned FULL = 0xffffffffu;
+    const DecodeParams &p = gp.p;
+
+    extern __shared__ __align__(1024) unsigned char group_smem[];
+    unsigned char *smem = group_smem + ((1024u - (smem_addr(group_smem) & 1023u)) & 1023u);
+    char *rings = reinterpret_cast<char *>(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kRingsBytes);
+    float *scales = reinterpret_cast<float *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes);
+    int32_t *rank_ctx =
+        reinterpret_cast<int32_t *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes + Cfg::kScaleBytes);
+    int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
+    __shared__ int cta_flags, ranked_seq;
+
+    pdl_launch_dependents();
+    const int kvh = blockIdx.x, part = blockIdx.z;
+    int s = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.num_heads, HK = p.num_kv_heads, G = H / HK;
+
+    if (tid == 0)
+        cta_flags = 0;
+    if (lane == 0)
+        for (int k = 0; k < NS; ++k)
+            mbar_init(smem_addr(&bars[warp * NS + k]), 1);
+    fence_mbar_init();
+    pdl_wait_prior_grid(); // every input may come from the previous kernel
+    if (p.rank_seqs) // longest sequences first (ranked_sequence)
+        s = ranked_sequence(p.context_lens, p.num_seqs, blockIdx.y, tid, NW * 32, rank_ctx,
+                            &ranked_seq);
+
+    Wp w;
+    w.init(lane);
+    // Loaded before the block table so that the two reads overlap.
+    w.load_q(p.query, (size_t)s * H + (size_t)kvh * G, G);
+
+    UnitInfo u;
+    const bool live = load_unit<BS>(p, s, part, tid, NW * 32, tid == 0 && kvh == 0 && part == 0,
+                                    table, u);
+    if (!live)
+        return; // uniform across the CTA
+    __syncthreads();
+    w.reset();
+
+    const int n_chunks = (u.n_tok + CH - 1) / CH;
+    const int my_chunks = n_chunks <= warp ? 0 : (n_chunks - warp + NW - 1) / NW;
+    char *ring = rings + (size_t)warp * Cfg::kRing;
+    const uint32_t ring_s = smem_addr(ring);
+    const uint32_t bar0 = smem_addr(&bars[warp * NS]);
+    float *wscales = scales + (size_t)warp * NS * 2 * CH; // fp8: [stage][K | V][CH]
+
+    // Fused append: the warp owning the chunk of the sequence's last token
+    // puts the new K/V row into that chunk once it has landed, and into the
+    // cache.
+    constexpr int RV = ROW / 16;
+    int patch_i = -1, patch_row = 0;
+    NewRow<T, D, BS> nr;
+    nr.val = make_uint4(0u, 0u, 0u, 0u);
+    nr.scale = 0.f;
+    uint4 *patch_dst = nullptr;
+    float *patch_sdst = nullptr;
+    if (p.new_key != nullptr && part == u.num_parts - 1 && u.n_tok > 0) {
+        const int c_last = (u.n_tok - 1) / CH;
+        if (c_last % NW == warp) { // warp-uniform
+            patch_i = c_last / NW;
+            patch_row = (u.n_tok - 1) - c_last * CH;
+            nr.load(p, (size_t)s * HK + kvh, lane);
+            nr.locate(p, table[(u.n_tok - 1) / BS], kvh, (u.n_tok - 1) % BS, lane, patch_dst,
+                      patch_sdst);
+        }
+    }
+
+    // Lane 0: the copies of local chunk i (global chunk warp + i*NW). Boxes
+    // that start past the context are not fetched; a block id outside the
+    // pool is replaced by block 0 and recorded.
+    int bad_id = 0;
+    const char *kpool = static_cast<const char *>(p.key_cache);
+    const char *vpool = static_cast<const char *>(p.value_cache);
+    auto issue = [&](int i) {
+        const int tok0 = (warp + i * NW) * CH;
+        const int rows = min(CH, u.n_tok - tok0);
+        const int nseg = (rows + SEG - 1) / SEG;
+        const int st = i % NS;
+        const uint32_t dk = ring_s + st * Cfg::kStage, dv = dk + Cfg::kHalf;
+        const uint32_t bar = bar0 + st * 8;
+        mbar_arrive_expect_tx(bar, (uint32_t)(nseg * SEG * (ROW + (kFp8 ? 4 : 0)) * 2));
+        for (int sg = 0; sg < nseg; ++sg) {
+            const int tok = tok0 + sg * SEG;
+            int b = table[tok / BS];
+            if (b < 0 || b >= p.num_blocks) {
+                bad_id = 1;
+                b = 0;
+            }
+            const int tile = b * HK + kvh;
+            if constexpr (kFp8) {
+                const int off = tok % BS;
+                tma_load_3d(dk + sg * SEG * ROW, &gp.tk, 0, off, tile, bar);
+                tma_load_3d(dv + sg * SEG * ROW, &gp.tv, 0, off, tile, bar);
+                const size_t sofs = (size_t)tile * (BS * (D + 4)) + BS * D + (size_t)off * 4;
+                float *sk = wscales + (st * 2) * CH + sg * SEG;
+                bulk_g2s(smem_addr(sk), kpool + sofs, SEG * 4, bar);
+                bulk_g2s(smem_addr(sk + CH), vpool + sofs, SEG * 4, bar);
+            } else {
+                const int y = tile * BS + tok % BS;
+                tma_load_3d(dk + sg * SEG * ROW, &gp.tk, 0, 0, y, bar);
+                tma_load_3d(dv + sg * SEG * ROW, &gp.tv, 0, 0, y, bar);
+            }
+        }
+    };
+
+    if (lane == 0)
+        for (int i = 0; i < min(NS, my_chunks); ++i)
+            issue(i);
+    int issued = min(NS, my_chunks);
+    const float qs = p.qk_scale_log2;
+
+    int i = 0;
+    for (; i < my_chunks; ++i) {
+        const int st = i % NS;
+        const bool ok = mbar_wait_bounded(bar0 + st * 8, (i / NS) & 1, kWaitLimitNs);
+        if (__any_sync(FULL, !ok))
+            break;
+        const int rows = min(CH, u.n_tok - (warp + i * NW) * CH);
+        char *sk = ring + st * Cfg::kStage;
+        char *sv = sk + Cfg::kHalf;
+        float *ksc = wscales + (st * 2) * CH; // fp8 scales of the stage
+        float *vsc = ksc + CH;
+        if (i == patch_i) { // warp-uniform
+            if (lane < 2 * RV) {
+                const bool isv = lane >= RV;
+                char *dst = (isv ? sv : sk) + Wp::piece_off(patch_row, lane % RV);
+                *reinterpret_cast<uint4 *>(dst) = nr.val;
+                if (patch_dst)
+                    *patch_dst = nr.val;
+                if constexpr (kFp8) {
+                    if (lane % RV == 0) {
+                        (isv ? vsc : ksc)[patch_row] = nr.scale;
+                        if (patch_sdst)
+                            *patch_sdst = nr.scale;
+                    }
+                }
+                fence_proxy_async_smem(); // before the stage is refilled by a copy
+            }
+            __syncwarp();
+        }
+        w.chunk(sk, sv, ksc, vsc, rows, qs);
         __syncwarp();
         if (i + NS < my_chunks) {
             if (lane == 0)
@@ -616,37 +739,9 @@ __global__ void __launch_bounds__(NW * 32)
             atomicOr(&cta_flags, 1);
     }
 
-    // Row sums over the quad; then this warp's (O, m, l) into its ring (fp8:
-    // O back in the scale of the codes' values, times R).
-    l0 += __shfl_xor_sync(FULL, l0, 1);
-    l0 += __shfl_xor_sync(FULL, l0, 2);
-    l1 += __shfl_xor_sync(FULL, l1, 1);
-    l1 += __shfl_xor_sync(FULL, l1, 2);
-    const float oscale = kFp8 ? vref : 1.f;
+    // This warp's (O, m, l) into its ring, then the warps merged.
     __syncwarp();
-    float *mw = reinterpret_cast<float *>(ring);
-    if (g0 < G) {
-#pragma unroll
-        for (int j = 0; j < 2 * KT; ++j)
-            *reinterpret_cast<float2 *>(mw + g0 * MS + dcol(j)) =
-                make_float2(o[j][0] * oscale, o[j][1] * oscale);
-        if ((lane & 3) == 0) {
-            mw[g0 * MS + D] = m0;
-            mw[g0 * MS + D + 1] = l0;
-        }
-    }
-    if constexpr (TWO) {
-        if (g1 < G) {
-#pragma unroll
-            for (int j = 0; j < 2 * KT; ++j)
-                *reinterpret_cast<float2 *>(mw + g1 * MS + dcol(j)) =
-                    make_float2(o[j][2] * oscale, o[j][3] * oscale);
-            if ((lane & 3) == 0) {
-                mw[g1 * MS + D] = m1;
-                mw[g1 * MS + D + 1] = l1;
-            }
-        }
-    }
+    w.store(reinterpret_cast<float *>(ring), G);
     __syncthreads();
 
     const bool failed = cta_flags != 0;
@@ -656,13 +751,14 @@ __global__ void __launch_bounds__(NW * 32)
         const int g = idx / D, d = idx - g * D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NW; ++w)
-            M = fmaxf(M, reinterpret_cast<const float *>(rings + w * Cfg::kRing)[g * MS + D]);
+        for (int w2 = 0; w2 < NW; ++w2)
+            M = fmaxf(M, reinterpret_cast<const float *>(rings + w2 * Cfg::kRing)[g * MS + D]);
         float L = 0.f, O = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float *mv = reinterpret_cast<const float *>(rings + w * Cfg::kRing) + g * MS;
+            for (int w2 = 0; w2 < NW; ++w2) {
+                const float *mv =
+                    reinterpret_cast<const float *>(rings + w2 * Cfg::kRing) + g * MS;
                 const float f = exp2f(mv[D] - M);
                 L = fmaf(mv[D + 1], f, L);
                 O = fmaf(mv[d], f, O);
@@ -685,6 +781,455 @@ __global__ void __launch_bounds__(NW * 32)
     if (u.num_parts > 1 && p.ws_count)
         merge_if_last<D>(p, s, kvh * G, G, s * HK + kvh, u.num_parts, tid, NW * 32, &cta_flags,
                          reinterpret_cast<float *>(rings));
+}
+
+// ---------------------------------------------------------------------------
+// decode_flat_kernel: balanced token ranges for grouped heads.
+//
+// The work of a launch is the list of units (sequence s, K/V head kvh), in
+// that order, each cut into chunks of CH tokens (n_s = ceil(ctx_s / CH) per
+// unit): C = num_kv_heads * sum_s n_s chunks in all. With R = min(N, C)
+// (N CTAs in the launch), CTA c < R takes the chunks [c*C/R, (c+1)*C/R) of
+// that list, whatever units they belong to, so every CTA streams the same
+// number of chunks (within one) however the context lengths are spread (a
+// fixed partition size leaves some SMs idle while a few long units finish). Every CTA derives the whole schedule from the context
+// lengths (a prefix sum in shared memory): the host needs no knowledge of
+// them and no extra launch is made.
+//
+// Inside a CTA the range falls into segments, one per unit it touches. The
+// NW warps share each segment as in decode_group_kernel (chunk j of the
+// segment to warp j % NW) and keep their bulk-copy rings going across
+// segment boundaries: a warp's copies of the next segment's chunks are in
+// flight while the CTA merges the current one. At the end of a segment every
+// warp leaves its (O, m, l) in a merge area, the CTA merges them, and writes
+// the output rows when the segment is the whole unit; else it writes its
+// piece (unnormalised O, m, l) to the workspace and counts in on the unit's
+// counter, and the last of the unit's CTAs merges the pieces, in CTA order.
+// A segment in the middle of a range is always a whole unit, so a CTA has at
+// most two pieces, in workspace slots (c, 0) (the unit that contains the
+// range's first chunk) and (c, 1).
+//
+// Fused append: before streaming, each CTA writes the new token's K/V rows
+// of every unit whose last chunk lies in its range (only that CTA reads
+// that chunk) straight into the cache, then fences the generic-proxy
+// writes against the copies that will read them.
+// ---------------------------------------------------------------------------
+constexpr int kFlatMaxSeqs = 512; // sequences per launch (context-length prefix in shared memory)
+constexpr int kFlatTable = 1024;  // block-table entries a CTA stages (its whole range)
+constexpr int kFlatMaxSegs = 32;  // segments per window (more: the range is walked in windows)
+
+// Chunks one CTA range may hold so that its block-table entries fit the
+// staged table: CH / BS entries per chunk when a chunk covers whole blocks;
+// else (a chunk is half a block) at most one per chunk, counting the
+// rounding at both ends of every segment.
+constexpr int flat_max_chunks_for(bool fp8, int block_size)
+{
+    return kFlatTable / ((fp8 ? 32 : 16) >= block_size ? (fp8 ? 32 : 16) / block_size : 2);
+}
+
+struct FlatSeg {
+    int s, kvh; // the unit
+    int a, b;   // its chunks [a, b) in this range
+    int n;      // chunks of the whole unit
+    int ctx;    // its context length (clamped)
+    int blk0;   // first block-table index of the sequence the segment reads
+    int tab;    // where those entries start in the staged table
+};
+
+template <typename T, int D, int BS, int NW, int NS, bool TWO> struct FlatCfg : GroupGeom<T, D> {
+    using Geo = GroupGeom<T, D>;
+    static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
+    static constexpr int kRows = TWO ? 16 : 8; // query rows a warp can hold
+    static constexpr int kRing = NS * Geo::kStage;
+    static constexpr int kSeg = BS < 16 ? BS : 16; // rows per TMA box
+    static constexpr int kRingsBytes = NW * kRing;
+    static constexpr int kMergeBytes = NW * kRows * Geo::kMergeStride * 4;
+    static constexpr int kBarBytes = NW * NS * 8;
+    static constexpr int kScaleBytes = Geo::kFp8 ? NW * NS * 2 * Geo::kChunk * 4 : 0;
+    static constexpr int kSegBytes = kFlatMaxSegs * (int)(sizeof(FlatSeg) + 4);
+    static constexpr int kSeqBytes = ((2 * kFlatMaxSeqs + 1) * 4 + 15) / 16 * 16;
+    static constexpr int kTableBytes = kFlatTable * 4;
+    static constexpr int kBytes = 1024 + kRingsBytes + kMergeBytes + kBarBytes + kScaleBytes +
+                                  kSegBytes + kSeqBytes + kTableBytes;
+    static constexpr int kMaxChunks = flat_max_chunks_for(Geo::kFp8, BS); // per CTA range
+    static_assert((kSeg * Geo::kRow) % 1024 == 0, "swizzle atoms");
+    static_assert(Geo::kChunk % kSeg == 0 && Geo::kChunk % 16 == 0, "chunk geometry");
+    static_assert(NW * 32 * 4 >= kFlatMaxSeqs, "four sequences per thread in the prefix sum");
+};
+
+// Bidirectional proxy fence for global memory: this thread's generic-proxy
+// writes before later async-proxy (bulk copy) reads of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+template <typename T, int D, int BS, int NW, int NS, bool TWO>
+__global__ void __launch_bounds__(NW * 32, 2)
+    decode_flat_kernel(const __grid_constant__ GroupParams gp)
+{
+    using Cfg = FlatCfg<T, D, BS, NW, NS, TWO>;
+    using Wp = GroupWarp<T, D, TWO>;
+    constexpr bool kFp8 = Cfg::kFp8;
+    constexpr int CH = Cfg::kChunk, SEG = Cfg::kSeg, ROW = Cfg::kRow, MS = Cfg::kMergeStride;
+    constexpr int NT = NW * 32, ROWS = Cfg::kRows;
+    constexpr int PER = (kFlatMaxSeqs + NT - 1) / NT;
+    constexpr unsigned FULL = 0xffffffffu;
+    const DecodeParams &p = gp.p;
+
+    extern __shared__ __align__(1024) unsigned char flat_smem[];
+    unsigned char *smem = flat_smem + ((1024u - (smem_addr(flat_smem) & 1023u)) & 1023u);
+    char *rings = reinterpret_cast<char *>(smem);
+    float *merge = reinterpret_cast<float *>(smem + Cfg::kRingsBytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kRingsBytes + Cfg::kMergeBytes);
+    float *scales = reinterpret_cast<float *>(reinterpret_cast<char *>(bars) + Cfg::kBarBytes);
+    FlatSeg *segs = reinterpret_cast<FlatSeg *>(reinterpret_cast<char *>(scales) + Cfg::kScaleBytes);
+    int *seg_bad = reinterpret_cast<int *>(segs + kFlatMaxSegs);
+    int *sQ = reinterpret_cast<int *>(reinterpret_cast<char *>(segs) + Cfg::kSegBytes);
+    int *sctx = sQ + kFlatMaxSeqs + 1;
+    int32_t *table = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(sQ) + Cfg::kSeqBytes);
+    __shared__ int s_flags; // 1: a block id outside the pool; 2: a wait ran out
+    __shared__ int s_nseg, s_ntab, s_last;
+    __shared__ long long s_wend;
+    __shared__ int s_warp_sum[NW];
+
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, N = gp.num_ctas;
+    const int S = p.num_seqs, H = p.num_heads, HK = p.num_kv_heads, G = H / HK;
+
+    if (tid == 0)
+        s_flags = 0;
+    if (lane == 0)
+        for (int k = 0; k < NS; ++k)
+            mbar_init(smem_addr(&bars[warp * NS + k]), 1);
+    fence_mbar_init();
+    pdl_wait_prior_grid(); // every input may come from the previous kernel
+
+    // Chunks per sequence and their exclusive prefix sum sQ (sQ[S] = total);
+    // thread t handles sequences PER*t .. PER*t + PER - 1.
+    {
+        int cnt[PER];
+        int tot = 0;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int s = tid * PER + k;
+            int n = 0;
+            if (s < S) {
+                const int ctx = checked_context(p, p.context_lens[s], BS, c == 0);
+                sctx[s] = ctx;
+                n = (ctx + CH - 1) / CH;
+            }
+            cnt[k] = n;
+            tot += n;
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(FULL, incl, o);
+            if (lane >= o)
+                incl += v;
+        }
+        if (lane == 31)
+            s_warp_sum[warp] = incl;
+        __syncthreads();
+        int run = incl - tot;
+        for (int w2 = 0; w2 < warp; ++w2)
+            run += s_warp_sum[w2];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int s = tid * PER + k;
+            if (s < S)
+                sQ[s] = run;
+            run += cnt[k];
+        }
+        if (tid == NT - 1)
+            sQ[S] = run;
+        __syncthreads();
+    }
+
+    // This CTA's chunks [R0, R1) of C. The ranges are cut over the first
+    // NR = min(N, C) CTAs, so none of them is empty (a unit's pieces then
+    // come from consecutive CTAs); CTAs past NR have nothing to stream.
+    // cta_of(x): the CTA holding chunk x.
+    const long long C = (long long)HK * sQ[S];
+    const long long NR = min((long long)N, C);
+    const long long R0 = c < NR ? C * c / NR : C, R1 = c < NR ? C * (c + 1) / NR : C;
+    auto cta_of = [&](long long x) { return (int)(((x + 1) * NR - 1) / C); };
+    auto range_start = [&](int cc) { return C * cc / NR; };
+
+    // Sequences without context get zero rows, from the CTA whose range
+    // holds their place in the list (the last CTA when that is the end).
+    for (int s = tid; s < S; s += NT) {
+        if (sQ[s + 1] != sQ[s])
+            continue;
+        const long long at = (long long)HK * sQ[s];
+        if ((at < C ? cta_of(at) : N - 1) != c)
+            continue;
+        for (int e = 0; e < H * D; ++e)
+            store_out(p.out, p.out_dtype, (size_t)s * H * D + e, 0.f);
+    }
+
+    Wp w;
+    w.init(lane);
+    w.reset();
+    const char *kpool = static_cast<const char *>(p.key_cache);
+    const char *vpool = static_cast<const char *>(p.value_cache);
+    char *ring = rings + (size_t)warp * Cfg::kRing;
+    const uint32_t ring_s = smem_addr(ring);
+    const uint32_t bar0 = smem_addr(&bars[warp * NS]);
+    float *wscales = scales + (size_t)warp * NS * 2 * CH; // fp8: [stage][K | V][CH]
+    const float qs = p.qk_scale_log2;
+    int issued = 0, consumed = 0; // this warp's copies, over all windows
+    bool failed = false;          // warp-uniform: a wait ran out
+
+    long long pos = R0;
+    while (pos < R1) { // CTA-uniform
+        // The next window of segments, from chunk pos (thread 0).
+        if (tid == 0) {
+            int lo = 0, hi = S - 1; // the last sequence with HK * sQ[s] <= pos
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if ((long long)HK * sQ[mid] <= pos)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            int s = lo;
+            int kvh = (int)((pos - (long long)HK * sQ[s]) / (sQ[s + 1] - sQ[s]));
+            int k = 0, tab = 0;
+            while (pos < R1 && k < kFlatMaxSegs) {
+                const int n = sQ[s + 1] - sQ[s];
+                const long long pu = (long long)HK * sQ[s] + (long long)kvh * n;
+                FlatSeg sg;
+                sg.s = s;
+                sg.kvh = kvh;
+                sg.a = (int)(pos - pu);
+                sg.b = (int)min((long long)n, R1 - pu);
+                sg.n = n;
+                sg.ctx = sctx[s];
+                sg.blk0 = sg.a * CH / BS;
+                sg.tab = tab;
+                const int entries = (min(sg.b * CH, sg.ctx) + BS - 1) / BS - sg.blk0;
+                if (k > 0 && tab + entries > kFlatTable)
+                    break; // the rest in the next window (the host sizes ranges to fit)
+                tab += entries;
+                segs[k] = sg;
+                seg_bad[k] = 0;
+                ++k;
+                pos = pu + sg.b;
+                if (pos < R1 && ++kvh == HK) {
+                    kvh = 0;
+                    do
+                        ++s;
+                    while (sQ[s + 1] == sQ[s]);
+                }
+            }
+            s_nseg = k;
+            s_ntab = tab;
+            s_wend = pos;
+        }
+        __syncthreads();
+        const int nseg = s_nseg, ntab = min(s_ntab, kFlatTable);
+        pos = s_wend;
+
+        // The window's block-table entries, and the first segment's query rows.
+        for (int e = tid; e < ntab; e += NT) {
+            int k = 0;
+            while (k + 1 < nseg && segs[k + 1].tab <= e)
+                ++k;
+            table[e] = p.block_tables[(size_t)segs[k].s * p.max_blocks_per_seq + segs[k].blk0 +
+                                      (e - segs[k].tab)];
+        }
+        w.load_q(p.query, (size_t)segs[0].s * H + (size_t)segs[0].kvh * G, G);
+        __syncthreads();
+
+        // Fused append: the new rows of the units that end in this window go
+        // to the cache before any copy of their last chunk is issued.
+        if (p.new_key != nullptr) {
+            for (int k = warp; k < nseg; k += NW) {
+                const FlatSeg sg = segs[k];
+                if (sg.b != sg.n) // warp-uniform
+                    continue;
+                NewRow<T, D, BS> nr;
+                nr.load(p, (size_t)sg.s * HK + sg.kvh, lane);
+                uint4 *dst;
+                float *sdst;
+                const int t = sg.ctx - 1;
+                const int te = sg.tab + t / BS - sg.blk0;
+                nr.locate(p, te < kFlatTable ? table[te] : -1, sg.kvh, t % BS, lane, dst, sdst);
+                if (dst)
+                    *dst = nr.val;
+                if (sdst)
+                    *sdst = nr.scale;
+            }
+            fence_proxy_async_global();
+        }
+        __syncthreads();
+
+        // This warp's chunks in window order: chunk a + warp + j*NW of each
+        // segment. Issue cursor (ik, ic), warp-uniform; lane 0 copies.
+        int ik = 0, ic = segs[0].a + warp;
+        auto advance = [&]() {
+            while (ik < nseg && ic >= segs[ik].b)
+                if (++ik < nseg)
+                    ic = segs[ik].a + warp;
+        };
+        advance();
+        auto issue = [&]() {
+            if (lane == 0) {
+                const FlatSeg &sg = segs[ik];
+                const int tok0 = ic * CH;
+                const int rows = min(CH, sg.ctx - tok0);
+                const int nbox = (rows + SEG - 1) / SEG;
+                const int st = issued % NS;
+                const uint32_t dk = ring_s + st * Cfg::kStage, dv = dk + Cfg::kHalf;
+                const uint32_t bar = bar0 + st * 8;
+                mbar_arrive_expect_tx(bar, (uint32_t)(nbox * SEG * (ROW + (kFp8 ? 4 : 0)) * 2));
+                for (int bx = 0; bx < nbox; ++bx) {
+                    const int tok = tok0 + bx * SEG;
+                    const int te = sg.tab + tok / BS - sg.blk0;
+                    int b = te < kFlatTable ? table[te] : -1;
+                    if (b < 0 || b >= p.num_blocks) {
+                        seg_bad[ik] = 1;
+                        b = 0;
+                    }
+                    const int tile = b * HK + sg.kvh;
+                    if constexpr (kFp8) {
+                        const int off = tok % BS;
+                        tma_load_3d(dk + bx * SEG * ROW, &gp.tk, 0, off, tile, bar);
+                        tma_load_3d(dv + bx * SEG * ROW, &gp.tv, 0, off, tile, bar);
+                        const size_t sofs =
+                            (size_t)tile * (BS * (D + 4)) + BS * D + (size_t)off * 4;
+                        float *sk = wscales + (st * 2) * CH + bx * SEG;
+                        bulk_g2s(smem_addr(sk), kpool + sofs, SEG * 4, bar);
+                        bulk_g2s(smem_addr(sk + CH), vpool + sofs, SEG * 4, bar);
+                    } else {
+                        const int y = tile * BS + tok % BS;
+                        tma_load_3d(dk + bx * SEG * ROW, &gp.tk, 0, 0, y, bar);
+                        tma_load_3d(dv + bx * SEG * ROW, &gp.tv, 0, 0, y, bar);
+                    }
+                }
+            }
+            ++issued;
+            ic += NW;
+            advance();
+        };
+        while (!failed && ik < nseg && issued - consumed < NS)
+            issue();
+
+        for (int k = 0; k < nseg; ++k) { // CTA-uniform
+            const FlatSeg sg = segs[k];
+            for (int cc = sg.a + warp; cc < sg.b; cc += NW) {
+                if (failed)
+                    continue;
+                const int st = consumed % NS;
+                const bool ok = mbar_wait_bounded(bar0 + st * 8, (consumed / NS) & 1, kWaitLimitNs);
+                if (__any_sync(FULL, !ok)) {
+                    failed = true;
+                    continue;
+                }
+                char *sk = ring + st * Cfg::kStage;
+                float *ksc = wscales + (st * 2) * CH;
+                w.chunk(sk, sk + Cfg::kHalf, ksc, ksc + CH, min(CH, sg.ctx - cc * CH), qs);
+                __syncwarp();
+                ++consumed;
+                if (ik < nseg)
+                    issue();
+            }
+
+            // End of the segment: this warp's state to the merge area, the
+            // next segment's query rows on their way, a fresh state.
+            float *mw = merge + (size_t)warp * ROWS * MS;
+            w.store(mw, G);
+            if (k + 1 < nseg)
+                w.load_q(p.query, (size_t)segs[k + 1].s * H + (size_t)segs[k + 1].kvh * G, G);
+            w.reset();
+            if (failed && lane == 0)
+                atomicOr(&s_flags, 2);
+            if (seg_bad[k] && tid == 0)
+                atomicOr(&s_flags, 1);
+            __syncthreads();
+
+            // Merge the warps: the unit's rows, or this CTA's piece of it.
+            const bool whole = sg.a == 0 && sg.b == sg.n;
+            const bool bad = seg_bad[k] != 0 || (s_flags & 2) != 0;
+            const long long pu = (long long)HK * sQ[sg.s] + (long long)sg.kvh * sg.n;
+            const size_t slot = 2 * (size_t)c + (pu <= R0 ? 0 : 1);
+            for (int idx = tid; idx < G * D; idx += NT) {
+                const int g = idx / D, d = idx - g * D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w2 = 0; w2 < NW; ++w2)
+                    M = fmaxf(M, merge[((size_t)w2 * ROWS + g) * MS + D]);
+                float L = 0.f, O = 0.f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int w2 = 0; w2 < NW; ++w2) {
+                        const float *mv = merge + ((size_t)w2 * ROWS + g) * MS;
+                        if (mv[D] == -INFINITY) // a warp without chunks here
+                            continue;
+                        const float f = exp2f(mv[D] - M);
+                        L = fmaf(mv[D + 1], f, L);
+                        O = fmaf(mv[d], f, O);
+                    }
+                }
+                if (bad)
+                    O = NAN;
+                if (whole) {
+                    store_out(p.out, p.out_dtype, ((size_t)sg.s * H + sg.kvh * G + g) * D + d,
+                              L > 0.f ? O / L : O);
+                } else {
+                    p.ws_acc[(slot * G + g) * D + d] = O;
+                    if (d == 0) {
+                        p.ws_ml[(slot * G + g) * 2] = bad ? 0.f : M;
+                        p.ws_ml[(slot * G + g) * 2 + 1] = bad ? 1.f : L;
+                    }
+                }
+            }
+            __syncthreads();
+            if (whole)
+                continue;
+
+            // Count this piece in; the unit's last CTA merges its pieces in
+            // CTA order and resets the counter.
+            const int c0 = cta_of(pu), c1 = cta_of(pu + sg.n - 1);
+            if (tid == 0)
+                s_last = arrive_acq_rel(&p.ws_count[sg.s * HK + sg.kvh]) == c1 - c0;
+            __syncthreads();
+            if (!s_last)
+                continue;
+            for (int idx = tid; idx < G * D; idx += NT) {
+                const int g = idx / D, d = idx - g * D;
+                float M = -INFINITY;
+                for (int cc = c0; cc <= c1; ++cc) {
+                    const size_t sl = 2 * (size_t)cc + (pu <= range_start(cc) ? 0 : 1);
+                    M = fmaxf(M, __ldcg(&p.ws_ml[(sl * G + g) * 2]));
+                }
+                float L = 0.f, O = 0.f;
+                for (int cc = c0; cc <= c1; ++cc) {
+                    const size_t sl = 2 * (size_t)cc + (pu <= range_start(cc) ? 0 : 1);
+                    const float f = exp2f(__ldcg(&p.ws_ml[(sl * G + g) * 2]) - M);
+                    L = fmaf(__ldcg(&p.ws_ml[(sl * G + g) * 2 + 1]), f, L);
+                    O = fmaf(__ldcg(&p.ws_acc[(sl * G + g) * D + d]), f, O);
+                }
+                store_out(p.out, p.out_dtype, ((size_t)sg.s * H + sg.kvh * G + g) * D + d, O / L);
+            }
+            if (tid == 0)
+                p.ws_count[sg.s * HK + sg.kvh] = 0;
+        }
+    }
+
+    if (failed) // the copies still in flight land before the CTA exits
+        for (int k = consumed; k < issued; ++k)
+            mbar_wait_bounded(bar0 + (k % NS) * 8, (k / NS) & 1, kWaitLimitNs);
+    __syncthreads();
+    if (tid == 0) {
+        if (s_flags & 2)
+            report(p.dev_err, PA_DEVERR_TIMEOUT);
+        if (s_flags & 1)
+            report(p.dev_err, PA_DEVERR_BLOCK_ID);
+    }
 }
 
 } // namespace pagedkv
