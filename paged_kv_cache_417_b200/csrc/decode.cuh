@@ -795,11 +795,10 @@ struct UnitInfo {
 };
 
 template <int BS>
-__device__ __forceinline__ bool load_unit(const DecodeParams &p, int s, int part, int tid,
+__device__ __forceinline__ bool load_unit(const DecodeParams &p, int s, int part, int P, int tid,
                                           int nthreads, bool report_ctx, int32_t *table,
                                           UnitInfo &u)
 {
-    const int P = p.partition_size;
     const int raw = p.context_lens[s];
     const int start_blk = part * (P / BS);
     const int n_load = min(P / BS, p.max_blocks_per_seq - start_blk);
@@ -868,8 +867,8 @@ __global__ void __launch_bounds__(NW * 32)
         s = ranked_sequence(p.context_lens, p.num_seqs, blockIdx.y, tid, NW * 32, rank_ctx,
                             &ranked_seq);
     UnitInfo u;
-    const bool live = load_unit<BS>(p, s, part, tid, NW * 32, tid == 0 && h == 0 && part == 0,
-                                    table, u);
+    const bool live = load_unit<BS>(p, s, part, p.partition_size, tid, NW * 32,
+                                    tid == 0 && h == 0 && part == 0, table, u);
     if (!live)
         return; // uniform across the CTA
     __syncthreads();

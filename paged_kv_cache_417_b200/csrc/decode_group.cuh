@@ -83,7 +83,16 @@ struct GroupParams {
     CUtensorMap tv; // value pool, same geometry
     DecodeParams p;
     int32_t num_ctas; // decode_flat_kernel: CTAs of the launch (balanced ranges)
+    // decode_group_kernel: 1 = balanced partitions (a 1-D grid of pieces,
+    // the partition size chosen in the kernel; p.partition_size is its
+    // floor and p.num_parts the workspace stride), 0 = the (K/V head,
+    // sequence, partition) grid of a fixed partition size.
+    int32_t balanced;
 };
+
+// Balanced partitions: at most this many sequences (their context lengths
+// and piece counts are staged in shared memory).
+constexpr int kBalMaxSeqs = 512;
 
 // Stage geometry of the grouped kernels (independent of the block size).
 template <typename T, int D> struct GroupGeom {
@@ -109,7 +118,10 @@ template <typename T, int D, int BS, int NW, int NS> struct GroupCfg : GroupGeom
     // fp8 row scales: per warp, [stage][K | V][kChunk] floats.
     static constexpr int kScaleBytes = Geo::kFp8 ? NW * NS * 2 * Geo::kChunk * 4 : 0;
     static constexpr int kRankBytes = kRankMaxSeqs * 4; // context lengths for ranking
-    static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kScaleBytes + kRankBytes;
+    // Balanced partitions: context lengths, then the pieces' prefix sum.
+    static constexpr int kBalBytes = ((2 * kBalMaxSeqs + 1) * 4 + 15) / 16 * 16;
+    static constexpr int kFixedBytes =
+        kRingsBytes + kBarBytes + kScaleBytes + kRankBytes + kBalBytes;
     // After its last chunk a warp of decode_group_kernel leaves (O, m, l) of
     // its rows in its ring.
     static_assert(kGroupMaxHeads * Geo::kMergeStride * 4 <= kRing, "merge area fits a ring");
@@ -561,8 +573,147 @@ template <typename T, int D, int BS> struct NewRow {
     }
 };
 
+// Sum over the CTA (every thread calls it; two barriers).
+template <int NW> __device__ __forceinline__ long long cta_sum(long long v, long long *red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads(); // red may still be read by an earlier call
+    if (lane == 0)
+        red[warp] = v;
+    __syncthreads();
+    long long t = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+        t += red[w];
+    return t;
+}
+
+// Maximum over the CTA (every thread calls it; two barriers).
+template <int NW> __device__ __forceinline__ long long cta_max(long long v, long long *red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    __syncthreads();
+    if (lane == 0)
+        red[warp] = v;
+    __syncthreads();
+    long long t = red[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w)
+        t = max(t, red[w]);
+    return t;
+}
+
+// Balanced partitions. Every CTA derives the same partition size P (tokens)
+// from the context lengths: the smallest multiple of 32 at or above the
+// floor p.partition_size (and at most the longest context, at most
+// kMaxPartition) found by the test below that cuts the launch into at most
+// gridDim.x pieces, num_kv_heads * sum_s max(1, ceil(ctx_s / P)) (a sequence
+// without context still gets a piece, which writes its zero rows). It then
+// returns the piece of this CTA: (sequence s, K/V head kvh, partition part);
+// false when the CTA has none. Every thread calls it (barriers inside);
+// ctxs: kBalMaxSeqs ints, pre: kBalMaxSeqs + 1 ints of shared memory.
+template <int BS, int NW>
+__device__ __forceinline__ bool balanced_piece(const DecodeParams &p, int32_t *ctxs, int32_t *pre,
+                                               long long *red, int &s, int &kvh, int &part,
+                                               int &P)
+{
+    constexpr int NT = NW * 32, PER = (kBalMaxSeqs + NT - 1) / NT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int S = p.num_seqs, HK = p.num_kv_heads;
+    long long tot = 0;
+    int mx = 0;
+    for (int q = tid; q < S; q += NT) {
+        const int ctx = checked_context(p, p.context_lens[q], BS, blockIdx.x == 0 && tid == 0);
+        ctxs[q] = ctx;
+        tot += ctx;
+        mx = max(mx, ctx);
+    }
+    tot = cta_sum<NW>(tot, red);
+    mx = (int)cta_max<NW>(mx, red);
+    const int floor_p = p.partition_size;
+    const int p_max = max(floor_p, min(kMaxPartition, (max(mx, 1) + 31) / 32 * 32));
+    const long long budget = gridDim.x / HK; // pieces per K/V head
+    auto round_p = [&](long long t) {
+        const long long r = (t + 31) / 32 * 32;
+        return (int)max((long long)floor_p, min((long long)p_max, r));
+    };
+    auto count = [&](int cand) { // sum_s max(1, ceil(ctx_s / cand)), over the CTA
+        long long c = 0;
+        for (int q = tid; q < S; q += NT)
+            c += max(1, (ctxs[q] + cand - 1) / cand);
+        return cta_sum<NW>(c, red);
+    };
+    // sum_s max(1, ceil(ctx_s / P)) <= tot / P + S: P >= tot / (budget - S)
+    // always fits; first try the estimate with half a piece of rounding per
+    // sequence.
+    P = p_max;
+    if (budget > S) {
+        P = round_p((tot + (budget - S / 2) - 1) / (budget - S / 2));
+        if (count(P) > budget)
+            P = round_p((tot + (budget - S) - 1) / (budget - S));
+    }
+    // Pieces per sequence and their exclusive prefix sum, PER sequences per
+    // thread.
+    int cnt[PER];
+    int mine = 0;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int q = tid * PER + k;
+        cnt[k] = q < S ? max(1, (ctxs[q] + P - 1) / P) : 0;
+        mine += cnt[k];
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += v;
+    }
+    __syncthreads(); // red reuse
+    if (lane == 31)
+        red[warp] = incl;
+    __syncthreads();
+    int run = incl - mine;
+    for (int w = 0; w < warp; ++w)
+        run += (int)red[w];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int q = tid * PER + k;
+        if (q < S)
+            pre[q] = run;
+        run += cnt[k];
+    }
+    if (tid == NT - 1)
+        pre[S] = run;
+    __syncthreads();
+    const long long b = blockIdx.x;
+    if (b >= (long long)HK * pre[S])
+        return false;
+    int lo = 0, hi = S - 1; // the last sequence with HK * pre[q] <= b
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((long long)HK * pre[mid] <= b)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    s = lo;
+    const int n = pre[s + 1] - pre[s];
+    const int r = (int)(b - (long long)HK * pre[s]);
+    kvh = r / n;
+    part = r - kvh * n;
+    return true;
+}
+
 // decode_group_kernel: one CTA per (K/V head, sequence, partition) of a
-// fixed partition size; grid (num_kv_heads, num_seqs, num_parts).
+// fixed partition size, grid (num_kv_heads, num_seqs, num_parts); or, with
+// balanced partitions, one CTA per piece of a 1-D grid.
 template <typename T, int D, int BS, int NW, int NS, bool TWO>
 __global__ void __launch_bounds__(NW * 32)
     decode_group_kernel(const __grid_constant__ GroupParams gp)
@@ -582,12 +733,14 @@ __global__ void __launch_bounds__(NW * 32)
     float *scales = reinterpret_cast<float *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes);
     int32_t *rank_ctx =
         reinterpret_cast<int32_t *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes + Cfg::kScaleBytes);
+    int32_t *bal_ctx = rank_ctx + kRankMaxSeqs;
+    int32_t *bal_pre = bal_ctx + kBalMaxSeqs;
     int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
     __shared__ int cta_flags, ranked_seq;
+    __shared__ long long bal_red[NW];
 
     pdl_launch_dependents();
-    const int kvh = blockIdx.x, part = blockIdx.z;
-    int s = blockIdx.y;
+    int kvh = blockIdx.x, part = blockIdx.z, s = blockIdx.y, P = p.partition_size;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads, HK = p.num_kv_heads, G = H / HK;
 
@@ -598,9 +751,13 @@ __global__ void __launch_bounds__(NW * 32)
             mbar_init(smem_addr(&bars[warp * NS + k]), 1);
     fence_mbar_init();
     pdl_wait_prior_grid(); // every input may come from the previous kernel
-    if (p.rank_seqs) // longest sequences first (ranked_sequence)
+    if (gp.balanced) {
+        if (!balanced_piece<BS, NW>(p, bal_ctx, bal_pre, bal_red, s, kvh, part, P))
+            return; // uniform: this CTA has no piece
+    } else if (p.rank_seqs) { // longest sequences first (ranked_sequence)
         s = ranked_sequence(p.context_lens, p.num_seqs, blockIdx.y, tid, NW * 32, rank_ctx,
                             &ranked_seq);
+    }
 
     Wp w;
     w.init(lane);
@@ -608,8 +765,8 @@ __global__ void __launch_bounds__(NW * 32)
     w.load_q(p.query, (size_t)s * H + (size_t)kvh * G, G);
 
     UnitInfo u;
-    const bool live = load_unit<BS>(p, s, part, tid, NW * 32, tid == 0 && kvh == 0 && part == 0,
-                                    table, u);
+    const bool live = load_unit<BS>(p, s, part, P, tid, NW * 32,
+                                    tid == 0 && kvh == 0 && part == 0, table, u);
     if (!live)
         return; // uniform across the CTA
     __syncthreads();
@@ -864,8 +1021,14 @@ __device__ __forceinline__ void fence_proxy_async_global()
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Resident CTAs per SM the flat launch is built for (registers are capped
+// to allow them). The macro exists for tuning sweeps.
+#ifndef PA_FLAT_CTAS_PER_SM
+#define PA_FLAT_CTAS_PER_SM 2
+#endif
+
 template <typename T, int D, int BS, int NW, int NS, bool TWO>
-__global__ void __launch_bounds__(NW * 32, 2)
+__global__ void __launch_bounds__(NW * 32, PA_FLAT_CTAS_PER_SM)
     decode_flat_kernel(const __grid_constant__ GroupParams gp)
 {
     using Cfg = FlatCfg<T, D, BS, NW, NS, TWO>;
@@ -889,7 +1052,9 @@ __global__ void __launch_bounds__(NW * 32, 2)
     int *sctx = sQ + kFlatMaxSeqs + 1;
     int32_t *table = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(sQ) + Cfg::kSeqBytes);
     __shared__ int s_flags; // 1: a block id outside the pool; 2: a wait ran out
-    __shared__ int s_nseg, s_ntab, s_last;
+    __shared__ int s_nseg, s_ntab, s_last, s_slot0, s_pieces;
+    __shared__ float s_fac[NW][kGroupMaxHeads]; // per warp and row: 2^(m_w - M)
+    __shared__ float2 s_rowml[kGroupMaxHeads];  // per row: (M, L)
     __shared__ long long s_wend;
     __shared__ int s_warp_sum[NW];
 
@@ -1151,39 +1316,46 @@ __global__ void __launch_bounds__(NW * 32, 2)
                 atomicOr(&s_flags, 1);
             __syncthreads();
 
-            // Merge the warps: the unit's rows, or this CTA's piece of it.
+            // Merge the warps: per row, each warp's factor 2^(m_w - M) (0 for
+            // a warp without chunks here) and the row's (M, L); then every
+            // output element sums its warps in warp order.
             const bool whole = sg.a == 0 && sg.b == sg.n;
             const bool bad = seg_bad[k] != 0 || (s_flags & 2) != 0;
             const long long pu = (long long)HK * sQ[sg.s] + (long long)sg.kvh * sg.n;
             const size_t slot = 2 * (size_t)c + (pu <= R0 ? 0 : 1);
-            for (int idx = tid; idx < G * D; idx += NT) {
-                const int g = idx / D, d = idx - g * D;
+            if (tid < G) {
                 float M = -INFINITY;
 #pragma unroll
                 for (int w2 = 0; w2 < NW; ++w2)
-                    M = fmaxf(M, merge[((size_t)w2 * ROWS + g) * MS + D]);
-                float L = 0.f, O = 0.f;
-                if (M != -INFINITY) {
+                    M = fmaxf(M, merge[((size_t)w2 * ROWS + tid) * MS + D]);
+                float L = 0.f;
 #pragma unroll
-                    for (int w2 = 0; w2 < NW; ++w2) {
-                        const float *mv = merge + ((size_t)w2 * ROWS + g) * MS;
-                        if (mv[D] == -INFINITY) // a warp without chunks here
-                            continue;
-                        const float f = exp2f(mv[D] - M);
-                        L = fmaf(mv[D + 1], f, L);
-                        O = fmaf(mv[d], f, O);
-                    }
+                for (int w2 = 0; w2 < NW; ++w2) {
+                    const float *mv = merge + ((size_t)w2 * ROWS + tid) * MS;
+                    const float f = mv[D] == -INFINITY ? 0.f : exp2f(mv[D] - M);
+                    L = fmaf(mv[D + 1], f, L);
+                    s_fac[w2][tid] = f;
                 }
+                s_rowml[tid] = make_float2(M, L);
+            }
+            __syncthreads();
+            for (int idx = tid; idx < G * D; idx += NT) {
+                const int g = idx / D, d = idx - g * D;
+                float O = 0.f;
+#pragma unroll
+                for (int w2 = 0; w2 < NW; ++w2)
+                    O = fmaf(merge[((size_t)w2 * ROWS + g) * MS + d], s_fac[w2][g], O);
+                const float2 ml = s_rowml[g];
                 if (bad)
                     O = NAN;
                 if (whole) {
                     store_out(p.out, p.out_dtype, ((size_t)sg.s * H + sg.kvh * G + g) * D + d,
-                              L > 0.f ? O / L : O);
+                              ml.y > 0.f ? O / ml.y : O);
                 } else {
                     p.ws_acc[(slot * G + g) * D + d] = O;
                     if (d == 0) {
-                        p.ws_ml[(slot * G + g) * 2] = bad ? 0.f : M;
-                        p.ws_ml[(slot * G + g) * 2 + 1] = bad ? 1.f : L;
+                        p.ws_ml[(slot * G + g) * 2] = bad ? 0.f : ml.x;
+                        p.ws_ml[(slot * G + g) * 2 + 1] = bad ? 1.f : ml.y;
                     }
                 }
             }
@@ -1192,31 +1364,105 @@ __global__ void __launch_bounds__(NW * 32, 2)
                 continue;
 
             // Count this piece in; the unit's last CTA merges its pieces in
-            // CTA order and resets the counter.
-            const int c0 = cta_of(pu), c1 = cta_of(pu + sg.n - 1);
-            if (tid == 0)
+            // CTA order and resets the counter. Piece i comes from CTA
+            // c0 + i; only the first can sit in slot 1 (when the unit starts
+            // inside that CTA's range), the others start their ranges.
+            if (tid == 0) {
+                const int c0 = cta_of(pu), c1 = cta_of(pu + sg.n - 1);
                 s_last = arrive_acq_rel(&p.ws_count[sg.s * HK + sg.kvh]) == c1 - c0;
+                s_slot0 = 2 * c0 + (pu == range_start(c0) ? 0 : 1);
+                s_pieces = c1 - c0 + 1;
+            }
             __syncthreads();
             if (!s_last)
                 continue;
-            for (int idx = tid; idx < G * D; idx += NT) {
-                const int g = idx / D, d = idx - g * D;
-                float M = -INFINITY;
-                for (int cc = c0; cc <= c1; ++cc) {
-                    const size_t sl = 2 * (size_t)cc + (pu <= range_start(cc) ? 0 : 1);
-                    M = fmaxf(M, __ldcg(&p.ws_ml[(sl * G + g) * 2]));
+            const int np = s_pieces;
+            const size_t slot0 = (size_t)s_slot0;
+            auto piece_slot = [&](int i) { return i == 0 ? slot0 : (slot0 & ~(size_t)1) + 2 * i; };
+            if (np <= 32 && np * G <= Cfg::kMergeBytes / 4) {
+                // Each row's normalised weights 2^(m_i - M) / L in the merge
+                // area: one warp per row, lane i holding piece i, every
+                // row's (m, l) loaded before any reduction.
+                float *wts = merge;
+                constexpr int RPW = (kGroupMaxHeads + NW - 1) / NW; // rows per warp
+                float2 ml[RPW];
+#pragma unroll
+                for (int j = 0; j < RPW; ++j) {
+                    const int g = warp + j * NW;
+                    ml[j] = make_float2(-INFINITY, 0.f);
+                    if (g < G && lane < np)
+                        ml[j] = __ldcg(reinterpret_cast<const float2 *>(p.ws_ml) +
+                                       piece_slot(lane) * G + g);
                 }
-                float L = 0.f, O = 0.f;
-                for (int cc = c0; cc <= c1; ++cc) {
-                    const size_t sl = 2 * (size_t)cc + (pu <= range_start(cc) ? 0 : 1);
-                    const float f = exp2f(__ldcg(&p.ws_ml[(sl * G + g) * 2]) - M);
-                    L = fmaf(__ldcg(&p.ws_ml[(sl * G + g) * 2 + 1]), f, L);
-                    O = fmaf(__ldcg(&p.ws_acc[(sl * G + g) * D + d]), f, O);
+#pragma unroll
+                for (int j = 0; j < RPW; ++j) {
+                    const int g = warp + j * NW;
+                    if (g >= G) // warp-uniform
+                        continue;
+                    float M = ml[j].x;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+                        M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
+                    const float f = lane < np ? exp2f(ml[j].x - M) : 0.f;
+                    float L = f * ml[j].y;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+                        L += __shfl_xor_sync(FULL, L, o);
+                    if (lane < np)
+                        wts[g * np + lane] = f / L;
                 }
-                store_out(p.out, p.out_dtype, ((size_t)sg.s * H + sg.kvh * G + g) * D + d, O / L);
+                __syncthreads();
+                // Every output element of this thread over the pieces, the
+                // loads of one piece issued together.
+                constexpr int KO = kGroupMaxHeads * D / NT; // outputs per thread, at most
+                float O[KO];
+#pragma unroll
+                for (int k2 = 0; k2 < KO; ++k2)
+                    O[k2] = 0.f;
+                for (int i = 0; i < np; ++i) {
+                    const float *acc = p.ws_acc + piece_slot(i) * G * D;
+                    float v[KO];
+#pragma unroll
+                    for (int k2 = 0; k2 < KO; ++k2) {
+                        const int idx = tid + k2 * NT;
+                        v[k2] = idx < G * D ? __ldcg(acc + idx) : 0.f;
+                    }
+#pragma unroll
+                    for (int k2 = 0; k2 < KO; ++k2) {
+                        const int idx = tid + k2 * NT;
+                        if (idx < G * D)
+                            O[k2] = fmaf(v[k2], wts[(idx / D) * np + i], O[k2]);
+                    }
+                }
+#pragma unroll
+                for (int k2 = 0; k2 < KO; ++k2) {
+                    const int idx = tid + k2 * NT;
+                    if (idx < G * D) {
+                        const int g = idx / D, d = idx - g * D;
+                        store_out(p.out, p.out_dtype,
+                                  ((size_t)sg.s * H + sg.kvh * G + g) * D + d, O[k2]);
+                    }
+                }
+            } else { // many pieces: per element
+                for (int idx = tid; idx < G * D; idx += NT) {
+                    const int g = idx / D, d = idx - g * D;
+                    float M = -INFINITY;
+                    for (int i = 0; i < np; ++i)
+                        M = fmaxf(M, __ldcg(&p.ws_ml[(piece_slot(i) * G + g) * 2]));
+                    float L = 0.f, O = 0.f;
+                    for (int i = 0; i < np; ++i) {
+                        const size_t sl = piece_slot(i);
+                        const float f = exp2f(__ldcg(&p.ws_ml[(sl * G + g) * 2]) - M);
+                        L = fmaf(__ldcg(&p.ws_ml[(sl * G + g) * 2 + 1]), f, L);
+                        O = fmaf(__ldcg(&p.ws_acc[(sl * G + g) * D + d]), f, O);
+                    }
+                    store_out(p.out, p.out_dtype, ((size_t)sg.s * H + sg.kvh * G + g) * D + d,
+                              O / L);
+                }
             }
             if (tid == 0)
                 p.ws_count[sg.s * HK + sg.kvh] = 0;
+            __syncthreads(); // the merge area holds the next segment's states next
         }
     }
 

@@ -222,9 +222,15 @@ size_t workspace_bytes_for(int64_t units, int64_t num_parts, int head_dim)
 // back to decode_group_kernel. Its workspace: the arrival counters (one per
 // (sequence, K/V head)), then two piece slots per CTA of G rows of (O [D],
 // then (m, l)).
-constexpr int kFlatWarps = 4;
-constexpr int kFlatStages = 2;
-constexpr int kFlatCtasPerSm = 2;
+#ifndef PA_FLAT_WARPS
+#define PA_FLAT_WARPS 4
+#endif
+#ifndef PA_FLAT_STAGES
+#define PA_FLAT_STAGES 2
+#endif
+constexpr int kFlatWarps = PA_FLAT_WARPS;
+constexpr int kFlatStages = PA_FLAT_STAGES;
+constexpr int kFlatCtasPerSm = PA_FLAT_CTAS_PER_SM;
 constexpr int kFlatCtaCap = 8;
 
 // Chunks one flat CTA range may hold for a cache (FlatCfg::kMaxChunks); the
@@ -260,6 +266,26 @@ int64_t flat_ctas(int64_t chunk_bound, int max_chunks, int resident_per_sm, int 
                                             sm_count,
                                         (chunk_bound + max_chunks - 1) / max_chunks);
     return n > (int64_t)kFlatCtaCap * sm_count ? 0 : n;
+}
+
+// Which launch grouped query heads with automatic partitioning take (when
+// the workspace allows; else fixed partitions): 0 decode_flat_kernel, 1
+// balanced partitions of decode_group_kernel, 2 fixed partitions. The macro
+// exists for comparisons.
+#ifndef PA_GROUP_LAUNCH
+#define PA_GROUP_LAUNCH 1
+#endif
+
+// Balanced partitions: the floor of the partition size, so that the merging
+// CTA can hold one weight per (head, partition) (G * parts <= kMergeWeights)
+// and no CTA streams less than 256 tokens; 0 when no floor fits.
+int balanced_floor(int32_t num_heads, const pa_cache_desc *c, int32_t max_ctx)
+{
+    const int G = num_heads / c->num_kv_heads;
+    const int64_t per = kMergeWeights / G; // partitions the merge can weigh
+    const int64_t need = (max_ctx + per - 1) / per;
+    const int64_t f = std::max<int64_t>(256, (need + 31) / 32 * 32);
+    return f <= kMaxPartition ? (int)f : 0;
 }
 
 size_t flat_workspace_bytes(int64_t ctas, int group, int head_dim)
@@ -411,16 +437,61 @@ pa_status encode_pool_rows(CUtensorMap *map, const void *pool, const pa_cache_de
     return PA_OK;
 }
 
+// Resident decode_group_kernel CTAs per SM (balanced partitions size their
+// grid by it), looked up once per device and instantiation.
+template <typename Kernel>
+int resident_ctas(Kernel k, int threads, size_t smem, std::atomic<int> (&cache)[kMaxDevices])
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 0;
+    }
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0)
+        return n;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// Balanced partitions: CTAs per launch, in waves of the resident CTAs. The
+// macro exists for tuning sweeps.
+#ifndef PA_BAL_WAVES
+#define PA_BAL_WAVES 2
+#endif
+
 template <typename T, int D, int BS, bool TWO>
-pa_status launch_group(const GroupParams &gp, cudaStream_t stream)
+pa_status launch_group(const GroupParams &gp_in, cudaStream_t stream)
 {
     using Cfg = GroupCfg<T, D, BS, kGroupWarps, kGroupStages>;
     auto kernel = decode_group_kernel<T, D, BS, kGroupWarps, kGroupStages, TWO>;
     static std::atomic<size_t> smem_set[kMaxDevices];
+    static std::atomic<int> resident[kMaxDevices];
+    GroupParams gp = gp_in;
     const DecodeParams &p = gp.p;
     cudaError_t e = allow_smem(kernel, Cfg::smem_bytes(kMaxPartition), smem_set);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute(group decode)");
+    if (gp.balanced) {
+        // Enough CTAs for PA_BAL_WAVES waves, for one piece per (sequence,
+        // K/V head), and for every piece at the largest partition.
+        const int occ = std::max(1, resident_ctas(kernel, kGroupWarps * 32,
+                                                  Cfg::smem_bytes(kMaxPartition), resident));
+        const int64_t units = (int64_t)p.num_seqs * p.num_kv_heads;
+        const int64_t n = std::max<int64_t>(
+            {(int64_t)PA_BAL_WAVES * occ * sm_count_of_current_device(), units,
+             units * ((p.max_context_len + kMaxPartition - 1) / kMaxPartition)});
+        gp.num_ctas = (int32_t)n;
+        e = launch_pdl(kernel, dim3((unsigned)n), dim3(kGroupWarps * 32),
+                       Cfg::smem_bytes(kMaxPartition), stream, gp);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "group decode launch");
+        return ok();
+    }
     e = launch_pdl(kernel, dim3(p.num_kv_heads, p.num_seqs, p.num_parts),
                    dim3(kGroupWarps * 32), Cfg::smem_bytes(p.partition_size), stream, gp);
     if (e != cudaSuccess)
@@ -453,11 +524,13 @@ pa_status group_bs(const GroupParams &gp, int bs, cudaStream_t st)
     return fail(PA_ERR_UNSUPPORTED, "block_size %d", bs);
 }
 
-pa_status dispatch_group(const DecodeParams &p, const pa_cache_desc *c, cudaStream_t st)
+pa_status dispatch_group(const DecodeParams &p, const pa_cache_desc *c, cudaStream_t st,
+                         bool balanced = false)
 {
     GroupParams gp;
     std::memset(&gp, 0, sizeof(gp));
     gp.p = p;
+    gp.balanced = balanced ? 1 : 0;
     pa_status s = encode_pool_rows(&gp.tk, p.key_cache, c);
     if (s == PA_OK)
         s = encode_pool_rows(&gp.tv, p.value_cache, c);
@@ -710,11 +783,15 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
         num_heads % cache->num_kv_heads != 0 || max_context_len < 0 ||
         check_partition_request(partition_size) != PA_OK)
         return -1;
-    if (flat_eligible(num_seqs, num_heads, cache, max_context_len, partition_size) &&
-        flat_ctas(flat_chunk_bound(num_seqs, cache->num_kv_heads, max_context_len,
-                                   cache->dtype == PA_FP8_E4M3 ? 32 : 16),
-                  flat_max_chunks(cache), kFlatCtasPerSm, sm_count_of_current_device()) > 0)
-        return 0; // token ranges balanced per launch (given a sufficient workspace)
+    if (PA_GROUP_LAUNCH != 2 &&
+        flat_eligible(num_seqs, num_heads, cache, max_context_len, partition_size) &&
+        (PA_GROUP_LAUNCH == 0
+             ? flat_ctas(flat_chunk_bound(num_seqs, cache->num_kv_heads, max_context_len,
+                                          cache->dtype == PA_FP8_E4M3 ? 32 : 16),
+                         flat_max_chunks(cache), kFlatCtasPerSm,
+                         sm_count_of_current_device()) > 0
+             : balanced_floor(num_heads, cache, max_context_len) > 0))
+        return 0; // work balanced per launch (given a sufficient workspace)
     return choose_partition(num_seqs, num_heads, cache, max_context_len, partition_size,
                             partition_size == 0 ? sm_count_of_current_device() : 148);
 }
@@ -859,9 +936,11 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
     p.qk_scale_log2 = scale * 1.4426950408889634f;
     p.new_key = new_key;
     p.new_value = new_value;
-    // Grouped heads with automatic partitioning: balanced token ranges
-    // (decode_flat_kernel) when the workspace holds its pieces.
-    if (flat_eligible(num_seqs, num_heads, cache, max_context_len, partition_size)) {
+    // Grouped heads with automatic partitioning: balanced work when the
+    // workspace holds it (decode_flat_kernel's pieces, or the partials of
+    // balanced partitions).
+    if (PA_GROUP_LAUNCH != 2 &&
+        flat_eligible(num_seqs, num_heads, cache, max_context_len, partition_size)) {
         void *fw = workspace;
         size_t fb = workspace_bytes;
         if (builtin_scratch) {
@@ -869,11 +948,34 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
                 return s;
             fb = PA_NOALLOC_SCRATCH_BYTES;
         }
-        bool launched = false;
-        s = dispatch_flat(p, cache, fw, fb, builtin_scratch, static_cast<cudaStream_t>(stream),
-                          &launched);
-        if (s != PA_OK || launched)
-            return s;
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        if (PA_GROUP_LAUNCH == 0) {
+            bool launched = false;
+            s = dispatch_flat(p, cache, fw, fb, builtin_scratch, st, &launched);
+            if (s != PA_OK || launched)
+                return s;
+        } else if (const int floor_p = balanced_floor(num_heads, cache, max_context_len)) {
+            const int64_t stride = (max_context_len + floor_p - 1) / floor_p;
+            const int64_t units = (int64_t)num_seqs * num_heads;
+            if (fw && aligned16(fw) && fb >= workspace_bytes_for(units, stride, cache->head_dim)) {
+                if (builtin_scratch) {
+                    const cudaError_t e = cudaMemsetAsync(
+                        fw, 0, (size_t)num_seqs * cache->num_kv_heads * sizeof(int32_t), st);
+                    if (e != cudaSuccess)
+                        return cuda_fail(e, "clearing the built-in scratch counters");
+                }
+                DecodeParams q = p;
+                char *w = static_cast<char *>(fw);
+                const size_t acc = (size_t)(units * stride * cache->head_dim) * sizeof(float);
+                q.partition_size = floor_p;
+                q.num_parts = (int32_t)stride;
+                q.rank_seqs = 0;
+                q.ws_count = reinterpret_cast<int32_t *>(w);
+                q.ws_acc = reinterpret_cast<float *>(w + kCounterBytes);
+                q.ws_ml = reinterpret_cast<float *>(w + kCounterBytes + (acc + 255) / 256 * 256);
+                return dispatch_group(q, cache, st, true);
+            }
+        }
     }
     if (parts > 1) {
         const int64_t units = (int64_t)num_seqs * num_heads;
