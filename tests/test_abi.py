@@ -160,11 +160,9 @@ def test_workspace_and_partition_sizes(lib):
         assert lib.decode_partition_size(*args, 0) == 0, args
     # Otherwise one CTA row per K/V head and fixed partitions: an explicit
     # size; past 512 sequences 1024 tokens (halved while the grid has fewer
-    # CTAs than SMs); and when the balanced launch would need more than 8
-    # CTAs per SM (512 sequences x 16 K/V heads x 64k tokens).
+    # CTAs than SMs).
     assert lib.decode_partition_size(96, 32, desc(8), 2048, 512) == 512
     assert lib.decode_partition_size(600, 32, desc(8), 2048, 0) == 1024
-    assert lib.decode_partition_size(512, 32, desc(16), 65536, 0) == 1024
     # fp8 without grouping, with bf16 rows or head_dim 64 stays on one CTA
     # row per query head.
     assert lib.decode_partition_size(96, 32, desc(32, lib.PA_FP8_E4M3), 2048, 0) == 2048
