@@ -471,13 +471,11 @@ class StepLauncher:
                                      partition, dev)
         self.P = pk.decode_partition_size(S, step.num_heads, d["key_caches"][0],
                                           step.max_context_len, partition)
-        # P == 0: grouped heads whose token ranges are balanced per launch
-        # (pieces of a split sequence merged inside the same kernel).
-        self.split = self.P == 0 or step.max_context_len > self.P
+        self.split = step.max_context_len > self.P
         # Split partitions are merged by the last CTA of each sequence, unless
         # the grid has more (sequence, head) slots than the workspace has
         # arrival counters (then a separate reduce kernel runs).
-        self.reduce_launch = self.P > 0 and self.split and S * step.num_heads > 65536
+        self.reduce_launch = self.split and S * step.num_heads > 65536
         self.has_copy = step.copy_pairs.shape[0] > 0
 
     @property
@@ -920,7 +918,7 @@ def main():
             "max_abs_err": acc["max_abs_err"] if acc else None, "accuracy": acc,
             "gpu_launches": launcher.launches_per_step * args.steps, "clocks": clocks,
             "host_paced_value": paced, "host_block_manager": bm_timing, "swap": swap_stats,
-            "partition_size": P if P else "balanced per launch", "split": split,
+            "partition_size": P, "split": split,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -104,10 +104,8 @@ pa_status pa_write_kv(const void *key, const void *value, int32_t num_tokens,
 
 /* Bytes of workspace pa_decode needs. partition_size as for pa_decode; with
  * 0 (automatic) the bound covers every partition size the automatic choice
- * can take and, when num_heads >= 2 and num_seqs <= 512, the balanced
- * launch of grouped query heads for any group size (pa_decode_partition_size
- * returns 0 for it); it depends on the current device's SM count. Returns 0
- * when no workspace is needed and (size_t)-1 on invalid arguments. */
+ * can take. Returns 0 when no workspace is needed and (size_t)-1 on
+ * invalid arguments. */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
                                 int32_t max_context_len, int32_t partition_size);
 
@@ -116,14 +114,8 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t hea
  * merge. The cache descriptor decides the kernel and so the work units: one
  * CTA row per (sequence, query head), or per (sequence, K/V head) when
  * grouped query heads take the grouped kernel (2 <= G <= 16 with a 16-bit
- * cache, or with an fp8 cache of f16 rows and head_dim 128).
- * 0 means no fixed partition: grouped query heads with partition_size 0 and
- * at most 512 sequences run one persistent launch in which every CTA
- * streams an equal share of all (sequence, K/V head) tokens, cutting
- * sequences wherever the shares end and merging the pieces in the same
- * kernel. It needs a workspace of pa_decode_workspace_size(..., 0) bytes;
- * with a smaller one pa_decode falls back to fixed partitions of the
- * automatic size. Returns -1 on invalid arguments. */
+ * cache, or with an fp8 cache of f16 rows and head_dim 128). Returns -1 on
+ * invalid arguments. */
 int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
                                  const pa_cache_desc *cache, int32_t max_context_len,
                                  int32_t partition_size);
@@ -151,9 +143,6 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
  *               unnormalised output, fp32) go to the workspace; the last CTA
  *               of a sequence to finish merges them with the log-sum-exp
  *               rule (when num_seqs * num_heads > 65536, a second kernel).
- *               With grouped query heads, 0 takes the balanced launch
- *               described at pa_decode_partition_size when the workspace
- *               allows it.
  * workspace     device, >= pa_decode_workspace_size(...) bytes when that is
  *               non-zero (may be NULL otherwise). Its first 256 KiB hold
  *               arrival counters that must be zero before the first call

@@ -3,19 +3,14 @@
 // sm_100a: 16-bit caches, and fp8 (e4m3) caches with f16 rows and head_dim
 // 128 (2 <= G <= 16 for both; the kernel itself also handles G = 1).
 //
-// Query heads kvh*G .. kvh*G+G-1 all attend over K/V head kvh. A CTA works
-// on (K/V head, sequence) units for the whole group, so each K/V byte
-// crosses HBM once per group instead of once per query head, and the G query
-// rows share every staged tile. Two kernels share the staging and the math
-// (GroupWarp):
-//   decode_group_kernel  one CTA per (K/V head kvh, sequence s, partition p)
-//                        of a fixed partition size; the outputs, the split
-//                        workspace and the merge of partitions are those of
-//                        decode_split_kernel (per query head; the last CTA
-//                        of a (K/V head, sequence) merges its G heads).
-//   decode_flat_kernel   a persistent launch in which every CTA streams an
-//                        equal share of all the launch's chunks, across
-//                        unit boundaries (described before it below).
+// Query heads kvh*G .. kvh*G+G-1 all attend over K/V head kvh. A CTA takes
+// the unit (K/V head kvh, sequence s, partition p) for the whole group, so
+// each K/V byte crosses HBM once per group instead of once per query head,
+// and the G query rows share every staged tile. The outputs, the split
+// workspace and the merge of partitions are those of decode_split_kernel
+// (per query head; the last CTA of a (K/V head, sequence) merges its G
+// heads). The per-warp state and the math of one staged chunk are GroupWarp;
+// the fused append's new rows, NewRow.
 //
 // Staging: each pool is viewed as a 3-D tensor for the TMA unit. 16-bit
 // pools: (64 elements, D/64 128-byte units, rows), row = one token of one
@@ -82,17 +77,7 @@ struct GroupParams {
     CUtensorMap tk; // key pool (see the staging note above), 128B swizzle
     CUtensorMap tv; // value pool, same geometry
     DecodeParams p;
-    int32_t num_ctas; // decode_flat_kernel: CTAs of the launch (balanced ranges)
-    // decode_group_kernel: 1 = balanced partitions (a 1-D grid of pieces,
-    // the partition size chosen in the kernel; p.partition_size is its
-    // floor and p.num_parts the workspace stride), 0 = the (K/V head,
-    // sequence, partition) grid of a fixed partition size.
-    int32_t balanced;
 };
-
-// Balanced partitions: at most this many sequences (their context lengths
-// and piece counts are staged in shared memory).
-constexpr int kBalMaxSeqs = 512;
 
 // Stage geometry of the grouped kernels (independent of the block size).
 template <typename T, int D> struct GroupGeom {
@@ -118,10 +103,7 @@ template <typename T, int D, int BS, int NW, int NS> struct GroupCfg : GroupGeom
     // fp8 row scales: per warp, [stage][K | V][kChunk] floats.
     static constexpr int kScaleBytes = Geo::kFp8 ? NW * NS * 2 * Geo::kChunk * 4 : 0;
     static constexpr int kRankBytes = kRankMaxSeqs * 4; // context lengths for ranking
-    // Balanced partitions: context lengths, then the pieces' prefix sum.
-    static constexpr int kBalBytes = ((2 * kBalMaxSeqs + 1) * 4 + 15) / 16 * 16;
-    static constexpr int kFixedBytes =
-        kRingsBytes + kBarBytes + kScaleBytes + kRankBytes + kBalBytes;
+    static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kScaleBytes + kRankBytes;
     // After its last chunk a warp of decode_group_kernel leaves (O, m, l) of
     // its rows in its ring.
     static_assert(kGroupMaxHeads * Geo::kMergeStride * 4 <= kRing, "merge area fits a ring");
@@ -573,147 +555,8 @@ template <typename T, int D, int BS> struct NewRow {
     }
 };
 
-// Sum over the CTA (every thread calls it; two barriers).
-template <int NW> __device__ __forceinline__ long long cta_sum(long long v, long long *red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    __syncthreads(); // red may still be read by an earlier call
-    if (lane == 0)
-        red[warp] = v;
-    __syncthreads();
-    long long t = 0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w)
-        t += red[w];
-    return t;
-}
-
-// Maximum over the CTA (every thread calls it; two barriers).
-template <int NW> __device__ __forceinline__ long long cta_max(long long v, long long *red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if (lane == 0)
-        red[warp] = v;
-    __syncthreads();
-    long long t = red[0];
-#pragma unroll
-    for (int w = 1; w < NW; ++w)
-        t = max(t, red[w]);
-    return t;
-}
-
-// Balanced partitions. Every CTA derives the same partition size P (tokens)
-// from the context lengths: the smallest multiple of 32 at or above the
-// floor p.partition_size (and at most the longest context, at most
-// kMaxPartition) found by the test below that cuts the launch into at most
-// gridDim.x pieces, num_kv_heads * sum_s max(1, ceil(ctx_s / P)) (a sequence
-// without context still gets a piece, which writes its zero rows). It then
-// returns the piece of this CTA: (sequence s, K/V head kvh, partition part);
-// false when the CTA has none. Every thread calls it (barriers inside);
-// ctxs: kBalMaxSeqs ints, pre: kBalMaxSeqs + 1 ints of shared memory.
-template <int BS, int NW>
-__device__ __forceinline__ bool balanced_piece(const DecodeParams &p, int32_t *ctxs, int32_t *pre,
-                                               long long *red, int &s, int &kvh, int &part,
-                                               int &P)
-{
-    constexpr int NT = NW * 32, PER = (kBalMaxSeqs + NT - 1) / NT;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int S = p.num_seqs, HK = p.num_kv_heads;
-    long long tot = 0;
-    int mx = 0;
-    for (int q = tid; q < S; q += NT) {
-        const int ctx = checked_context(p, p.context_lens[q], BS, blockIdx.x == 0 && tid == 0);
-        ctxs[q] = ctx;
-        tot += ctx;
-        mx = max(mx, ctx);
-    }
-    tot = cta_sum<NW>(tot, red);
-    mx = (int)cta_max<NW>(mx, red);
-    const int floor_p = p.partition_size;
-    const int p_max = max(floor_p, min(kMaxPartition, (max(mx, 1) + 31) / 32 * 32));
-    const long long budget = gridDim.x / HK; // pieces per K/V head
-    auto round_p = [&](long long t) {
-        const long long r = (t + 31) / 32 * 32;
-        return (int)max((long long)floor_p, min((long long)p_max, r));
-    };
-    auto count = [&](int cand) { // sum_s max(1, ceil(ctx_s / cand)), over the CTA
-        long long c = 0;
-        for (int q = tid; q < S; q += NT)
-            c += max(1, (ctxs[q] + cand - 1) / cand);
-        return cta_sum<NW>(c, red);
-    };
-    // sum_s max(1, ceil(ctx_s / P)) <= tot / P + S: P >= tot / (budget - S)
-    // always fits; first try the estimate with half a piece of rounding per
-    // sequence.
-    P = p_max;
-    if (budget > S) {
-        P = round_p((tot + (budget - S / 2) - 1) / (budget - S / 2));
-        if (count(P) > budget)
-            P = round_p((tot + (budget - S) - 1) / (budget - S));
-    }
-    // Pieces per sequence and their exclusive prefix sum, PER sequences per
-    // thread.
-    int cnt[PER];
-    int mine = 0;
-#pragma unroll
-    for (int k = 0; k < PER; ++k) {
-        const int q = tid * PER + k;
-        cnt[k] = q < S ? max(1, (ctxs[q] + P - 1) / P) : 0;
-        mine += cnt[k];
-    }
-    int incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o)
-            incl += v;
-    }
-    __syncthreads(); // red reuse
-    if (lane == 31)
-        red[warp] = incl;
-    __syncthreads();
-    int run = incl - mine;
-    for (int w = 0; w < warp; ++w)
-        run += (int)red[w];
-#pragma unroll
-    for (int k = 0; k < PER; ++k) {
-        const int q = tid * PER + k;
-        if (q < S)
-            pre[q] = run;
-        run += cnt[k];
-    }
-    if (tid == NT - 1)
-        pre[S] = run;
-    __syncthreads();
-    const long long b = blockIdx.x;
-    if (b >= (long long)HK * pre[S])
-        return false;
-    int lo = 0, hi = S - 1; // the last sequence with HK * pre[q] <= b
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if ((long long)HK * pre[mid] <= b)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    s = lo;
-    const int n = pre[s + 1] - pre[s];
-    const int r = (int)(b - (long long)HK * pre[s]);
-    kvh = r / n;
-    part = r - kvh * n;
-    return true;
-}
-
 // decode_group_kernel: one CTA per (K/V head, sequence, partition) of a
-// fixed partition size, grid (num_kv_heads, num_seqs, num_parts); or, with
-// balanced partitions, one CTA per piece of a 1-D grid.
+// fixed partition size; grid (num_kv_heads, num_seqs, num_parts).
 template <typename T, int D, int BS, int NW, int NS, bool TWO>
 __global__ void __launch_bounds__(NW * 32)
     decode_group_kernel(const __grid_constant__ GroupParams gp)
@@ -733,14 +576,12 @@ __global__ void __launch_bounds__(NW * 32)
     float *scales = reinterpret_cast<float *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes);
     int32_t *rank_ctx =
         reinterpret_cast<int32_t *>(smem + Cfg::kRingsBytes + Cfg::kBarBytes + Cfg::kScaleBytes);
-    int32_t *bal_ctx = rank_ctx + kRankMaxSeqs;
-    int32_t *bal_pre = bal_ctx + kBalMaxSeqs;
     int32_t *table = reinterpret_cast<int32_t *>(smem + Cfg::kFixedBytes);
     __shared__ int cta_flags, ranked_seq;
-    __shared__ long long bal_red[NW];
 
     pdl_launch_dependents();
-    int kvh = blockIdx.x, part = blockIdx.z, s = blockIdx.y, P = p.partition_size;
+    const int kvh = blockIdx.x, part = blockIdx.z, P = p.partition_size;
+    int s = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads, HK = p.num_kv_heads, G = H / HK;
 
@@ -751,13 +592,9 @@ __global__ void __launch_bounds__(NW * 32)
             mbar_init(smem_addr(&bars[warp * NS + k]), 1);
     fence_mbar_init();
     pdl_wait_prior_grid(); // every input may come from the previous kernel
-    if (gp.balanced) {
-        if (!balanced_piece<BS, NW>(p, bal_ctx, bal_pre, bal_red, s, kvh, part, P))
-            return; // uniform: this CTA has no piece
-    } else if (p.rank_seqs) { // longest sequences first (ranked_sequence)
+    if (p.rank_seqs) // longest sequences first (ranked_sequence)
         s = ranked_sequence(p.context_lens, p.num_seqs, blockIdx.y, tid, NW * 32, rank_ctx,
                             &ranked_seq);
-    }
 
     Wp w;
     w.init(lane);
@@ -938,544 +775,6 @@ __global__ void __launch_bounds__(NW * 32)
     if (u.num_parts > 1 && p.ws_count)
         merge_if_last<D>(p, s, kvh * G, G, s * HK + kvh, u.num_parts, tid, NW * 32, &cta_flags,
                          reinterpret_cast<float *>(rings));
-}
-
-// ---------------------------------------------------------------------------
-// decode_flat_kernel: balanced token ranges for grouped heads.
-//
-// The work of a launch is the list of units (sequence s, K/V head kvh), in
-// that order, each cut into chunks of CH tokens (n_s = ceil(ctx_s / CH) per
-// unit): C = num_kv_heads * sum_s n_s chunks in all. With R = min(N, C)
-// (N CTAs in the launch), CTA c < R takes the chunks [c*C/R, (c+1)*C/R) of
-// that list, whatever units they belong to, so every CTA streams the same
-// number of chunks (within one) however the context lengths are spread (a
-// fixed partition size leaves some SMs idle while a few long units finish). Every CTA derives the whole schedule from the context
-// lengths (a prefix sum in shared memory): the host needs no knowledge of
-// them and no extra launch is made.
-//
-// Inside a CTA the range falls into segments, one per unit it touches. The
-// NW warps share each segment as in decode_group_kernel (chunk j of the
-// segment to warp j % NW) and keep their bulk-copy rings going across
-// segment boundaries: a warp's copies of the next segment's chunks are in
-// flight while the CTA merges the current one. At the end of a segment every
-// warp leaves its (O, m, l) in a merge area, the CTA merges them, and writes
-// the output rows when the segment is the whole unit; else it writes its
-// piece (unnormalised O, m, l) to the workspace and counts in on the unit's
-// counter, and the last of the unit's CTAs merges the pieces, in CTA order.
-// A segment in the middle of a range is always a whole unit, so a CTA has at
-// most two pieces, in workspace slots (c, 0) (the unit that contains the
-// range's first chunk) and (c, 1).
-//
-// Fused append: before streaming, each CTA writes the new token's K/V rows
-// of every unit whose last chunk lies in its range (only that CTA reads
-// that chunk) straight into the cache, then fences the generic-proxy
-// writes against the copies that will read them.
-// ---------------------------------------------------------------------------
-constexpr int kFlatMaxSeqs = 512; // sequences per launch (context-length prefix in shared memory)
-constexpr int kFlatTable = 1024;  // block-table entries a CTA stages (its whole range)
-constexpr int kFlatMaxSegs = 32;  // segments per window (more: the range is walked in windows)
-
-// Chunks one CTA range may hold so that its block-table entries fit the
-// staged table: CH / BS entries per chunk when a chunk covers whole blocks;
-// else (a chunk is half a block) at most one per chunk, counting the
-// rounding at both ends of every segment.
-constexpr int flat_max_chunks_for(bool fp8, int block_size)
-{
-    return kFlatTable / ((fp8 ? 32 : 16) >= block_size ? (fp8 ? 32 : 16) / block_size : 2);
-}
-
-struct FlatSeg {
-    int s, kvh; // the unit
-    int a, b;   // its chunks [a, b) in this range
-    int n;      // chunks of the whole unit
-    int ctx;    // its context length (clamped)
-    int blk0;   // first block-table index of the sequence the segment reads
-    int tab;    // where those entries start in the staged table
-};
-
-template <typename T, int D, int BS, int NW, int NS, bool TWO> struct FlatCfg : GroupGeom<T, D> {
-    using Geo = GroupGeom<T, D>;
-    static_assert(BS == 8 || BS == 16 || BS == 32, "block_size");
-    static constexpr int kRows = TWO ? 16 : 8; // query rows a warp can hold
-    static constexpr int kRing = NS * Geo::kStage;
-    static constexpr int kSeg = BS < 16 ? BS : 16; // rows per TMA box
-    static constexpr int kRingsBytes = NW * kRing;
-    static constexpr int kMergeBytes = NW * kRows * Geo::kMergeStride * 4;
-    static constexpr int kBarBytes = NW * NS * 8;
-    static constexpr int kScaleBytes = Geo::kFp8 ? NW * NS * 2 * Geo::kChunk * 4 : 0;
-    static constexpr int kSegBytes = kFlatMaxSegs * (int)(sizeof(FlatSeg) + 4);
-    static constexpr int kSeqBytes = ((2 * kFlatMaxSeqs + 1) * 4 + 15) / 16 * 16;
-    static constexpr int kTableBytes = kFlatTable * 4;
-    static constexpr int kBytes = 1024 + kRingsBytes + kMergeBytes + kBarBytes + kScaleBytes +
-                                  kSegBytes + kSeqBytes + kTableBytes;
-    static constexpr int kMaxChunks = flat_max_chunks_for(Geo::kFp8, BS); // per CTA range
-    static_assert((kSeg * Geo::kRow) % 1024 == 0, "swizzle atoms");
-    static_assert(Geo::kChunk % kSeg == 0 && Geo::kChunk % 16 == 0, "chunk geometry");
-    static_assert(NW * 32 * 4 >= kFlatMaxSeqs, "four sequences per thread in the prefix sum");
-};
-
-// Bidirectional proxy fence for global memory: this thread's generic-proxy
-// writes before later async-proxy (bulk copy) reads of the same bytes.
-__device__ __forceinline__ void fence_proxy_async_global()
-{
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Resident CTAs per SM the flat launch is built for (registers are capped
-// to allow them). The macro exists for tuning sweeps.
-#ifndef PA_FLAT_CTAS_PER_SM
-#define PA_FLAT_CTAS_PER_SM 2
-#endif
-
-template <typename T, int D, int BS, int NW, int NS, bool TWO>
-__global__ void __launch_bounds__(NW * 32, PA_FLAT_CTAS_PER_SM)
-    decode_flat_kernel(const __grid_constant__ GroupParams gp)
-{
-    using Cfg = FlatCfg<T, D, BS, NW, NS, TWO>;
-    using Wp = GroupWarp<T, D, TWO>;
-    constexpr bool kFp8 = Cfg::kFp8;
-    constexpr int CH = Cfg::kChunk, SEG = Cfg::kSeg, ROW = Cfg::kRow, MS = Cfg::kMergeStride;
-    constexpr int NT = NW * 32, ROWS = Cfg::kRows;
-    constexpr int PER = (kFlatMaxSeqs + NT - 1) / NT;
-    constexpr unsigned FULL = 0xffffffffu;
-    const DecodeParams &p = gp.p;
-
-    extern __shared__ __align__(1024) unsigned char flat_smem[];
-    unsigned char *smem = flat_smem + ((1024u - (smem_addr(flat_smem) & 1023u)) & 1023u);
-    char *rings = reinterpret_cast<char *>(smem);
-    float *merge = reinterpret_cast<float *>(smem + Cfg::kRingsBytes);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kRingsBytes + Cfg::kMergeBytes);
-    float *scales = reinterpret_cast<float *>(reinterpret_cast<char *>(bars) + Cfg::kBarBytes);
-    FlatSeg *segs = reinterpret_cast<FlatSeg *>(reinterpret_cast<char *>(scales) + Cfg::kScaleBytes);
-    int *seg_bad = reinterpret_cast<int *>(segs + kFlatMaxSegs);
-    int *sQ = reinterpret_cast<int *>(reinterpret_cast<char *>(segs) + Cfg::kSegBytes);
-    int *sctx = sQ + kFlatMaxSeqs + 1;
-    int32_t *table = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(sQ) + Cfg::kSeqBytes);
-    __shared__ int s_flags; // 1: a block id outside the pool; 2: a wait ran out
-    __shared__ int s_nseg, s_ntab, s_last, s_slot0, s_pieces;
-    __shared__ float s_fac[NW][kGroupMaxHeads]; // per warp and row: 2^(m_w - M)
-    __shared__ float2 s_rowml[kGroupMaxHeads];  // per row: (M, L)
-    __shared__ long long s_wend;
-    __shared__ int s_warp_sum[NW];
-
-    pdl_launch_dependents();
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, N = gp.num_ctas;
-    const int S = p.num_seqs, H = p.num_heads, HK = p.num_kv_heads, G = H / HK;
-
-    if (tid == 0)
-        s_flags = 0;
-    if (lane == 0)
-        for (int k = 0; k < NS; ++k)
-            mbar_init(smem_addr(&bars[warp * NS + k]), 1);
-    fence_mbar_init();
-    pdl_wait_prior_grid(); // every input may come from the previous kernel
-
-    // Chunks per sequence and their exclusive prefix sum sQ (sQ[S] = total);
-    // thread t handles sequences PER*t .. PER*t + PER - 1.
-    {
-        int cnt[PER];
-        int tot = 0;
-#pragma unroll
-        for (int k = 0; k < PER; ++k) {
-            const int s = tid * PER + k;
-            int n = 0;
-            if (s < S) {
-                const int ctx = checked_context(p, p.context_lens[s], BS, c == 0);
-                sctx[s] = ctx;
-                n = (ctx + CH - 1) / CH;
-            }
-            cnt[k] = n;
-            tot += n;
-        }
-        int incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(FULL, incl, o);
-            if (lane >= o)
-                incl += v;
-        }
-        if (lane == 31)
-            s_warp_sum[warp] = incl;
-        __syncthreads();
-        int run = incl - tot;
-        for (int w2 = 0; w2 < warp; ++w2)
-            run += s_warp_sum[w2];
-#pragma unroll
-        for (int k = 0; k < PER; ++k) {
-            const int s = tid * PER + k;
-            if (s < S)
-                sQ[s] = run;
-            run += cnt[k];
-        }
-        if (tid == NT - 1)
-            sQ[S] = run;
-        __syncthreads();
-    }
-
-    // This CTA's chunks [R0, R1) of C. The ranges are cut over the first
-    // NR = min(N, C) CTAs, so none of them is empty (a unit's pieces then
-    // come from consecutive CTAs); CTAs past NR have nothing to stream.
-    // cta_of(x): the CTA holding chunk x.
-    const long long C = (long long)HK * sQ[S];
-    const long long NR = min((long long)N, C);
-    const long long R0 = c < NR ? C * c / NR : C, R1 = c < NR ? C * (c + 1) / NR : C;
-    auto cta_of = [&](long long x) { return (int)(((x + 1) * NR - 1) / C); };
-    auto range_start = [&](int cc) { return C * cc / NR; };
-
-    // Sequences without context get zero rows, from the CTA whose range
-    // holds their place in the list (the last CTA when that is the end).
-    for (int s = tid; s < S; s += NT) {
-        if (sQ[s + 1] != sQ[s])
-            continue;
-        const long long at = (long long)HK * sQ[s];
-        if ((at < C ? cta_of(at) : N - 1) != c)
-            continue;
-        for (int e = 0; e < H * D; ++e)
-            store_out(p.out, p.out_dtype, (size_t)s * H * D + e, 0.f);
-    }
-
-    Wp w;
-    w.init(lane);
-    w.reset();
-    const char *kpool = static_cast<const char *>(p.key_cache);
-    const char *vpool = static_cast<const char *>(p.value_cache);
-    char *ring = rings + (size_t)warp * Cfg::kRing;
-    const uint32_t ring_s = smem_addr(ring);
-    const uint32_t bar0 = smem_addr(&bars[warp * NS]);
-    float *wscales = scales + (size_t)warp * NS * 2 * CH; // fp8: [stage][K | V][CH]
-    const float qs = p.qk_scale_log2;
-    int issued = 0, consumed = 0; // this warp's copies, over all windows
-    bool failed = false;          // warp-uniform: a wait ran out
-
-    long long pos = R0;
-    while (pos < R1) { // CTA-uniform
-        // The next window of segments, from chunk pos (thread 0).
-        if (tid == 0) {
-            int lo = 0, hi = S - 1; // the last sequence with HK * sQ[s] <= pos
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if ((long long)HK * sQ[mid] <= pos)
-                    lo = mid;
-                else
-                    hi = mid - 1;
-            }
-            int s = lo;
-            int kvh = (int)((pos - (long long)HK * sQ[s]) / (sQ[s + 1] - sQ[s]));
-            int k = 0, tab = 0;
-            while (pos < R1 && k < kFlatMaxSegs) {
-                const int n = sQ[s + 1] - sQ[s];
-                const long long pu = (long long)HK * sQ[s] + (long long)kvh * n;
-                FlatSeg sg;
-                sg.s = s;
-                sg.kvh = kvh;
-                sg.a = (int)(pos - pu);
-                sg.b = (int)min((long long)n, R1 - pu);
-                sg.n = n;
-                sg.ctx = sctx[s];
-                sg.blk0 = sg.a * CH / BS;
-                sg.tab = tab;
-                const int entries = (min(sg.b * CH, sg.ctx) + BS - 1) / BS - sg.blk0;
-                if (k > 0 && tab + entries > kFlatTable)
-                    break; // the rest in the next window (the host sizes ranges to fit)
-                tab += entries;
-                segs[k] = sg;
-                seg_bad[k] = 0;
-                ++k;
-                pos = pu + sg.b;
-                if (pos < R1 && ++kvh == HK) {
-                    kvh = 0;
-                    do
-                        ++s;
-                    while (sQ[s + 1] == sQ[s]);
-                }
-            }
-            s_nseg = k;
-            s_ntab = tab;
-            s_wend = pos;
-        }
-        __syncthreads();
-        const int nseg = s_nseg, ntab = min(s_ntab, kFlatTable);
-        pos = s_wend;
-
-        // The window's block-table entries, and the first segment's query rows.
-        for (int e = tid; e < ntab; e += NT) {
-            int k = 0;
-            while (k + 1 < nseg && segs[k + 1].tab <= e)
-                ++k;
-            table[e] = p.block_tables[(size_t)segs[k].s * p.max_blocks_per_seq + segs[k].blk0 +
-                                      (e - segs[k].tab)];
-        }
-        w.load_q(p.query, (size_t)segs[0].s * H + (size_t)segs[0].kvh * G, G);
-        __syncthreads();
-
-        // Fused append: the new rows of the units that end in this window go
-        // to the cache before any copy of their last chunk is issued.
-        if (p.new_key != nullptr) {
-            for (int k = warp; k < nseg; k += NW) {
-                const FlatSeg sg = segs[k];
-                if (sg.b != sg.n) // warp-uniform
-                    continue;
-                NewRow<T, D, BS> nr;
-                nr.load(p, (size_t)sg.s * HK + sg.kvh, lane);
-                uint4 *dst;
-                float *sdst;
-                const int t = sg.ctx - 1;
-                const int te = sg.tab + t / BS - sg.blk0;
-                nr.locate(p, te < kFlatTable ? table[te] : -1, sg.kvh, t % BS, lane, dst, sdst);
-                if (dst)
-                    *dst = nr.val;
-                if (sdst)
-                    *sdst = nr.scale;
-            }
-            fence_proxy_async_global();
-        }
-        __syncthreads();
-
-        // This warp's chunks in window order: chunk a + warp + j*NW of each
-        // segment. Issue cursor (ik, ic), warp-uniform; lane 0 copies.
-        int ik = 0, ic = segs[0].a + warp;
-        auto advance = [&]() {
-            while (ik < nseg && ic >= segs[ik].b)
-                if (++ik < nseg)
-                    ic = segs[ik].a + warp;
-        };
-        advance();
-        auto issue = [&]() {
-            if (lane == 0) {
-                const FlatSeg &sg = segs[ik];
-                const int tok0 = ic * CH;
-                const int rows = min(CH, sg.ctx - tok0);
-                const int nbox = (rows + SEG - 1) / SEG;
-                const int st = issued % NS;
-                const uint32_t dk = ring_s + st * Cfg::kStage, dv = dk + Cfg::kHalf;
-                const uint32_t bar = bar0 + st * 8;
-                mbar_arrive_expect_tx(bar, (uint32_t)(nbox * SEG * (ROW + (kFp8 ? 4 : 0)) * 2));
-                for (int bx = 0; bx < nbox; ++bx) {
-                    const int tok = tok0 + bx * SEG;
-                    const int te = sg.tab + tok / BS - sg.blk0;
-                    int b = te < kFlatTable ? table[te] : -1;
-                    if (b < 0 || b >= p.num_blocks) {
-                        seg_bad[ik] = 1;
-                        b = 0;
-                    }
-                    const int tile = b * HK + sg.kvh;
-                    if constexpr (kFp8) {
-                        const int off = tok % BS;
-                        tma_load_3d(dk + bx * SEG * ROW, &gp.tk, 0, off, tile, bar);
-                        tma_load_3d(dv + bx * SEG * ROW, &gp.tv, 0, off, tile, bar);
-                        const size_t sofs =
-                            (size_t)tile * (BS * (D + 4)) + BS * D + (size_t)off * 4;
-                        float *sk = wscales + (st * 2) * CH + bx * SEG;
-                        bulk_g2s(smem_addr(sk), kpool + sofs, SEG * 4, bar);
-                        bulk_g2s(smem_addr(sk + CH), vpool + sofs, SEG * 4, bar);
-                    } else {
-                        const int y = tile * BS + tok % BS;
-                        tma_load_3d(dk + bx * SEG * ROW, &gp.tk, 0, 0, y, bar);
-                        tma_load_3d(dv + bx * SEG * ROW, &gp.tv, 0, 0, y, bar);
-                    }
-                }
-            }
-            ++issued;
-            ic += NW;
-            advance();
-        };
-        while (!failed && ik < nseg && issued - consumed < NS)
-            issue();
-
-        for (int k = 0; k < nseg; ++k) { // CTA-uniform
-            const FlatSeg sg = segs[k];
-            for (int cc = sg.a + warp; cc < sg.b; cc += NW) {
-                if (failed)
-                    continue;
-                const int st = consumed % NS;
-                const bool ok = mbar_wait_bounded(bar0 + st * 8, (consumed / NS) & 1, kWaitLimitNs);
-                if (__any_sync(FULL, !ok)) {
-                    failed = true;
-                    continue;
-                }
-                char *sk = ring + st * Cfg::kStage;
-                float *ksc = wscales + (st * 2) * CH;
-                w.chunk(sk, sk + Cfg::kHalf, ksc, ksc + CH, min(CH, sg.ctx - cc * CH), qs);
-                __syncwarp();
-                ++consumed;
-                if (ik < nseg)
-                    issue();
-            }
-
-            // End of the segment: this warp's state to the merge area, the
-            // next segment's query rows on their way, a fresh state.
-            float *mw = merge + (size_t)warp * ROWS * MS;
-            w.store(mw, G);
-            if (k + 1 < nseg)
-                w.load_q(p.query, (size_t)segs[k + 1].s * H + (size_t)segs[k + 1].kvh * G, G);
-            w.reset();
-            if (failed && lane == 0)
-                atomicOr(&s_flags, 2);
-            if (seg_bad[k] && tid == 0)
-                atomicOr(&s_flags, 1);
-            __syncthreads();
-
-            // Merge the warps: per row, each warp's factor 2^(m_w - M) (0 for
-            // a warp without chunks here) and the row's (M, L); then every
-            // output element sums its warps in warp order.
-            const bool whole = sg.a == 0 && sg.b == sg.n;
-            const bool bad = seg_bad[k] != 0 || (s_flags & 2) != 0;
-            const long long pu = (long long)HK * sQ[sg.s] + (long long)sg.kvh * sg.n;
-            const size_t slot = 2 * (size_t)c + (pu <= R0 ? 0 : 1);
-            if (tid < G) {
-                float M = -INFINITY;
-#pragma unroll
-                for (int w2 = 0; w2 < NW; ++w2)
-                    M = fmaxf(M, merge[((size_t)w2 * ROWS + tid) * MS + D]);
-                float L = 0.f;
-#pragma unroll
-                for (int w2 = 0; w2 < NW; ++w2) {
-                    const float *mv = merge + ((size_t)w2 * ROWS + tid) * MS;
-                    const float f = mv[D] == -INFINITY ? 0.f : exp2f(mv[D] - M);
-                    L = fmaf(mv[D + 1], f, L);
-                    s_fac[w2][tid] = f;
-                }
-                s_rowml[tid] = make_float2(M, L);
-            }
-            __syncthreads();
-            for (int idx = tid; idx < G * D; idx += NT) {
-                const int g = idx / D, d = idx - g * D;
-                float O = 0.f;
-#pragma unroll
-                for (int w2 = 0; w2 < NW; ++w2)
-                    O = fmaf(merge[((size_t)w2 * ROWS + g) * MS + d], s_fac[w2][g], O);
-                const float2 ml = s_rowml[g];
-                if (bad)
-                    O = NAN;
-                if (whole) {
-                    store_out(p.out, p.out_dtype, ((size_t)sg.s * H + sg.kvh * G + g) * D + d,
-                              ml.y > 0.f ? O / ml.y : O);
-                } else {
-                    p.ws_acc[(slot * G + g) * D + d] = O;
-                    if (d == 0) {
-                        p.ws_ml[(slot * G + g) * 2] = bad ? 0.f : ml.x;
-                        p.ws_ml[(slot * G + g) * 2 + 1] = bad ? 1.f : ml.y;
-                    }
-                }
-            }
-            __syncthreads();
-            if (whole)
-                continue;
-
-            // Count this piece in; the unit's last CTA merges its pieces in
-            // CTA order and resets the counter. Piece i comes from CTA
-            // c0 + i; only the first can sit in slot 1 (when the unit starts
-            // inside that CTA's range), the others start their ranges.
-            if (tid == 0) {
-                const int c0 = cta_of(pu), c1 = cta_of(pu + sg.n - 1);
-                s_last = arrive_acq_rel(&p.ws_count[sg.s * HK + sg.kvh]) == c1 - c0;
-                s_slot0 = 2 * c0 + (pu == range_start(c0) ? 0 : 1);
-                s_pieces = c1 - c0 + 1;
-            }
-            __syncthreads();
-            if (!s_last)
-                continue;
-            const int np = s_pieces;
-            const size_t slot0 = (size_t)s_slot0;
-            auto piece_slot = [&](int i) { return i == 0 ? slot0 : (slot0 & ~(size_t)1) + 2 * i; };
-            if (np <= 32 && np * G <= Cfg::kMergeBytes / 4) {
-                // Each row's normalised weights 2^(m_i - M) / L in the merge
-                // area: one warp per row, lane i holding piece i, every
-                // row's (m, l) loaded before any reduction.
-                float *wts = merge;
-                constexpr int RPW = (kGroupMaxHeads + NW - 1) / NW; // rows per warp
-                float2 ml[RPW];
-#pragma unroll
-                for (int j = 0; j < RPW; ++j) {
-                    const int g = warp + j * NW;
-                    ml[j] = make_float2(-INFINITY, 0.f);
-                    if (g < G && lane < np)
-                        ml[j] = __ldcg(reinterpret_cast<const float2 *>(p.ws_ml) +
-                                       piece_slot(lane) * G + g);
-                }
-#pragma unroll
-                for (int j = 0; j < RPW; ++j) {
-                    const int g = warp + j * NW;
-                    if (g >= G) // warp-uniform
-                        continue;
-                    float M = ml[j].x;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1)
-                        M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
-                    const float f = lane < np ? exp2f(ml[j].x - M) : 0.f;
-                    float L = f * ml[j].y;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1)
-                        L += __shfl_xor_sync(FULL, L, o);
-                    if (lane < np)
-                        wts[g * np + lane] = f / L;
-                }
-                __syncthreads();
-                // Every output element of this thread over the pieces, the
-                // loads of one piece issued together.
-                constexpr int KO = kGroupMaxHeads * D / NT; // outputs per thread, at most
-                float O[KO];
-#pragma unroll
-                for (int k2 = 0; k2 < KO; ++k2)
-                    O[k2] = 0.f;
-                for (int i = 0; i < np; ++i) {
-                    const float *acc = p.ws_acc + piece_slot(i) * G * D;
-                    float v[KO];
-#pragma unroll
-                    for (int k2 = 0; k2 < KO; ++k2) {
-                        const int idx = tid + k2 * NT;
-                        v[k2] = idx < G * D ? __ldcg(acc + idx) : 0.f;
-                    }
-#pragma unroll
-                    for (int k2 = 0; k2 < KO; ++k2) {
-                        const int idx = tid + k2 * NT;
-                        if (idx < G * D)
-                            O[k2] = fmaf(v[k2], wts[(idx / D) * np + i], O[k2]);
-                    }
-                }
-#pragma unroll
-                for (int k2 = 0; k2 < KO; ++k2) {
-                    const int idx = tid + k2 * NT;
-                    if (idx < G * D) {
-                        const int g = idx / D, d = idx - g * D;
-                        store_out(p.out, p.out_dtype,
-                                  ((size_t)sg.s * H + sg.kvh * G + g) * D + d, O[k2]);
-                    }
-                }
-            } else { // many pieces: per element
-                for (int idx = tid; idx < G * D; idx += NT) {
-                    const int g = idx / D, d = idx - g * D;
-                    float M = -INFINITY;
-                    for (int i = 0; i < np; ++i)
-                        M = fmaxf(M, __ldcg(&p.ws_ml[(piece_slot(i) * G + g) * 2]));
-                    float L = 0.f, O = 0.f;
-                    for (int i = 0; i < np; ++i) {
-                        const size_t sl = piece_slot(i);
-                        const float f = exp2f(__ldcg(&p.ws_ml[(sl * G + g) * 2]) - M);
-                        L = fmaf(__ldcg(&p.ws_ml[(sl * G + g) * 2 + 1]), f, L);
-                        O = fmaf(__ldcg(&p.ws_acc[(sl * G + g) * D + d]), f, O);
-                    }
-                    store_out(p.out, p.out_dtype, ((size_t)sg.s * H + sg.kvh * G + g) * D + d,
-                              O / L);
-                }
-            }
-            if (tid == 0)
-                p.ws_count[sg.s * HK + sg.kvh] = 0;
-            __syncthreads(); // the merge area holds the next segment's states next
-        }
-    }
-
-    if (failed) // the copies still in flight land before the CTA exits
-        for (int k = consumed; k < issued; ++k)
-            mbar_wait_bounded(bar0 + (k % NS) * 8, (k / NS) & 1, kWaitLimitNs);
-    __syncthreads();
-    if (tid == 0) {
-        if (s_flags & 2)
-            report(p.dev_err, PA_DEVERR_TIMEOUT);
-        if (s_flags & 1)
-            report(p.dev_err, PA_DEVERR_BLOCK_ID);
-    }
 }
 
 } // namespace pagedkv

@@ -215,85 +215,6 @@ size_t workspace_bytes_for(int64_t units, int64_t num_parts, int head_dim)
     return kCounterBytes + acc_padded + (size_t)(units * num_parts * 2) * sizeof(float);
 }
 
-// decode_flat_kernel (grouped heads with automatic partitioning): 4 warps x
-// 2 TMA stages, persistent at up to kFlatCtasPerSm CTAs per SM; more CTAs
-// (up to kFlatCtaCap per SM) only when a CTA's range would hold more chunks
-// than it can stage block-table entries for; beyond that the launch falls
-// back to decode_group_kernel. Its workspace: the arrival counters (one per
-// (sequence, K/V head)), then two piece slots per CTA of G rows of (O [D],
-// then (m, l)).
-#ifndef PA_FLAT_WARPS
-#define PA_FLAT_WARPS 4
-#endif
-#ifndef PA_FLAT_STAGES
-#define PA_FLAT_STAGES 2
-#endif
-constexpr int kFlatWarps = PA_FLAT_WARPS;
-constexpr int kFlatStages = PA_FLAT_STAGES;
-constexpr int kFlatCtasPerSm = PA_FLAT_CTAS_PER_SM;
-constexpr int kFlatCtaCap = 8;
-
-// Chunks one flat CTA range may hold for a cache (FlatCfg::kMaxChunks); the
-// smallest over the built formats and block sizes bounds the workspace.
-int flat_max_chunks(const pa_cache_desc *c)
-{
-    return flat_max_chunks_for(c->dtype == PA_FP8_E4M3, c->block_size);
-}
-constexpr int kFlatMinMaxChunks = flat_max_chunks_for(true, 8);
-static_assert(kFlatMinMaxChunks <= flat_max_chunks_for(false, 8) &&
-                  kFlatMinMaxChunks <= flat_max_chunks_for(false, 32) &&
-                  kFlatMinMaxChunks <= flat_max_chunks_for(true, 32),
-              "the workspace bound takes the smallest range");
-
-bool flat_eligible(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c,
-                   int32_t max_ctx, int32_t requested)
-{
-    return requested == 0 && max_ctx > 0 && num_seqs <= kFlatMaxSeqs &&
-           use_group_kernel(c, num_heads) &&
-           (int64_t)num_seqs * c->num_kv_heads <= kSplitCounters;
-}
-
-// Upper bound of a launch's chunks (every sequence at max_ctx).
-int64_t flat_chunk_bound(int32_t num_seqs, int32_t num_kv_heads, int32_t max_ctx, int chunk)
-{
-    return (int64_t)num_seqs * num_kv_heads * ((max_ctx + chunk - 1) / chunk);
-}
-
-// CTAs of a flat launch, or 0 when it would need more than kFlatCtaCap per SM.
-int64_t flat_ctas(int64_t chunk_bound, int max_chunks, int resident_per_sm, int sm_count)
-{
-    const int64_t n = std::max<int64_t>((int64_t)std::min(resident_per_sm, kFlatCtasPerSm) *
-                                            sm_count,
-                                        (chunk_bound + max_chunks - 1) / max_chunks);
-    return n > (int64_t)kFlatCtaCap * sm_count ? 0 : n;
-}
-
-// Which launch grouped query heads with automatic partitioning take (when
-// the workspace allows; else fixed partitions): 0 decode_flat_kernel, 1
-// balanced partitions of decode_group_kernel, 2 fixed partitions. The macro
-// exists for comparisons.
-#ifndef PA_GROUP_LAUNCH
-#define PA_GROUP_LAUNCH 1
-#endif
-
-// Balanced partitions: the floor of the partition size, so that the merging
-// CTA can hold one weight per (head, partition) (G * parts <= kMergeWeights)
-// and no CTA streams less than 256 tokens; 0 when no floor fits.
-int balanced_floor(int32_t num_heads, const pa_cache_desc *c, int32_t max_ctx)
-{
-    const int G = num_heads / c->num_kv_heads;
-    const int64_t per = kMergeWeights / G; // partitions the merge can weigh
-    const int64_t need = (max_ctx + per - 1) / per;
-    const int64_t f = std::max<int64_t>(256, (need + 31) / 32 * 32);
-    return f <= kMaxPartition ? (int)f : 0;
-}
-
-size_t flat_workspace_bytes(int64_t ctas, int group, int head_dim)
-{
-    const size_t acc = (size_t)ctas * 2 * group * head_dim * sizeof(float);
-    return kCounterBytes + (acc + 255) / 256 * 256 + (size_t)ctas * 2 * group * 2 * sizeof(float);
-}
-
 // Raise a kernel's dynamic shared-memory limit once per device. `done` must
 // be distinct for every kernel (one static per template instantiation of the
 // caller), since the attribute belongs to the function.
@@ -437,61 +358,16 @@ pa_status encode_pool_rows(CUtensorMap *map, const void *pool, const pa_cache_de
     return PA_OK;
 }
 
-// Resident decode_group_kernel CTAs per SM (balanced partitions size their
-// grid by it), looked up once per device and instantiation.
-template <typename Kernel>
-int resident_ctas(Kernel k, int threads, size_t smem, std::atomic<int> (&cache)[kMaxDevices])
-{
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        cudaGetLastError();
-        return 0;
-    }
-    int n = cache[dev].load(std::memory_order_relaxed);
-    if (n > 0)
-        return n;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess) {
-        cudaGetLastError();
-        return 0;
-    }
-    cache[dev].store(n, std::memory_order_relaxed);
-    return n;
-}
-
-// Balanced partitions: CTAs per launch, in waves of the resident CTAs. The
-// macro exists for tuning sweeps.
-#ifndef PA_BAL_WAVES
-#define PA_BAL_WAVES 2
-#endif
-
 template <typename T, int D, int BS, bool TWO>
-pa_status launch_group(const GroupParams &gp_in, cudaStream_t stream)
+pa_status launch_group(const GroupParams &gp, cudaStream_t stream)
 {
     using Cfg = GroupCfg<T, D, BS, kGroupWarps, kGroupStages>;
     auto kernel = decode_group_kernel<T, D, BS, kGroupWarps, kGroupStages, TWO>;
     static std::atomic<size_t> smem_set[kMaxDevices];
-    static std::atomic<int> resident[kMaxDevices];
-    GroupParams gp = gp_in;
     const DecodeParams &p = gp.p;
     cudaError_t e = allow_smem(kernel, Cfg::smem_bytes(kMaxPartition), smem_set);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute(group decode)");
-    if (gp.balanced) {
-        // Enough CTAs for PA_BAL_WAVES waves, for one piece per (sequence,
-        // K/V head), and for every piece at the largest partition.
-        const int occ = std::max(1, resident_ctas(kernel, kGroupWarps * 32,
-                                                  Cfg::smem_bytes(kMaxPartition), resident));
-        const int64_t units = (int64_t)p.num_seqs * p.num_kv_heads;
-        const int64_t n = std::max<int64_t>(
-            {(int64_t)PA_BAL_WAVES * occ * sm_count_of_current_device(), units,
-             units * ((p.max_context_len + kMaxPartition - 1) / kMaxPartition)});
-        gp.num_ctas = (int32_t)n;
-        e = launch_pdl(kernel, dim3((unsigned)n), dim3(kGroupWarps * 32),
-                       Cfg::smem_bytes(kMaxPartition), stream, gp);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "group decode launch");
-        return ok();
-    }
     e = launch_pdl(kernel, dim3(p.num_kv_heads, p.num_seqs, p.num_parts),
                    dim3(kGroupWarps * 32), Cfg::smem_bytes(p.partition_size), stream, gp);
     if (e != cudaSuccess)
@@ -524,13 +400,11 @@ pa_status group_bs(const GroupParams &gp, int bs, cudaStream_t st)
     return fail(PA_ERR_UNSUPPORTED, "block_size %d", bs);
 }
 
-pa_status dispatch_group(const DecodeParams &p, const pa_cache_desc *c, cudaStream_t st,
-                         bool balanced = false)
+pa_status dispatch_group(const DecodeParams &p, const pa_cache_desc *c, cudaStream_t st)
 {
     GroupParams gp;
     std::memset(&gp, 0, sizeof(gp));
     gp.p = p;
-    gp.balanced = balanced ? 1 : 0;
     pa_status s = encode_pool_rows(&gp.tk, p.key_cache, c);
     if (s == PA_OK)
         s = encode_pool_rows(&gp.tv, p.value_cache, c);
@@ -544,106 +418,6 @@ pa_status dispatch_group(const DecodeParams &p, const pa_cache_desc *c, cudaStre
                   : group_bs<__half, 64>(gp, c->block_size, st);
     return bf ? group_bs<__nv_bfloat16, 128>(gp, c->block_size, st)
               : group_bs<__half, 128>(gp, c->block_size, st);
-}
-
-// One decode_flat_kernel launch if the workspace holds what it needs (else
-// *launched stays false and the caller falls back to decode_group_kernel).
-// clear_counters: zero the counters it uses first (the built-in scratch).
-template <typename T, int D, int BS, bool TWO>
-pa_status launch_flat(GroupParams gp, void *ws, size_t ws_bytes, bool clear_counters,
-                      cudaStream_t stream, bool *launched)
-{
-    using Cfg = FlatCfg<T, D, BS, kFlatWarps, kFlatStages, TWO>;
-    auto kernel = decode_flat_kernel<T, D, BS, kFlatWarps, kFlatStages, TWO>;
-    static std::atomic<size_t> smem_set[kMaxDevices];
-    static std::atomic<int> resident[kMaxDevices];
-    const DecodeParams &p = gp.p;
-    cudaError_t e = allow_smem(kernel, Cfg::kBytes, smem_set);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "cudaFuncSetAttribute(flat decode)");
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess)
-        return cuda_fail(e, "cudaGetDevice");
-    int occ = dev >= 0 && dev < kMaxDevices ? resident[dev].load(std::memory_order_relaxed) : 0;
-    if (occ <= 0) {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kFlatWarps * 32,
-                                                          Cfg::kBytes);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "occupancy query (flat decode)");
-        if (occ <= 0)
-            return ok(); // cannot be resident: the grid kernel instead
-        if (dev >= 0 && dev < kMaxDevices)
-            resident[dev].store(occ, std::memory_order_relaxed);
-    }
-    static_assert(Cfg::kMaxChunks >= kFlatMinMaxChunks, "workspace bound");
-    const int G = p.num_heads / p.num_kv_heads;
-    const int64_t n = flat_ctas(flat_chunk_bound(p.num_seqs, p.num_kv_heads, p.max_context_len,
-                                                 Cfg::kChunk),
-                                Cfg::kMaxChunks, occ, sm_count_of_current_device());
-    if (n == 0 || !ws || !aligned16(ws) || ws_bytes < flat_workspace_bytes(n, G, D))
-        return ok();
-    char *w = static_cast<char *>(ws);
-    const size_t acc = (size_t)n * 2 * G * D * sizeof(float);
-    gp.p.ws_count = reinterpret_cast<int32_t *>(w);
-    gp.p.ws_acc = reinterpret_cast<float *>(w + kCounterBytes);
-    gp.p.ws_ml = reinterpret_cast<float *>(w + kCounterBytes + (acc + 255) / 256 * 256);
-    gp.num_ctas = (int32_t)n;
-    if (clear_counters) {
-        e = cudaMemsetAsync(ws, 0, (size_t)p.num_seqs * p.num_kv_heads * sizeof(int32_t), stream);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "clearing the built-in scratch counters");
-    }
-    e = launch_pdl(kernel, dim3((unsigned)n), dim3(kFlatWarps * 32), Cfg::kBytes, stream, gp);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "flat decode launch");
-    *launched = true;
-    return ok();
-}
-
-template <typename T, int D, int BS>
-pa_status flat_rows(const GroupParams &gp, void *ws, size_t b, bool clr, cudaStream_t st,
-                    bool *launched)
-{
-    if (gp.p.num_heads / gp.p.num_kv_heads > 8)
-        return launch_flat<T, D, BS, true>(gp, ws, b, clr, st, launched);
-    return launch_flat<T, D, BS, false>(gp, ws, b, clr, st, launched);
-}
-
-template <typename T, int D>
-pa_status flat_bs(const GroupParams &gp, int bs, void *ws, size_t b, bool clr, cudaStream_t st,
-                  bool *launched)
-{
-    switch (bs) {
-    case 8: return flat_rows<T, D, 8>(gp, ws, b, clr, st, launched);
-    case 16: return flat_rows<T, D, 16>(gp, ws, b, clr, st, launched);
-    case 32: return flat_rows<T, D, 32>(gp, ws, b, clr, st, launched);
-    }
-    return fail(PA_ERR_UNSUPPORTED, "block_size %d", bs);
-}
-
-pa_status dispatch_flat(const DecodeParams &p, const pa_cache_desc *c, void *ws, size_t bytes,
-                        bool clear_counters, cudaStream_t st, bool *launched)
-{
-    *launched = false;
-    GroupParams gp;
-    std::memset(&gp, 0, sizeof(gp));
-    gp.p = p;
-    pa_status s = encode_pool_rows(&gp.tk, p.key_cache, c);
-    if (s == PA_OK)
-        s = encode_pool_rows(&gp.tv, p.value_cache, c);
-    if (s != PA_OK)
-        return s;
-    if (c->dtype == PA_FP8_E4M3) // f16 rows, head_dim 128 (use_group_kernel)
-        return flat_bs<E4M3, 128>(gp, c->block_size, ws, bytes, clear_counters, st, launched);
-    const bool bf = c->dtype == PA_BF16;
-    if (c->head_dim == 64)
-        return bf ? flat_bs<__nv_bfloat16, 64>(gp, c->block_size, ws, bytes, clear_counters, st,
-                                               launched)
-                  : flat_bs<__half, 64>(gp, c->block_size, ws, bytes, clear_counters, st,
-                                        launched);
-    return bf ? flat_bs<__nv_bfloat16, 128>(gp, c->block_size, ws, bytes, clear_counters, st,
-                                            launched)
-              : flat_bs<__half, 128>(gp, c->block_size, ws, bytes, clear_counters, st, launched);
 }
 
 template <typename T, typename QT>
@@ -753,26 +527,10 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t hea
         check_partition_request(partition_size) != PA_OK)
         return (size_t)-1;
     const int P = partition_size == 0 ? kMinAutoPartition : partition_size;
-    size_t bytes = 0;
-    if (max_context_len > P) {
-        const int64_t parts = (max_context_len + P - 1) / P;
-        bytes = workspace_bytes_for((int64_t)num_seqs * num_heads, parts, head_dim);
-    }
-    // Automatic partitioning may take the balanced grouped-heads launch:
-    // cover its pieces for any group size G = num_heads / num_kv_heads >= 2
-    // (at most num_heads / 2 K/V heads, G <= 16, 16-token chunks or longer).
-    if (partition_size == 0 && num_heads >= 2 && max_context_len > 0 &&
-        num_seqs <= kFlatMaxSeqs) {
-        const int sms = sm_count_of_current_device();
-        const int64_t bound = flat_chunk_bound(num_seqs, num_heads / 2, max_context_len, 16);
-        const int64_t n = std::min<int64_t>(
-            (int64_t)kFlatCtaCap * sms,
-            std::max<int64_t>((int64_t)kFlatCtasPerSm * sms,
-                              (bound + kFlatMinMaxChunks - 1) / kFlatMinMaxChunks));
-        bytes = std::max(bytes,
-                         flat_workspace_bytes(n, std::min(num_heads, kGroupMaxHeads), head_dim));
-    }
-    return bytes;
+    if (max_context_len <= P)
+        return 0;
+    const int64_t parts = (max_context_len + P - 1) / P;
+    return workspace_bytes_for((int64_t)num_seqs * num_heads, parts, head_dim);
 }
 
 int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
@@ -783,15 +541,6 @@ int32_t pa_decode_partition_size(int32_t num_seqs, int32_t num_heads,
         num_heads % cache->num_kv_heads != 0 || max_context_len < 0 ||
         check_partition_request(partition_size) != PA_OK)
         return -1;
-    if (PA_GROUP_LAUNCH != 2 &&
-        flat_eligible(num_seqs, num_heads, cache, max_context_len, partition_size) &&
-        (PA_GROUP_LAUNCH == 0
-             ? flat_ctas(flat_chunk_bound(num_seqs, cache->num_kv_heads, max_context_len,
-                                          cache->dtype == PA_FP8_E4M3 ? 32 : 16),
-                         flat_max_chunks(cache), kFlatCtasPerSm,
-                         sm_count_of_current_device()) > 0
-             : balanced_floor(num_heads, cache, max_context_len) > 0))
-        return 0; // work balanced per launch (given a sufficient workspace)
     return choose_partition(num_seqs, num_heads, cache, max_context_len, partition_size,
                             partition_size == 0 ? sm_count_of_current_device() : 148);
 }
@@ -936,47 +685,6 @@ pa_status decode_common(void *out, pa_dtype out_dtype, const void *query, int32_
     p.qk_scale_log2 = scale * 1.4426950408889634f;
     p.new_key = new_key;
     p.new_value = new_value;
-    // Grouped heads with automatic partitioning: balanced work when the
-    // workspace holds it (decode_flat_kernel's pieces, or the partials of
-    // balanced partitions).
-    if (PA_GROUP_LAUNCH != 2 &&
-        flat_eligible(num_seqs, num_heads, cache, max_context_len, partition_size)) {
-        void *fw = workspace;
-        size_t fb = workspace_bytes;
-        if (builtin_scratch) {
-            if ((s = noalloc_scratch(&fw)) != PA_OK)
-                return s;
-            fb = PA_NOALLOC_SCRATCH_BYTES;
-        }
-        const cudaStream_t st = static_cast<cudaStream_t>(stream);
-        if (PA_GROUP_LAUNCH == 0) {
-            bool launched = false;
-            s = dispatch_flat(p, cache, fw, fb, builtin_scratch, st, &launched);
-            if (s != PA_OK || launched)
-                return s;
-        } else if (const int floor_p = balanced_floor(num_heads, cache, max_context_len)) {
-            const int64_t stride = (max_context_len + floor_p - 1) / floor_p;
-            const int64_t units = (int64_t)num_seqs * num_heads;
-            if (fw && aligned16(fw) && fb >= workspace_bytes_for(units, stride, cache->head_dim)) {
-                if (builtin_scratch) {
-                    const cudaError_t e = cudaMemsetAsync(
-                        fw, 0, (size_t)num_seqs * cache->num_kv_heads * sizeof(int32_t), st);
-                    if (e != cudaSuccess)
-                        return cuda_fail(e, "clearing the built-in scratch counters");
-                }
-                DecodeParams q = p;
-                char *w = static_cast<char *>(fw);
-                const size_t acc = (size_t)(units * stride * cache->head_dim) * sizeof(float);
-                q.partition_size = floor_p;
-                q.num_parts = (int32_t)stride;
-                q.rank_seqs = 0;
-                q.ws_count = reinterpret_cast<int32_t *>(w);
-                q.ws_acc = reinterpret_cast<float *>(w + kCounterBytes);
-                q.ws_ml = reinterpret_cast<float *>(w + kCounterBytes + (acc + 255) / 256 * 256);
-                return dispatch_group(q, cache, st, true);
-            }
-        }
-    }
     if (parts > 1) {
         const int64_t units = (int64_t)num_seqs * num_heads;
         const size_t need = workspace_bytes_for(units, parts, cache->head_dim);

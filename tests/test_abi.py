@@ -108,28 +108,10 @@ def test_write_and_copy_reject_bad_arguments(lib):
                             None) == lib.PA_ERR_INVALID_ARG
 
 
-def flat_bound(S, H, D, ctx, sms=148):
-    """The balanced grouped-heads launch's workspace bound: 65536 counters,
-    then two piece slots per CTA of min(H, 16) rows (O [D], then (m, l)),
-    for min(8 * SMs, max(2 * SMs, chunks / 256)) CTAs, chunks counted at
-    H / 2 K/V heads and 16 tokens each."""
-    chunks = S * (H // 2) * -(-ctx // 16)
-    n = min(8 * sms, max(2 * sms, -(-chunks // 256)))
-    g = min(H, 16)
-    acc = n * 2 * g * D * 4
-    return 65536 * 4 + -(-acc // 256) * 256 + n * 2 * g * 2 * 4
-
-
 def test_workspace_and_partition_sizes(lib):
-    # single pass: no workspace (one head cannot be grouped; an explicit
-    # partition never takes the balanced launch)
-    assert lib.decode_workspace_size(4, 1, 64, 100, 0) == 0
+    # single pass: no workspace
+    assert lib.decode_workspace_size(4, 4, 64, 100, 0) == 0
     assert lib.decode_workspace_size(4, 4, 64, 512, 512) == 0
-    # automatic partitioning with two or more heads also covers the balanced
-    # grouped-heads launch
-    assert lib.decode_workspace_size(4, 4, 64, 100, 0) == flat_bound(4, 4, 64, 100)
-    assert lib.decode_workspace_size(96, 32, 128, 2048, 0) >= flat_bound(96, 32, 128, 2048)
-    assert lib.decode_workspace_size(600, 32, 128, 2048, 0) > 0
     # explicit partitions: 65536 int32 arrival counters, acc [S,H,P,D] fp32
     # padded to 256 B, then (m, l) pairs
     S, H, D, ctx, P = 3, 5, 128, 1000, 256
@@ -152,19 +134,20 @@ def test_workspace_and_partition_sizes(lib):
     assert lib.decode_partition_size(96, 32, desc(32), 2048, 1024) == 1024
     assert lib.decode_partition_size(1, 1, desc(1), 30000, 0) == 128
     # Grouped heads (2 <= G <= 16) on a 16-bit cache, or on an fp8 cache with
-    # f16 rows and head_dim 128, with automatic partitioning and at most 512
-    # sequences: token ranges balanced per launch, reported as 0.
-    for args in [(96, 32, desc(8), 2048), (96, 32, desc(8, lib.PA_BF16), 4096),
-                 (96, 32, desc(2), 2048), (1, 32, desc(8), 32768), (256, 32, desc(8), 2048),
-                 (96, 32, desc(8, lib.PA_FP8_E4M3), 4096), (512, 16, desc(8, d=64, bs=8), 300)]:
-        assert lib.decode_partition_size(*args, 0) == 0, args
-    # Otherwise one CTA row per K/V head and fixed partitions: an explicit
-    # size; past 512 sequences 1024 tokens (halved while the grid has fewer
-    # CTAs than SMs).
-    assert lib.decode_partition_size(96, 32, desc(8), 2048, 512) == 512
-    assert lib.decode_partition_size(600, 32, desc(8), 2048, 0) == 1024
+    # f16 rows and head_dim 128: the tensor-core kernel, one CTA row per K/V
+    # head. Batches of up to 128 sequences (handed out longest first):
+    # 2048-token partitions halved while the grid has fewer than 2 CTAs per
+    # SM; larger batches: 1024 halved while it has fewer CTAs than SMs.
     # fp8 without grouping, with bf16 rows or head_dim 64 stays on one CTA
     # row per query head.
+    assert lib.decode_partition_size(96, 32, desc(8), 2048, 0) == 2048  # single pass
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_BF16), 4096, 0) == 2048
+    assert lib.decode_partition_size(96, 32, desc(2), 2048, 0) == 1024  # 192 x 2 CTAs
+    assert lib.decode_partition_size(96, 32, desc(8), 1000, 0) == 1024  # single pass
+    assert lib.decode_partition_size(1, 32, desc(8), 32768, 0) == 512  # 8 x 64 CTAs
+    assert lib.decode_partition_size(1, 32, desc(8), 4096, 0) == 256  # 8 x 16 CTAs
+    assert lib.decode_partition_size(256, 32, desc(8), 2048, 0) == 1024  # natural order
+    assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3), 4096, 0) == 2048
     assert lib.decode_partition_size(96, 32, desc(32, lib.PA_FP8_E4M3), 2048, 0) == 2048
     assert lib.decode_partition_size(96, 32, desc(8, lib.PA_FP8_E4M3, io=lib.PA_BF16),
                                       2048, 0) == 2048

@@ -1,12 +1,12 @@
-"""decode_flat_kernel: grouped query heads with automatic partitioning, every
-CTA streaming an equal share of the launch's chunks across unit boundaries.
+"""Grouped query heads on decode_group_kernel (one CTA per K/V head and
+partition): shapes at the edges of its launch logic, against the fp64 oracle.
 
-Against the fp64 oracle: many tiny units per CTA (several windows of
-segments), fewer chunks than CTAs, one unit cut into hundreds of pieces,
-the 512-sequence limit and the fall-back just past it, a workspace too small
-for the balanced launch (the fixed-partition kernel takes over), repeated
-calls and CUDA-graph replays (bit-identical outputs, counters back at zero),
-and a bad block id inside a unit that spans several CTAs.
+Many tiny units (512 sequences x 32 K/V heads), tiny inputs with empty
+sequences, one long unit split into many partitions, batches on both sides of
+the longest-first ordering limit, a workspace too small (refused before any
+launch), repeated calls and CUDA-graph replays (bit-identical outputs,
+arrival counters back at zero), a bad block id inside a split sequence, and
+the benchmark's grouped layers at full size.
 """
 import numpy as np
 import pytest
@@ -40,16 +40,9 @@ def check(out, ref, what=""):
     assert mx <= TOL, f"{what}: max err {mx:.3e} at {worst}, mean {mean:.3e}"
 
 
-def test_partition_size_reports_balanced_launch():
-    desc = pk.CacheDesc(1000, 16, 8, 128, pk.PA_F16, pk.PA_F16)
-    assert pk.decode_partition_size(96, 32, desc, 2048, 0) == 0
-    assert pk.decode_partition_size(96, 32, desc, 2048, 512) == 512
-    assert pk.decode_partition_size(513, 32, desc, 2048, 0) > 0  # past the sequence limit
-
-
-def test_many_tiny_units_span_several_windows():
-    """512 sequences x 32 K/V heads of 1-20 tokens: each CTA's range holds
-    dozens of units, more than one window of segments."""
+def test_many_tiny_units():
+    """512 sequences x 32 K/V heads of 1-20 tokens: 16,384 single-chunk
+    units in natural order."""
     rng = np.random.default_rng(70)
     ctxs = rng.integers(1, 21, size=512).tolist()
     c = gqa_case(rng, ctxs, 2, 32, 64, 8)
@@ -58,7 +51,7 @@ def test_many_tiny_units_span_several_windows():
     check(out, orc(c), "tiny units")
 
 
-def test_fewer_chunks_than_ctas():
+def test_tiny_inputs_with_empty_sequences():
     rng = np.random.default_rng(71)
     for ctxs in ([5], [1, 2], [17, 0, 3]):
         c = gqa_case(rng, ctxs, 4, 2, 128, 16)
@@ -68,9 +61,9 @@ def test_fewer_chunks_than_ctas():
 
 
 @pytest.mark.parametrize("G", [4, 16])
-def test_one_unit_in_hundreds_of_pieces(G):
-    """A single 33000-token unit: every CTA holds a piece of it; the last to
-    finish merges them all."""
+def test_one_long_unit_in_many_partitions(G):
+    """A single 33000-token unit: the automatic partition splits it into
+    many CTAs; the last to finish merges them all."""
     rng = np.random.default_rng(72 + G)
     c = gqa_case(rng, [33000], G, 1, 128, 16)
     out, err = decode_case(c, out_dtype=torch.float32)
@@ -78,33 +71,22 @@ def test_one_unit_in_hundreds_of_pieces(G):
     check(out, orc(c), "one long unit")
 
 
-@pytest.mark.parametrize("S", [512, 513])
-def test_sequence_limit_and_fallback(S):
-    """512 sequences take the balanced launch, 513 the fixed-partition
-    kernel; both match the oracle."""
+@pytest.mark.parametrize("S", [128, 129, 513])
+def test_large_batches(S):
+    """128 sequences are handed out longest first, 129 and 513 in natural
+    order; all match the oracle, fused and separate."""
     st = wl.llama_layer(seed=73, num_seqs=S, ctx_range=(1, 300), num_blocks=S * 20 + 64,
                         num_heads=16, num_kv_heads=4, head_dim=64)
-    desc = pk.CacheDesc(st.num_blocks, 16, 4, 64, pk.PA_F16, pk.PA_F16)
-    assert (pk.decode_partition_size(S, 16, desc, st.max_context_len, 0) == 0) == (S <= 512)
     for runner in (run_step, run_step_fused):
         outs, d, err = runner(st)
         assert err == 0
         check_outputs_and_pools(st, outs, d, [0])
 
 
-def grid_workspace_bound(S, H, D, mcl):
-    """Bytes the fixed-partition kernels need for any automatic partition
-    (128 tokens or longer): 256 KiB of counters, then the partial sums and
-    the (max, sum) pairs of S * H units of ceil(mcl / 128) partitions."""
-    parts = -(-mcl // 128)
-    acc = S * H * parts * D * 4
-    return 256 * 1024 + -(-acc // 256) * 256 + S * H * parts * 2 * 4
-
-
-def test_small_workspace_falls_back_to_fixed_partitions():
-    """A workspace that holds the fixed-partition kernel's partials but not
-    the balanced launch's pieces: the call still succeeds and matches; with
-    far too little, the call is refused before any launch."""
+def test_workspace_too_small_is_refused():
+    """A split decode with a workspace smaller than
+    pa_decode_workspace_size is refused before any launch; with the full
+    size it matches the oracle."""
     rng = np.random.default_rng(74)
     c = gqa_case(rng, [3000, 40, 2600, 900], 8, 2, 128, 16)
     dt = torch.float16
@@ -113,19 +95,15 @@ def test_small_workspace_falls_back_to_fixed_partitions():
     bt, ctx = torch.from_numpy(c["bt"]).cuda(), torch.from_numpy(c["ctx"]).cuda()
     S, H, D = q.shape
     mcl = int(c["ctx"].max())
-    ref = orc(c)
-    grid_bytes = grid_workspace_bound(S, H, D, mcl)
-    assert grid_bytes < pk.decode_workspace_size(S, H, D, mcl)
-    for nbytes in (pk.decode_workspace_size(S, H, D, mcl), grid_bytes):
-        ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
-        out = torch.empty_like(q)
-        pk.decode(out, q, kc, vc, bt, ctx, mcl, float(c["scale"]), workspace=ws)
-        torch.cuda.synchronize()
-        check(out, ref, f"workspace of {nbytes} bytes")
+    out = torch.empty_like(q)
+    pk.decode(out, q, kc, vc, bt, ctx, mcl, float(c["scale"]),
+              workspace=pk.alloc_workspace(S, H, D, mcl))
+    torch.cuda.synchronize()
+    check(out, orc(c), "full workspace")
     small = torch.zeros(64, dtype=torch.uint8, device="cuda")
     with pytest.raises(pk.PagedKVError) as e:
         pk.decode(torch.empty_like(q), q, kc, vc, bt, ctx, mcl, float(c["scale"]),
-                  workspace=small)
+                  partition_size=256, workspace=small)
     assert e.value.status == pk.PA_ERR_WORKSPACE
 
 
@@ -161,8 +139,8 @@ def test_repeated_calls_and_graph_replays_are_bit_identical():
 
 
 def test_bad_block_id_inside_a_split_unit():
-    """A bad id in a long unit (cut across CTAs) makes that sequence NaN and
-    sets the flag; the other sequences are unaffected."""
+    """A bad id in a long unit (split across CTAs) makes that sequence NaN
+    and sets the flag; the other sequences are unaffected."""
     rng = np.random.default_rng(76)
     c = gqa_case(rng, [20000, 300, 150], 8, 1, 128, 16)
     c["bt"][0, 700] = c["kpool"].shape[0] + 3
