@@ -766,19 +766,28 @@ __device__ __forceinline__ void merge_if_last(const DecodeParams &p, int s, int 
 constexpr int kRankMaxSeqs = 128;
 
 // Every thread of the CTA calls it (two barriers): the sequence of rank y.
-// ctx_buf: kRankMaxSeqs ints of shared memory; out: one shared int.
+// ctx_buf: kRankMaxSeqs ints of 16-byte aligned shared memory; out: one
+// shared int. Sequence k gets the key (min(max(len, 0), 2^24 - 1) << 7) |
+// (127 - k): keys are distinct, larger for longer sequences and, among equal
+// (or clamped) lengths, for smaller indices; the rank of k is the number of
+// larger keys, a permutation of 0 .. S-1 whatever the lengths. Keys are
+// padded with -1 (below every key) to a multiple of 4 and compared four at
+// a time.
 __device__ __forceinline__ int ranked_sequence(const int32_t *context_lens, int S, int y,
                                                int tid, int nthreads, int32_t *ctx_buf, int *out)
 {
-    for (int k = tid; k < S; k += nthreads)
-        ctx_buf[k] = context_lens[k];
+    const int S4 = (S + 3) >> 2;
+    for (int k = tid; k < 4 * S4; k += nthreads)
+        ctx_buf[k] = k < S ? (min(max(context_lens[k], 0), (1 << 24) - 1) << 7) | (127 - k) : -1;
     __syncthreads();
+    const int4 *c4 = reinterpret_cast<const int4 *>(ctx_buf);
     for (int k = tid; k < S; k += nthreads) {
         const int c = ctx_buf[k];
         int r = 0;
-        for (int j = 0; j < S; ++j) {
-            const int cj = ctx_buf[j];
-            r += (cj > c) | ((cj == c) & (j < k));
+#pragma unroll 4
+        for (int j = 0; j < S4; ++j) {
+            const int4 v = c4[j];
+            r += (v.x > c) + (v.y > c) + (v.z > c) + (v.w > c);
         }
         if (r == y)
             *out = k; // ranks are a permutation: exactly one writer
@@ -821,6 +830,7 @@ template <typename T, int D, int BS, int NW, int NS> struct SplitCfg {
     static constexpr int kMergeBytes = NW * (D + 2) * 4;
     static constexpr int kRankBytes = kRankMaxSeqs * 4;
     static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kMergeBytes + kRankBytes;
+    static_assert((kRingsBytes + kBarBytes + kMergeBytes) % 16 == 0, "ranking buffer alignment");
     static size_t smem_bytes(int partition)
     {
         return kFixedBytes + ((partition / BS) * 4 + 15) / 16 * 16;

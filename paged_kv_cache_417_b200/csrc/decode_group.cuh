@@ -26,8 +26,11 @@
 // (fp8, 16-bit at D = 64) and 4 when it is two (2-way at D = 128).
 //
 // Math per 16-token step in one warp, on tensor-core tiles (mma.sync
-// m16n8k16, f16/bf16 operands, fp32 accumulation); the G query heads are the
-// M rows, padded to 16 with zeros (G <= 8 uses rows 0-7 only):
+// m16n8k16, f16/bf16 operands, fp32 accumulation), in one of two
+// orientations. G <= 8 (GroupWarpT): S^T = K Q^T and O^T += V^T P^T, with
+// tokens and d on the 16-row side of the tiles and the heads as their 8
+// columns (described at GroupWarpT). G > 8 (GroupWarp), described here: the
+// G query heads are the M rows, padded to 16 with zeros:
 //   S = Q K^T      2 column tiles of 8 tokens x D/16 k-steps, K tiles by
 //                  ldmatrix straight from the swizzled stage. fp8: a tile
 //                  register holds 4 consecutive codes of one token; they are
@@ -89,8 +92,16 @@ template <typename T, int D> struct GroupGeom {
     static constexpr int kChunk = kFp8 ? 32 : 16;    // tokens per stage
     static constexpr int kHalf = kChunk * kRow;      // the K (or V) codes of a stage
     static constexpr int kStage = 2 * kHalf;
-    static constexpr int kMergeStride = D + 2;       // a row's (O, m, l) in a merge area
+    static constexpr int kMergeStride = D + 4;       // a row's (O, m, l) in a merge area (16-byte rows)
     static_assert(kHalf % 1024 == 0, "swizzle atoms");
+
+    // Piece p (16 bytes) of row t sits in unit t*kUnits + p/8 at position
+    // (p % 8) ^ ((t*kUnits + p/8) % 8) of a swizzled stage.
+    static __device__ __forceinline__ int piece_off(int t, int piece)
+    {
+        const int unit = t * kUnits + (piece >> 3);
+        return unit * 128 + (((piece & 7) ^ (unit & 7)) << 4);
+    }
 };
 
 template <typename T, int D, int BS, int NW, int NS> struct GroupCfg : GroupGeom<T, D> {
@@ -99,14 +110,18 @@ template <typename T, int D, int BS, int NW, int NS> struct GroupCfg : GroupGeom
     static constexpr int kRing = NS * Geo::kStage;         // one warp's stages
     static constexpr int kSeg = BS < 16 ? BS : 16;         // rows per TMA box
     static constexpr int kRingsBytes = NW * kRing;
-    static constexpr int kBarBytes = NW * NS * 8;
+    static constexpr int kBarBytes = (NW * NS * 8 + 15) / 16 * 16; // mbarriers, 16-byte padded
     // fp8 row scales: per warp, [stage][K | V][kChunk] floats.
     static constexpr int kScaleBytes = Geo::kFp8 ? NW * NS * 2 * Geo::kChunk * 4 : 0;
     static constexpr int kRankBytes = kRankMaxSeqs * 4; // context lengths for ranking
     static constexpr int kFixedBytes = kRingsBytes + kBarBytes + kScaleBytes + kRankBytes;
+    static_assert((kRingsBytes + kBarBytes + kScaleBytes) % 16 == 0, "ranking buffer alignment");
     // After its last chunk a warp of decode_group_kernel leaves (O, m, l) of
-    // its rows in its ring.
-    static_assert(kGroupMaxHeads * Geo::kMergeStride * 4 <= kRing, "merge area fits a ring");
+    // its rows in its ring; warp 0's ring then also holds, per row, the NW
+    // weights of the warps and the row's (M, L) (kMergeWeights).
+    static constexpr int kMergeWeights = kGroupMaxHeads * Geo::kMergeStride; // floats
+    static_assert((kMergeWeights + kGroupMaxHeads * (NW + 2)) * 4 <= kRing,
+                  "merge area fits a ring");
     static_assert((kSeg * Geo::kRow) % 1024 == 0, "swizzle atoms");
     static_assert(Geo::kChunk % kSeg == 0 && Geo::kChunk % 16 == 0, "chunk geometry");
     // 1 KiB of slack to align the rings to 1024 bytes.
@@ -153,7 +168,7 @@ template <typename T, int D, bool TWO> struct GroupWarp {
     static constexpr bool kFp8 = Geo::kFp8;
     static constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     using QT = typename std::conditional<kFp8, __half, T>::type; // operand / row type
-    static constexpr int CH = Geo::kChunk, ROW = Geo::kRow, U = Geo::kUnits;
+    static constexpr int CH = Geo::kChunk, ROW = Geo::kRow;
     static constexpr int KT = D / 16; // k-steps of q.k = pairs of 8-wide d tiles of O
     static constexpr int MS = Geo::kMergeStride;
     static constexpr unsigned FULL = 0xffffffffu;
@@ -174,12 +189,9 @@ template <typename T, int D, bool TWO> struct GroupWarp {
     float m0, m1, l0, l1;
     float vref; // fp8: largest V scale so far (R), floored at FLT_MIN
 
-    // Piece p (16 bytes) of row t sits in unit t*U + p/8 at position
-    // (p % 8) ^ ((t*U + p/8) % 8) of a swizzled stage.
     static __device__ __forceinline__ int piece_off(int t, int piece)
     {
-        const int unit = t * U + (piece >> 3);
-        return unit * 128 + (((piece & 7) ^ (unit & 7)) << 4);
+        return Geo::piece_off(t, piece);
     }
 
     // O tile j covers 8 d: 16-bit d = 8j + q2 (+1); fp8 d = 16(j/2) + 4q +
@@ -486,6 +498,298 @@ template <typename T, int D, bool TWO> struct GroupWarp {
     }
 };
 
+// One warp's share of a group of G <= 8 query heads in the transposed
+// orientation: S^T = K Q^T and O^T += V^T P^T. The 16 tokens of a step (for
+// S^T) and 16 values of d (for O^T) fill the 16 rows of each m16n8k16 tile
+// and the heads its 8 columns, so every tile is fully used; GroupWarp's
+// orientation (heads as rows) leaves rows 8-15 of every tile empty when
+// G <= 8 and needs twice the tiles and accumulators. Same interface and
+// merge-area output as GroupWarp. Heads >= G are zero query columns (their
+// outputs are never stored).
+//
+// Fragment coordinates: g = lane / 4, q = lane % 4. S^T: rows = tokens g,
+// g + 8, columns = heads 2q, 2q + 1. Q^T (B operand): k = d pair, n = head
+// g. P^T (B operand): k = tokens 2q, 2q + 1 (and + 8), n = head g, made from
+// the S^T fragments by one 8x8 register transpose (movmatrix) per 8 tokens.
+// O^T tile j: rows = d (drow), columns = heads 2q, 2q + 1.
+// K and V tiles both come from ldmatrix with rows (tokens) 0-7 / 8-15 /
+// 0-7 / 8-15 at pieces c / c / c+1 / c+1: non-transposed K is exactly the A
+// fragment of one k-step; transposed 16-bit V gives the A fragment of O^T
+// tile j in register order 0, 2, 1, 3. fp8: each register holds 4 codes of
+// one token; widened to f16 pairs (codes 0-1, 2-3) they are K's A fragment
+// with the k order d = 4q, 4q+1 | 4q+2, 4q+3 (the query is loaded in the
+// same order), and, transposed in registers, V's A fragment whose rows are
+// the d values {0,1,4,5,8,9,12,13} / {2,3,6,7,10,11,14,15} of each piece.
+template <typename T, int D> struct GroupWarpT {
+    using Geo = GroupGeom<T, D>;
+    static constexpr bool kFp8 = Geo::kFp8;
+    static constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    using QT = typename std::conditional<kFp8, __half, T>::type; // operand / row type
+    static constexpr int CH = Geo::kChunk, ROW = Geo::kRow;
+    static constexpr int KT = D / 16; // 16-wide d pieces: k-steps of S^T, row tiles of O^T
+    static constexpr int MS = Geo::kMergeStride;
+    static constexpr unsigned FULL = 0xffffffffu;
+
+    int lane, g, q;
+    int rt, rc;          // ldmatrix row (token) and piece offset of this lane
+    uint32_t qb[KT][2];  // Q^T as the B operand of each k-step
+    float o[KT][4];      // O^T tiles
+    float ma, mb;        // running maxima of heads 2q, 2q + 1
+    float la, lb;        // this lane's tokens' share of their sums
+    float vref;          // fp8: largest V scale so far (R), floored at FLT_MIN
+
+    static __device__ __forceinline__ int piece_off(int t, int piece)
+    {
+        return Geo::piece_off(t, piece);
+    }
+
+    // d of row g (hi = 0) or g + 8 (hi = 1) of O^T tile j.
+    __device__ __forceinline__ int drow(int j, int hi) const
+    {
+        return kFp8 ? 16 * j + 4 * (g >> 1) + (g & 1) + 2 * hi : 16 * j + g + 8 * hi;
+    }
+
+    __device__ __forceinline__ void init(int lane_)
+    {
+        lane = lane_;
+        g = lane >> 2;
+        q = lane & 3;
+        rt = (lane & 7) + (((lane >> 3) & 1) << 3);
+        rc = lane >> 4;
+    }
+
+    // Head g's query row (row0 + g) as B fragments: 16-bit k-slots (2q, 2q+1)
+    // / (2q+8, 2q+9) hold d = 16kk + 2q (+1) / + 8 (+1); fp8: d = 16kk + 4q
+    // (+1) / + 2 (+1), matching the widened K codes. Heads >= G: zero.
+    __device__ __forceinline__ void load_q(const void *query, size_t row0, int G)
+    {
+        const uint32_t *qp = static_cast<const uint32_t *>(query); // element pairs
+        const size_t r = (row0 + g) * (D / 2);
+#pragma unroll
+        for (int kk = 0; kk < KT; ++kk) {
+            const int c0 = kFp8 ? 8 * kk + 2 * q : 8 * kk + q;
+            const int c1 = kFp8 ? c0 + 1 : c0 + 4;
+            qb[kk][0] = g < G ? qp[r + c0] : 0u;
+            qb[kk][1] = g < G ? qp[r + c1] : 0u;
+        }
+    }
+
+    __device__ __forceinline__ void reset()
+    {
+#pragma unroll
+        for (int j = 0; j < KT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o[j][e] = 0.f;
+        ma = mb = -INFINITY;
+        la = lb = 0.f;
+        vref = 1.17549435e-38f;
+    }
+
+    // S^T of tokens t0 .. t0 + 15, even and odd k-steps in separate
+    // accumulators (two shorter dependency chains).
+    __device__ __forceinline__ void scores(uint32_t kb, int t0, float (&sa)[4]) const
+    {
+        float sb[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            sa[e] = sb[e] = 0.f;
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int kp = 0; kp < KT / 2; ++kp) { // pieces 2kp, 2kp + 1
+                uint32_t r[4];
+                ldsm_x4(kb + piece_off(t0 + rt, 2 * kp + rc), r);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t a[4];
+                    e4m3x4_to_h2x2(r[2 * h], a[0], a[2]);     // tokens 0-7
+                    e4m3x4_to_h2x2(r[2 * h + 1], a[1], a[3]); // tokens 8-15
+                    mma_16816<false>(h ? sb : sa, a, qb[2 * kp + h][0], qb[2 * kp + h][1]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int kk = 0; kk < KT; ++kk) {
+                uint32_t a[4];
+                ldsm_x4(kb + piece_off(t0 + rt, 2 * kk + rc), a);
+                mma_16816<kBf16>(kk & 1 ? sb : sa, a, qb[kk][0], qb[kk][1]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            sa[e] += sb[e];
+    }
+
+    // One staged chunk (as GroupWarp::chunk): K codes at sk, V at sv, fp8 row
+    // scales at ksc / vsc, `rows` valid tokens, qs = scale * log2(e).
+    __device__ __forceinline__ void chunk(char *sk, char *sv, const float *ksc, const float *vsc,
+                                          int rows, float qs)
+    {
+        if (rows < CH) { // zero the V rows past the context
+            for (int k = rows * (ROW / 16) + lane; k < CH * (ROW / 16); k += 32)
+                reinterpret_cast<uint4 *>(sv)[k] = make_uint4(0u, 0u, 0u, 0u);
+            fence_proxy_async_smem(); // before the stage is refilled by a copy
+            __syncwarp();
+        }
+        const uint32_t kb = smem_addr(sk), vb = smem_addr(sv);
+#pragma unroll
+        for (int sub = 0; sub < CH / 16; ++sub) {
+            const int srows = rows - 16 * sub; // valid tokens of this step
+            if (srows <= 0)
+                break; // warp-uniform
+            const int t0 = 16 * sub;
+            float sa[4];
+            scores(kb, t0, sa);
+
+            // Online softmax (base 2) per head over the step's tokens: sa[0]
+            // / sa[1]: token t0 + g, heads 2q / 2q + 1; sa[2] / sa[3]: token
+            // t0 + g + 8. The 16 tokens of a head live in the 8 lanes of one q.
+            float k0 = qs, k1 = qs;
+            if constexpr (kFp8) {
+                k0 = ksc[t0 + g] * qs;
+                k1 = ksc[t0 + g + 8] * qs;
+            }
+            float x0 = sa[0] * k0, x1 = sa[1] * k0, x2 = sa[2] * k1, x3 = sa[3] * k1;
+            const bool partial = srows < 16; // warp-uniform
+            if (partial) {
+                if (g >= srows)
+                    x0 = x1 = -INFINITY;
+                if (g + 8 >= srows)
+                    x2 = x3 = -INFINITY;
+            }
+            float mxa = fmaxf(x0, x2), mxb = fmaxf(x1, x3);
+#pragma unroll
+            for (int sh = 4; sh < 32; sh <<= 1) {
+                mxa = fmaxf(mxa, __shfl_xor_sync(FULL, mxa, sh));
+                mxb = fmaxf(mxb, __shfl_xor_sync(FULL, mxb, sh));
+            }
+            const float na = fmaxf(ma, mxa), nb = fmaxf(mb, mxb); // finite: token t0 is valid
+            const float ca = exp2f(ma - na), cb = exp2f(mb - nb);
+            ma = na;
+            mb = nb;
+            float p0 = exp2f(x0 - na), p1 = exp2f(x1 - nb);
+            float p2 = exp2f(x2 - na), p3 = exp2f(x3 - nb);
+            la = fmaf(la, ca, p0 + p2);
+            lb = fmaf(lb, cb, p1 + p3);
+            float cr = 1.f; // fp8: R_old / R_new
+            if constexpr (kFp8) {
+                // Fold the V scales into P relative to R (tokens past the
+                // context get P' = 0 by selection).
+                float v0 = vsc[t0 + g], v1 = vsc[t0 + g + 8];
+                if (partial) { // stale scales past the context must not reach P'
+                    if (g >= srows)
+                        v0 = 0.f;
+                    if (g + 8 >= srows)
+                        v1 = 0.f;
+                }
+                float vmax = fmaxf(v0, v1);
+#pragma unroll
+                for (int sh = 4; sh < 32; sh <<= 1)
+                    vmax = fmaxf(vmax, __shfl_xor_sync(FULL, vmax, sh));
+                const float rn = fmaxf(vref, vmax);
+                cr = vref / rn;
+                vref = rn;
+                const float inv = 1.f / rn;
+                const float w0 = v0 * inv, w1 = v1 * inv;
+                p0 *= w0;
+                p1 *= w0;
+                p2 *= w1;
+                p3 *= w1;
+            }
+            if (__any_sync(FULL, ca != 1.f || cb != 1.f || cr != 1.f)) { // a max moved
+                const float fa = ca * cr, fb = cb * cr;
+#pragma unroll
+                for (int j = 0; j < KT; ++j) {
+                    o[j][0] *= fa;
+                    o[j][2] *= fa;
+                    o[j][1] *= fb;
+                    o[j][3] *= fb;
+                }
+            }
+
+            // P^T as the B operand: the S^T fragment pair of tokens g (and
+            // g + 8), heads 2q, 2q + 1, transposed in registers, is head g at
+            // tokens 2q, 2q + 1 (and + 8).
+            const uint32_t pb0 = movmatrix_trans(pack2<QT>(p0, p1));
+            const uint32_t pb1 = movmatrix_trans(pack2<QT>(p2, p3));
+            uint32_t pl0 = 0u, pl1 = 0u; // bf16: the remainder P - bf16(P)
+            if constexpr (kBf16) {
+                const float2 h01 = unpack_bf2(pack2<T>(p0, p1));
+                const float2 h23 = unpack_bf2(pack2<T>(p2, p3));
+                pl0 = movmatrix_trans(pack2<T>(p0 - h01.x, p1 - h01.y));
+                pl1 = movmatrix_trans(pack2<T>(p2 - h23.x, p3 - h23.y));
+            }
+
+            if constexpr (kFp8) {
+                // O^T += V^T P^T per piece: widen the codes of tokens 0-7 and
+                // 8-15 and transpose each 8x8 half in registers.
+#pragma unroll
+                for (int kp = 0; kp < KT / 2; ++kp) {
+                    uint32_t r[4];
+                    ldsm_x4(vb + piece_off(t0 + rt, 2 * kp + rc), r);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t w0l, w0h, w1l, w1h;
+                        e4m3x4_to_h2x2(r[2 * h], w0l, w0h);     // tokens 0-7
+                        e4m3x4_to_h2x2(r[2 * h + 1], w1l, w1h); // tokens 8-15
+                        const uint32_t a[4] = {movmatrix_trans(w0l), movmatrix_trans(w0h),
+                                               movmatrix_trans(w1l), movmatrix_trans(w1h)};
+                        mma_16816<false>(o[2 * kp + h], a, pb0, pb1);
+                    }
+                }
+            } else {
+                // O^T += V^T P^T, one 16-row tile of d per transposed ldmatrix.
+#pragma unroll
+                for (int j = 0; j < KT; ++j) {
+                    uint32_t r[4];
+                    ldsm_x4_trans(vb + piece_off(t0 + rt, 2 * j + rc), r);
+                    const uint32_t a[4] = {r[0], r[2], r[1], r[3]};
+                    mma_16816<kBf16>(o[j], a, pb0, pb1);
+                    if constexpr (kBf16)
+                        mma_16816<kBf16>(o[j], a, pl0, pl1);
+                }
+            }
+        }
+    }
+
+    // Sums over each head's 8 lanes, then this warp's (O, m, l) of heads < G
+    // into mw (row stride MS; fp8: O back in the scale of the codes' values,
+    // times R).
+    __device__ __forceinline__ void store(float *mw, int G)
+    {
+#pragma unroll
+        for (int sh = 4; sh < 32; sh <<= 1) {
+            la += __shfl_xor_sync(FULL, la, sh);
+            lb += __shfl_xor_sync(FULL, lb, sh);
+        }
+        const float oscale = kFp8 ? vref : 1.f;
+        const int ha = 2 * q, hb = ha + 1;
+        __syncwarp();
+        if (ha < G) {
+#pragma unroll
+            for (int j = 0; j < KT; ++j) {
+                mw[ha * MS + drow(j, 0)] = o[j][0] * oscale;
+                mw[ha * MS + drow(j, 1)] = o[j][2] * oscale;
+            }
+            if (g == 0) {
+                mw[ha * MS + D] = ma;
+                mw[ha * MS + D + 1] = la;
+            }
+        }
+        if (hb < G) {
+#pragma unroll
+            for (int j = 0; j < KT; ++j) {
+                mw[hb * MS + drow(j, 0)] = o[j][1] * oscale;
+                mw[hb * MS + drow(j, 1)] = o[j][3] * oscale;
+            }
+            if (g == 0) {
+                mw[hb * MS + D] = mb;
+                mw[hb * MS + D + 1] = lb;
+            }
+        }
+    }
+};
+
 // The new token's K and V rows for the fused append (pa_write_kv_decode),
 // one (sequence, K/V head) row per warp: lanes [0, RV) hold 16 bytes of the
 // stored K row each, the next RV lanes the V row (fp8: 16 codes quantised
@@ -562,7 +866,9 @@ __global__ void __launch_bounds__(NW * 32)
     decode_group_kernel(const __grid_constant__ GroupParams gp)
 {
     using Cfg = GroupCfg<T, D, BS, NW, NS>;
-    using Wp = GroupWarp<T, D, TWO>;
+    static_assert(kGroupMaxHeads * D <= kMergeOutPerThread * NW * 32, "merge_if_last capacity");
+    // G > 8: heads as tile rows; G <= 8: the transposed orientation.
+    using Wp = typename std::conditional<TWO, GroupWarp<T, D, true>, GroupWarpT<T, D>>::type;
     constexpr bool kFp8 = Cfg::kFp8;
     constexpr int CH = Cfg::kChunk, SEG = Cfg::kSeg, ROW = Cfg::kRow;
     constexpr int MS = Cfg::kMergeStride;
@@ -733,7 +1039,10 @@ __global__ void __launch_bounds__(NW * 32)
             atomicOr(&cta_flags, 1);
     }
 
-    // This warp's (O, m, l) into its ring, then the warps merged.
+    // This warp's (O, m, l) into its ring, then the warps merged in two
+    // passes: one thread per query row turns the NW (m, l) pairs into
+    // weights 2^(m_w - M) (divided by L = sum_w l_w 2^(m_w - M) for a single
+    // pass), then every thread sums four columns of a row at a time.
     __syncwarp();
     w.store(reinterpret_cast<float *>(ring), G);
     __syncthreads();
@@ -741,34 +1050,66 @@ __global__ void __launch_bounds__(NW * 32)
     const bool failed = cta_flags != 0;
     if (tid == 0 && (cta_flags & 1))
         report(p.dev_err, PA_DEVERR_BLOCK_ID);
-    for (int idx = tid; idx < G * D; idx += NW * 32) {
-        const int g = idx / D, d = idx - g * D;
-        float M = -INFINITY;
+    constexpr int WS = NW + 2; // per row: NW weights, M, L
+    float *wts = reinterpret_cast<float *>(rings) + Cfg::kMergeWeights;
+    if (tid < G) {
+        const int g = tid;
+        float mw[NW], M = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < NW; ++w2) {
+            mw[w2] = reinterpret_cast<const float *>(rings + w2 * Cfg::kRing)[g * MS + D];
+            M = fmaxf(M, mw[w2]);
+        }
+        float L = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < NW; ++w2) {
+            // A warp without tokens has m = -inf and weight 0; so has every
+            // warp of an empty unit (M = -inf, output 0).
+            mw[w2] = M == -INFINITY ? 0.f : exp2f(mw[w2] - M);
+            L = fmaf(reinterpret_cast<const float *>(rings + w2 * Cfg::kRing)[g * MS + D + 1],
+                     mw[w2], L);
+        }
+        const bool normalise = u.num_parts == 1 && L > 0.f;
 #pragma unroll
         for (int w2 = 0; w2 < NW; ++w2)
-            M = fmaxf(M, reinterpret_cast<const float *>(rings + w2 * Cfg::kRing)[g * MS + D]);
-        float L = 0.f, O = 0.f;
-        if (M != -INFINITY) {
+            wts[g * WS + w2] = normalise ? mw[w2] / L : mw[w2];
+        if (u.num_parts > 1) {
+            const size_t unit = ((size_t)s * H + kvh * G + g) * p.num_parts + part;
+            p.ws_ml[unit * 2] = failed ? 0.f : M;
+            p.ws_ml[unit * 2 + 1] = failed ? 1.f : L;
+        }
+    }
+    __syncthreads();
+    constexpr int D4 = D / 4;
+    constexpr int kPasses = (kGroupMaxHeads * D4 + NW * 32 - 1) / (NW * 32);
+#pragma unroll
+    for (int k = 0; k < kPasses; ++k) {
+        const int idx = tid + k * NW * 32;
+        if (idx < G * D4) {
+            const int g = idx / D4, d = (idx - g * D4) * 4;
+            float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int w2 = 0; w2 < NW; ++w2) {
-                const float *mv =
-                    reinterpret_cast<const float *>(rings + w2 * Cfg::kRing) + g * MS;
-                const float f = exp2f(mv[D] - M);
-                L = fmaf(mv[D + 1], f, L);
-                O = fmaf(mv[d], f, O);
+                const float f = wts[g * WS + w2];
+                const float4 v = *reinterpret_cast<const float4 *>(
+                    reinterpret_cast<const float *>(rings + w2 * Cfg::kRing) + g * MS + d);
+                o4.x = fmaf(v.x, f, o4.x);
+                o4.y = fmaf(v.y, f, o4.y);
+                o4.z = fmaf(v.z, f, o4.z);
+                o4.w = fmaf(v.w, f, o4.w);
             }
-        }
-        if (failed)
-            O = NAN;
-        const int h = kvh * G + g;
-        if (u.num_parts == 1) {
-            store_out(p.out, p.out_dtype, ((size_t)s * H + h) * D + d, L > 0.f ? O / L : O);
-        } else {
-            const size_t unit = ((size_t)s * H + h) * p.num_parts + part;
-            p.ws_acc[unit * D + d] = O;
-            if (d == 0) {
-                p.ws_ml[unit * 2] = failed ? 0.f : M;
-                p.ws_ml[unit * 2 + 1] = failed ? 1.f : L;
+            if (failed)
+                o4 = make_float4(NAN, NAN, NAN, NAN);
+            const int h = kvh * G + g;
+            if (u.num_parts == 1) {
+                const size_t o = ((size_t)s * H + h) * D + d;
+                store_out(p.out, p.out_dtype, o, o4.x);
+                store_out(p.out, p.out_dtype, o + 1, o4.y);
+                store_out(p.out, p.out_dtype, o + 2, o4.z);
+                store_out(p.out, p.out_dtype, o + 3, o4.w);
+            } else {
+                const size_t unit = ((size_t)s * H + h) * p.num_parts + part;
+                *reinterpret_cast<float4 *>(p.ws_acc + unit * D + d) = o4;
             }
         }
     }

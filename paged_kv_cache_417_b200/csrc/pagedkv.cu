@@ -42,8 +42,11 @@ constexpr int kSplitStages = PA_SPLIT_STAGES;
 #ifndef PA_GROUP_WARPS
 #define PA_GROUP_WARPS 4
 #endif
+#ifndef PA_GROUP_STAGES
+#define PA_GROUP_STAGES 2
+#endif
 constexpr int kGroupWarps = PA_GROUP_WARPS;
-constexpr int kGroupStages = 2;
+constexpr int kGroupStages = PA_GROUP_STAGES;
 constexpr int kTargetCtasPerSm = 12; // ~4 waves of 3 resident CTAs
 constexpr int kMinAutoPartition = 128;
 constexpr int kAutoPartition = 2048;
