@@ -42,11 +42,11 @@
 //                  a row live in one quad of lanes (2 shuffles per max);
 //   O += P V       P goes from the S fragments into the A operand without
 //                  leaving registers. 16-bit V tiles by ldmatrix.trans. fp8
-//                  V: ldmatrix cannot transpose bytes, so each 8x8 tile of
-//                  widened codes is transposed in registers (movmatrix); the
-//                  d columns then come out as {0,1,4,5,8,9,12,13} and
-//                  {2,3,6,7,10,11,14,15} of each 16, i.e. lane quad q holds
-//                  d = 16c + 4q .. 4q+3 of piece c. The token's V scale is
+//                  V: ldmatrix.trans on code pairs gives a lane tokens 2q,
+//                  2q+1 at codes d = 2g, 2g+1 of a piece; one byte permute
+//                  and the widening make the B fragments of two column
+//                  tiles, d even and d odd (tile 2c + o: column n is d =
+//                  16c + 2n + o). The token's V scale is
 //                  folded into P relative to the largest V scale met so far
 //                  (R): P' = p * s_v / R <= 1, so an f16 P' keeps its
 //                  precision however small the scales; O is rescaled when R
@@ -179,10 +179,9 @@ template <typename T, int D, bool TWO> struct GroupWarp {
     // ldmatrix row addresses (rows within a 16-token step). 16-bit K
     // (non-transposed, B of S = Q K^T): lanes 0-7 / 8-15 / 16-23 / 24-31
     // give token rows 0-7 / 0-7 / 8-15 / 8-15 at pieces c / c+1 / c / c+1.
-    // 16-bit V (transposed, B of O = P V): rows 0-7 / 8-15 / 0-7 / 8-15 at
-    // pieces c / c / c+1 / c+1. fp8 K and V (non-transposed): rows 0-7 /
-    // 8-15 / 0-7 / 8-15 at pieces c / c / c+1 / c+1, register = (token tile,
-    // piece).
+    // V (transposed, B of O = P V; fp8 on code pairs) and fp8 K
+    // (non-transposed): rows 0-7 / 8-15 / 0-7 / 8-15 at pieces c / c / c+1 /
+    // c+1, register = (token tile, piece).
     int kt, kc, vt, vc;
     uint32_t qa[KT][4]; // Q as the A operand, one 16x16 tile per k-step
     float o[2 * KT][4];
@@ -194,11 +193,27 @@ template <typename T, int D, bool TWO> struct GroupWarp {
         return Geo::piece_off(t, piece);
     }
 
-    // O tile j covers 8 d: 16-bit d = 8j + q2 (+1); fp8 d = 16(j/2) + 4q +
-    // 2(j%2) (+1). Elements 0, 1: row g0; 2, 3: row g1.
-    __device__ __forceinline__ int dcol(int j) const
+    // O tile j covers 8 d. 16-bit: d = 8j + q2 (+1 for the second
+    // element). fp8, j = 2c + o: d = 16c + 2*q2 + o (+2 for the second), so
+    // tiles 2c and 2c + 1 together hold d = 16c + 2*q2 .. 16c + 2*q2 + 3.
+    // Elements 0, 1: row g0; 2, 3: row g1.
+    __device__ __forceinline__ void store_row(float *row, int e, float scale) const
     {
-        return kFp8 ? 16 * (j >> 1) + 4 * q + 2 * (j & 1) : 8 * j + q2;
+#pragma unroll
+        for (int j = 0; j < 2 * KT; j += 2) {
+            if constexpr (kFp8) {
+                const int d = 8 * j + 2 * q2; // 16c + 2*q2 with c = j / 2
+                *reinterpret_cast<float2 *>(row + d) =
+                    make_float2(o[j][e] * scale, o[j + 1][e] * scale);
+                *reinterpret_cast<float2 *>(row + d + 2) =
+                    make_float2(o[j][e + 1] * scale, o[j + 1][e + 1] * scale);
+            } else {
+                *reinterpret_cast<float2 *>(row + 8 * j + q2) =
+                    make_float2(o[j][e] * scale, o[j][e + 1] * scale);
+                *reinterpret_cast<float2 *>(row + 8 * j + 8 + q2) =
+                    make_float2(o[j + 1][e] * scale, o[j + 1][e + 1] * scale);
+            }
+        }
     }
 
     __device__ __forceinline__ void init(int lane_)
@@ -424,25 +439,22 @@ template <typename T, int D, bool TWO> struct GroupWarp {
             }
 
             if constexpr (kFp8) {
-                // O += P V: per pair of pieces, widen the codes and transpose
-                // each 8x8 half-tile in registers. r[0] / r[1]: token tiles
-                // 0 / 1 of piece 2kp, r[2] / r[3]: of piece 2kp + 1.
+                // O += P V per pair of pieces: r[2h] / r[2h + 1] hold tokens
+                // 2q, 2q + 1 (of 0-7 / 8-15) at codes d = 2g, 2g + 1 of piece
+                // c; reordered to (d 2g: both tokens | d 2g + 1: both) and
+                // widened, they are b0 / b1 of the even and odd d tiles.
 #pragma unroll
                 for (int kp = 0; kp < KT / 2; ++kp) {
                     uint32_t r[4];
-                    ldsm_x4(vb + piece_off(t0 + vt, 2 * kp + vc), r);
+                    ldsm_x4_trans(vb + piece_off(t0 + vt, 2 * kp + vc), r);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int c = 2 * kp + h; // piece: d = 16c .. 16c + 15
-                        uint32_t w0l, w0h, w1l, w1h;
-                        e4m3x4_to_h2x2(r[2 * h], w0l, w0h);
-                        e4m3x4_to_h2x2(r[2 * h + 1], w1l, w1h);
-                        const uint32_t lo0 = movmatrix_trans(w0l);
-                        const uint32_t lo1 = movmatrix_trans(w1l);
-                        const uint32_t hi0 = movmatrix_trans(w0h);
-                        const uint32_t hi1 = movmatrix_trans(w1h);
-                        mma_16816<false>(o[2 * c], pa, lo0, lo1);
-                        mma_16816<false>(o[2 * c + 1], pa, hi0, hi1);
+                        uint32_t e0, o0, e1, o1;
+                        e4m3x4_to_h2x2(__byte_perm(r[2 * h], 0u, 0x3120u), e0, o0);
+                        e4m3x4_to_h2x2(__byte_perm(r[2 * h + 1], 0u, 0x3120u), e1, o1);
+                        mma_16816<false>(o[2 * c], pa, e0, e1);
+                        mma_16816<false>(o[2 * c + 1], pa, o0, o1);
                     }
                 }
             } else {
@@ -474,10 +486,7 @@ template <typename T, int D, bool TWO> struct GroupWarp {
         const float oscale = kFp8 ? vref : 1.f;
         __syncwarp();
         if (g0 < G) {
-#pragma unroll
-            for (int j = 0; j < 2 * KT; ++j)
-                *reinterpret_cast<float2 *>(mw + g0 * MS + dcol(j)) =
-                    make_float2(o[j][0] * oscale, o[j][1] * oscale);
+            store_row(mw + g0 * MS, 0, oscale);
             if ((lane & 3) == 0) {
                 mw[g0 * MS + D] = m0;
                 mw[g0 * MS + D + 1] = l0;
@@ -485,10 +494,7 @@ template <typename T, int D, bool TWO> struct GroupWarp {
         }
         if constexpr (TWO) {
             if (g1 < G) {
-#pragma unroll
-                for (int j = 0; j < 2 * KT; ++j)
-                    *reinterpret_cast<float2 *>(mw + g1 * MS + dcol(j)) =
-                        make_float2(o[j][2] * oscale, o[j][3] * oscale);
+                store_row(mw + g1 * MS, 2, oscale);
                 if ((lane & 3) == 0) {
                     mw[g1 * MS + D] = m1;
                     mw[g1 * MS + D + 1] = l1;
@@ -518,8 +524,8 @@ template <typename T, int D, bool TWO> struct GroupWarp {
 // tile j in register order 0, 2, 1, 3. fp8: each register holds 4 codes of
 // one token; widened to f16 pairs (codes 0-1, 2-3) they are K's A fragment
 // with the k order d = 4q, 4q+1 | 4q+2, 4q+3 (the query is loaded in the
-// same order), and, transposed in registers, V's A fragment whose rows are
-// the d values {0,1,4,5,8,9,12,13} / {2,3,6,7,10,11,14,15} of each piece.
+// same order). fp8 V comes through transposed ldmatrix on code pairs (see
+// chunk); the rows of O^T tile j are then d = 16j + 2g and 16j + 2g + 1.
 template <typename T, int D> struct GroupWarpT {
     using Geo = GroupGeom<T, D>;
     static constexpr bool kFp8 = Geo::kFp8;
@@ -546,7 +552,7 @@ template <typename T, int D> struct GroupWarpT {
     // d of row g (hi = 0) or g + 8 (hi = 1) of O^T tile j.
     __device__ __forceinline__ int drow(int j, int hi) const
     {
-        return kFp8 ? 16 * j + 4 * (g >> 1) + (g & 1) + 2 * hi : 16 * j + g + 8 * hi;
+        return kFp8 ? 16 * j + 2 * g + hi : 16 * j + g + 8 * hi;
     }
 
     __device__ __forceinline__ void init(int lane_)
@@ -721,19 +727,20 @@ template <typename T, int D> struct GroupWarpT {
             }
 
             if constexpr (kFp8) {
-                // O^T += V^T P^T per piece: widen the codes of tokens 0-7 and
-                // 8-15 and transpose each 8x8 half in registers.
+                // O^T += V^T P^T per piece. Transposed ldmatrix on code
+                // pairs: a lane gets tokens 2q, 2q + 1 at codes d = 2g, 2g + 1
+                // of the piece; reordered to (d 2g: both tokens, d 2g + 1:
+                // both tokens) and widened, these are the A fragment rows of
+                // d = 2g (rows 0-7) and 2g + 1 (rows 8-15).
 #pragma unroll
                 for (int kp = 0; kp < KT / 2; ++kp) {
                     uint32_t r[4];
-                    ldsm_x4(vb + piece_off(t0 + rt, 2 * kp + rc), r);
+                    ldsm_x4_trans(vb + piece_off(t0 + rt, 2 * kp + rc), r);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        uint32_t w0l, w0h, w1l, w1h;
-                        e4m3x4_to_h2x2(r[2 * h], w0l, w0h);     // tokens 0-7
-                        e4m3x4_to_h2x2(r[2 * h + 1], w1l, w1h); // tokens 8-15
-                        const uint32_t a[4] = {movmatrix_trans(w0l), movmatrix_trans(w0h),
-                                               movmatrix_trans(w1l), movmatrix_trans(w1h)};
+                        uint32_t a[4];
+                        e4m3x4_to_h2x2(__byte_perm(r[2 * h], 0u, 0x3120u), a[0], a[1]);
+                        e4m3x4_to_h2x2(__byte_perm(r[2 * h + 1], 0u, 0x3120u), a[2], a[3]);
                         mma_16816<false>(o[2 * kp + h], a, pb0, pb1);
                     }
                 }
