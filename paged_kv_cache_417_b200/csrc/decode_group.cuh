@@ -187,6 +187,7 @@ template <typename T, int D, bool TWO> struct GroupWarp {
     float o[2 * KT][4];
     float m0, m1, l0, l1;
     float vref; // fp8: largest V scale so far (R), floored at FLT_MIN
+    float vinv; // fp8: 1 / vref
 
     static __device__ __forceinline__ int piece_off(int t, int piece)
     {
@@ -259,6 +260,7 @@ template <typename T, int D, bool TWO> struct GroupWarp {
         m0 = m1 = -INFINITY;
         l0 = l1 = 0.f;
         vref = 1.17549435e-38f;
+        vinv = 1.f / vref;
     }
 
     // One staged chunk: K codes at sk, V at sv (swizzled), fp8 row scales at
@@ -397,16 +399,17 @@ template <typename T, int D, bool TWO> struct GroupWarp {
                 }
                 vmax = fmaxf(vmax, __shfl_xor_sync(FULL, vmax, 1));
                 vmax = fmaxf(vmax, __shfl_xor_sync(FULL, vmax, 2));
-                const float rn = fmaxf(vref, vmax);
-                cr = vref / rn;
-                vref = rn;
-                const float inv = 1.f / rn;
+                if (vmax > vref) { // warp-uniform; R (and 1/R) change only here
+                    cr = vref / vmax;
+                    vref = vmax;
+                    vinv = 1.f / vmax;
+                }
                 // Tokens past the context have p = 0 and a zeroed scale.
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        pr[j][e] *= vs[j][e & 1] * inv;
+                        pr[j][e] *= vs[j][e & 1] * vinv;
             }
             if (__any_sync(FULL, c0 != 1.f || c1 != 1.f || cr != 1.f)) { // a max moved
                 const float f0 = c0 * cr, f1 = c1 * cr;
@@ -543,6 +546,7 @@ template <typename T, int D> struct GroupWarpT {
     float ma, mb;        // running maxima of heads 2q, 2q + 1
     float la, lb;        // this lane's tokens' share of their sums
     float vref;          // fp8: largest V scale so far (R), floored at FLT_MIN
+    float vinv;          // fp8: 1 / vref
 
     static __device__ __forceinline__ int piece_off(int t, int piece)
     {
@@ -590,6 +594,7 @@ template <typename T, int D> struct GroupWarpT {
         ma = mb = -INFINITY;
         la = lb = 0.f;
         vref = 1.17549435e-38f;
+        vinv = 1.f / vref;
     }
 
     // S^T of tokens t0 .. t0 + 15, even and odd k-steps in separate
@@ -692,11 +697,12 @@ template <typename T, int D> struct GroupWarpT {
 #pragma unroll
                 for (int sh = 4; sh < 32; sh <<= 1)
                     vmax = fmaxf(vmax, __shfl_xor_sync(FULL, vmax, sh));
-                const float rn = fmaxf(vref, vmax);
-                cr = vref / rn;
-                vref = rn;
-                const float inv = 1.f / rn;
-                const float w0 = v0 * inv, w1 = v1 * inv;
+                if (vmax > vref) { // warp-uniform; R (and 1/R) change only here
+                    cr = vref / vmax;
+                    vref = vmax;
+                    vinv = 1.f / vmax;
+                }
+                const float w0 = v0 * vinv, w1 = v1 * vinv;
                 p0 *= w0;
                 p1 *= w0;
                 p2 *= w1;
