@@ -47,7 +47,13 @@ constexpr int kSplitStages = PA_SPLIT_STAGES;
 #endif
 constexpr int kGroupWarps = PA_GROUP_WARPS;
 constexpr int kGroupStages = PA_GROUP_STAGES;
-constexpr int kTargetCtasPerSm = 12; // ~4 waves of 3 resident CTAs
+// Automatic partition of decode_split_kernel: halve 2048 while the grid
+// (sequences x heads x partitions at max_context_len) has fewer CTAs than
+// this many per SM, about 1.3 waves of 3 resident CTAs. B200, 8 sequences x
+// 32 layers (contexts of a few hundred tokens): 19.1 us per layer at 128
+// tokens (the floor, reached with 12 per SM), 15.1 us at 256 (this target),
+// 16.9 at 512; launches with more units are unaffected (2048).
+constexpr int kTargetCtasPerSm = 4;
 constexpr int kMinAutoPartition = 128;
 constexpr int kAutoPartition = 2048;
 // The grouped kernel streams best in long partitions. When it hands out the
@@ -165,7 +171,7 @@ bool rank_sequences(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c,
 // Partition (tokens per work unit) for a decode; >= max_context_len means a
 // single pass. Automatic choice for decode_split_kernel (one CTA row per
 // (sequence, query head)): 2048 tokens, halved (down to 128) while the grid
-// would give fewer than about four waves of resident CTAs. For
+// would give fewer than kTargetCtasPerSm CTAs per SM. For
 // decode_group_kernel (one CTA row per (sequence, K/V head)): 2048, halved
 // (down to 256) while the grid has fewer than 2 CTAs per SM.
 int choose_partition(int32_t num_seqs, int32_t num_heads, const pa_cache_desc *c,

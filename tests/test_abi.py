@@ -130,7 +130,7 @@ def test_workspace_and_partition_sizes(lib):
     assert lib.decode_partition_size(S, H, desc(H, d=D), 100, 0) == 128  # single, rounded to 32
     assert lib.decode_partition_size(96, 32, desc(32), 2048, 0) == 2048  # single pass
     assert lib.decode_partition_size(8, 32, desc(32), 32768, 0) == 2048
-    assert lib.decode_partition_size(1, 32, desc(32), 32768, 0) == 512
+    assert lib.decode_partition_size(1, 32, desc(32), 32768, 0) == 1024  # 32 x 32 CTAs
     assert lib.decode_partition_size(96, 32, desc(32), 2048, 1024) == 1024
     assert lib.decode_partition_size(1, 1, desc(1), 30000, 0) == 128
     # Grouped heads (2 <= G <= 16) on a 16-bit cache, or on an fp8 cache with
