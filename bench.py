@@ -756,13 +756,14 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # Warm-up (also measures how long the host takes to enqueue a step), then
-    # an untimed soak so clocks settle and get sampled.
+    # Warm-up (also measures how long the host takes to enqueue a step on the
+    # eager path with decode events, the slowest way a timed loop below
+    # enqueues one), then an untimed soak so clocks settle and get sampled.
     torch.cuda.synchronize(dev)
     t0 = time.perf_counter()
     for _ in range(args.warmup):
         flush_l2()
-        one_step()
+        one_step(([], []))
     host_step_s = (time.perf_counter() - t0) / args.warmup
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(device_uuid(torch, dev))
@@ -776,7 +777,7 @@ def main():
     def head_start():
         """Hold the GPU in a bounded sleep while the host queues the timed
         steps, so no step waits for a launch (at most about 1 s)."""
-        secs = min(1.0, 1.5 * args.steps * host_step_s + 0.002)
+        secs = min(1.0, 2.0 * args.steps * host_step_s + 0.002)
         torch.cuda._sleep(int(secs * 2.0e9))
 
     run_step = one_step

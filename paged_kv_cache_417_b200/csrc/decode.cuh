@@ -640,47 +640,25 @@ __device__ __forceinline__ void merge_partitions(const DecodeParams &p, int s, i
 // over 128 threads).
 constexpr int kMergeOutPerThread = 16;
 
-// Split counters: one 32-bit word per (sequence, head slot) in the
-// workspace, arrivals in the low 16 bits and published partials in the high
-// 16 (num_parts <= 65535 keeps both halves apart). Every word is zero
-// between calls: the merging CTA clears its own.
-//
-// merge_arrive (thread 0, right after the CTA's chunk loop): a relaxed add of
-// one arrival. The CTA whose add completes the count (num_parts - 1 arrivals
-// before it) will merge. The add only elects; it publishes nothing, so it is
-// issued before the CTA's epilogue and its round trip overlaps that work.
-__device__ __forceinline__ uint32_t merge_arrive(int32_t *word)
+// Arrival on a split counter: an atomic add with acquire-release semantics
+// at GPU scope. Release publishes every write the CTA ordered before it
+// (its barrier); acquire lets the last arriver see all earlier arrivers'
+// writes.
+__device__ __forceinline__ int arrive_acq_rel(int32_t *counter)
 {
-    uint32_t old;
-    asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], 1;"
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
                  : "=r"(old)
-                 : "l"(word)
+                 : "l"(counter)
                  : "memory");
     return old;
 }
 
-// Adds 1 << 16 (one published partial) with release semantics at GPU scope:
-// every write the CTA ordered before it (its barrier) is visible first.
-__device__ __forceinline__ void merge_publish(int32_t *word)
-{
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(word), "r"(1u << 16)
-                 : "memory");
-}
-
-__device__ __forceinline__ uint32_t load_acquire(const int32_t *word)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(word) : "memory");
-    return v;
-}
-
 // Called by every thread of a CTA that has just written the partials of
-// query heads h0 .. h0+nh-1 of sequence s; `arrived` is thread 0's value
-// from merge_arrive on word `slot`. A CTA that was not elected publishes its
-// partials and returns. The elected CTA waits (acquire loads, nanosleep
-// back-off, kWaitLimitNs; the others have all arrived, so they are running
-// and about to publish) until the other num_parts - 1 partials are
-// published, merges the heads into the output and clears the word. The
+// query heads h0 .. h0+nh-1 of sequence s: counts the CTA in on counter
+// `slot`; the CTA that completes the count (the last of the num_parts
+// partitions to finish) merges those heads into the output and resets the
+// counter to zero for the next call (the classic last-block pattern). The
 // merge turns each head's (m, l) pairs into normalised weights
 // 2^(m_p - M) / L in shared memory `wbuf` (nh * num_parts floats; one warp
 // per head, each lane holding up to kMergeLanePairs pairs, all heads' loads
@@ -691,29 +669,12 @@ __device__ __forceinline__ uint32_t load_acquire(const int32_t *word)
 constexpr int kMergeLanePairs = 4; // partitions per lane held in registers
 template <int D>
 __device__ __forceinline__ void merge_if_last(const DecodeParams &p, int s, int h0, int nh,
-                                              int slot, int num_parts, uint32_t arrived,
-                                              int tid, int nthreads, int *flag, float *wbuf)
+                                              int slot, int num_parts, int tid, int nthreads,
+                                              int *flag, float *wbuf)
 {
     __syncthreads();
-    if (tid == 0) {
-        const bool last = (arrived & 0xffffu) == (uint32_t)(num_parts - 1);
-        if (last) {
-            const uint32_t want = (uint32_t)(num_parts - 1);
-            if ((load_acquire(&p.ws_count[slot]) >> 16) != want) {
-                const uint64_t t0 = global_timer_ns();
-                while ((load_acquire(&p.ws_count[slot]) >> 16) != want) {
-                    if (global_timer_ns() - t0 > kWaitLimitNs) {
-                        report(p.dev_err, PA_DEVERR_TIMEOUT);
-                        break;
-                    }
-                    __nanosleep(32);
-                }
-            }
-        } else {
-            merge_publish(&p.ws_count[slot]);
-        }
-        *flag = last;
-    }
+    if (tid == 0)
+        *flag = arrive_acq_rel(&p.ws_count[slot]) == num_parts - 1;
     __syncthreads();
     if (!*flag)
         return;
@@ -982,9 +943,6 @@ __global__ void __launch_bounds__(NW * 32)
                            static_cast<const char *>(p.value_cache), (size_t)kvh * TILE,
                            (size_t)HK * TILE, p.num_blocks, table, u.n_tok, warp, NW, my_chunks,
                            rings + (size_t)warp * W::C::kRingBytes, smem_addr(&bars[warp * NS]));
-    uint32_t arrived = 0; // thread 0: arrivals before this CTA on its split counter
-    if (tid == 0 && u.num_parts > 1 && p.ws_count)
-        arrived = merge_arrive(&p.ws_count[s * H + h]);
     if (lane == 0) {
         if (!ok) {
             report(p.dev_err, PA_DEVERR_TIMEOUT);
@@ -1039,8 +997,8 @@ __global__ void __launch_bounds__(NW * 32)
         }
     }
     if (u.num_parts > 1 && p.ws_count)
-        merge_if_last<D>(p, s, h, 1, s * H + h, u.num_parts, arrived, tid, NW * 32,
-                         &cta_flags, reinterpret_cast<float *>(rings));
+        merge_if_last<D>(p, s, h, 1, s * H + h, u.num_parts, tid, NW * 32, &cta_flags,
+                         reinterpret_cast<float *>(rings));
 }
 
 // Separate merge kernel, for grids with more (sequence, head) slots than a

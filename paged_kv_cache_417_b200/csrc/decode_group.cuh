@@ -1037,9 +1037,6 @@ __global__ void __launch_bounds__(NW * 32)
             issued = i + NS + 1;
         }
     }
-    uint32_t arrived = 0; // thread 0: arrivals before this CTA on its split counter
-    if (tid == 0 && u.num_parts > 1 && p.ws_count)
-        arrived = merge_arrive(&p.ws_count[s * HK + kvh]);
     const bool timed_out = i < my_chunks;
     if (timed_out) {
         // Let the copies still in flight land before the ring is reused.
@@ -1130,8 +1127,8 @@ __global__ void __launch_bounds__(NW * 32)
         }
     }
     if (u.num_parts > 1 && p.ws_count)
-        merge_if_last<D>(p, s, kvh * G, G, s * HK + kvh, u.num_parts, arrived, tid, NW * 32,
-                         &cta_flags, reinterpret_cast<float *>(rings));
+        merge_if_last<D>(p, s, kvh * G, G, s * HK + kvh, u.num_parts, tid, NW * 32, &cta_flags,
+                         reinterpret_cast<float *>(rings));
 }
 
 } // namespace pagedkv
