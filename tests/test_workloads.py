@@ -125,3 +125,55 @@ def test_bf16_rounding_matches_torch():
     x = np.random.default_rng(0).standard_normal(10000).astype(np.float32) * 100
     ref = torch.from_numpy(x).bfloat16().view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(wl.to_storage_bits(x, "bf16"), ref)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "fp8"])
+def test_large_pool_tiles_are_distinct(monkeypatch, dtype):
+    """Pools with more tiles than the bank give every tile its own code (bank
+    row, sign mask): no two tiles hold the same values, each tile is its bank
+    row with whole token rows negated (fp8: the code bytes' sign bit; the row
+    scales untouched), and the device-side assembly gives the same bytes."""
+    import torch
+    import workloads.steps as steps
+    from workloads.device import device_pools
+    monkeypatch.setattr(steps, "MAX_BANK_ROWS", 64)
+    st = wl.tiny(seed=3, dtype=dtype)
+    R = st.base.shape[0]
+    assert R == 64
+    k, v = wl.host_pools(st)
+    L = st.layers[0]
+    NB, H, bs = st.num_blocks, st.num_kv_heads, st.block_size
+    tiles, codes = [], []
+    for pool, rows in ((k, L.tile_rows_k), (v, L.tile_rows_v)):
+        flat = pool.reshape(NB * H, -1)
+        live = (rows >= 0).reshape(-1)
+        tiles.append(flat[live])
+        codes.append(rows.reshape(-1)[live])
+    tiles, codes = np.concatenate(tiles), np.concatenate(codes)
+    assert len(tiles) > R                                   # the bank is reused...
+    assert len(np.unique(codes)) == len(codes)              # ...under distinct codes
+    assert len(np.unique(tiles, axis=0)) == len(tiles)      # and distinct contents
+    bank_row, flips = steps.tile_parts(codes, R, bs)
+    D = st.head_dim
+    for t in range(len(tiles)):
+        base = st.base[bank_row[t]]
+        got = tiles[t]
+        if dtype == "fp8":
+            c_got, c_base = got[: bs * D].reshape(bs, D), base[: bs * D].reshape(bs, D)
+            s_got, s_base = got[bs * D:].reshape(bs, 4), base[bs * D:].reshape(bs, 4)
+            signs = (c_got ^ c_base) == 0x80
+            nan = steps.E4M3_NAN
+        else:
+            c_got, c_base = got.reshape(bs, D), base.reshape(bs, D)
+            signs = (c_got ^ c_base) == 0x8000
+            nan = steps.nan_bits(dtype)
+        same = c_got == c_base
+        # Slots past a block's last token are NaN-filled: only live rows count.
+        for r in np.nonzero(~np.all(c_got == nan, axis=1))[0]:
+            assert signs[r].all() if flips[t, r] else same[r].all()
+            if dtype == "fp8":
+                assert np.array_equal(s_got[r], s_base[r])            # scales kept
+    if dtype != "fp8":
+        dk, dv = device_pools(st, 0, "cpu")
+        assert np.array_equal(dk.view(torch.int16).numpy().view(np.uint16), k)
+        assert np.array_equal(dv.view(torch.int16).numpy().view(np.uint16), v)

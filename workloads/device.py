@@ -1,8 +1,9 @@
 """Upload a :class:`~workloads.steps.DecodeStep` to a torch device.
 
-Plumbing only: the pools are assembled from the tile bank with torch indexing
-and NaN fills, exactly as :func:`workloads.steps.host_pools` does on the host,
-so both sides see the same bytes.
+Plumbing only: the pools are assembled from the tile bank with torch indexing,
+the tile codes' sign flips and NaN fills, exactly as
+:func:`workloads.steps.host_pools` does on the host, so both sides see the same
+bytes.
 """
 from __future__ import annotations
 
@@ -34,11 +35,16 @@ def device_pools(step: DecodeStep, layer: int, device, base_dev=None):
     nan = nan.view(TORCH_DTYPE[step.dtype]).item()
     valid = torch.from_numpy(step.valid_slots).to(device)
     slot_dead = torch.arange(bs, device=device)[None, :] >= valid[:, None]  # [NB, bs]
+    R = step.base.shape[0]
+    shifts = torch.arange(bs, device=device, dtype=torch.int64)
     pools = []
     for rows in (L.tile_rows_k, L.tile_rows_v):
         r = torch.from_numpy(rows).to(device)
-        p = base_dev.index_select(0, r.clamp(min=0).reshape(-1)).view(
-            step.num_blocks, H, bs, D)
+        code = r.clamp(min=0)
+        p = base_dev.index_select(0, (code % R).reshape(-1)).view(step.num_blocks, H, bs, D)
+        # Sign flips of the tile code's mask (workloads.steps.tile_parts).
+        flips = (((code // R)[..., None] >> shifts) & 1).to(torch.int16) * -32768
+        p = (p.view(torch.int16) ^ flips[..., None]).view(p.dtype)
         p.masked_fill_((r < 0)[:, :, None, None], nan)
         p.masked_fill_(slot_dead[:, None, :, None], nan)
         pools.append(p)

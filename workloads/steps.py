@@ -10,12 +10,17 @@ all of its context, the new token included.
 This module only draws numbers and builds integer tables. It holds none of the
 attention arithmetic, so it can feed both the CUDA path and the CPU oracle.
 
-Cache contents are stored compactly: every (block, head) tile of a pool is one
+Cache contents are stored compactly: every (block, head) tile of a pool is a
 row of a bank ``base`` of N(0,1) tiles (drawn in fp32, rounded to the storage
-type). Small pools get a distinct row per tile; large pools draw rows with
-replacement from a 32768-row bank, which keeps generation fast while every
-element is still an N(0,1) draw. Unused blocks, and slots past the last token
-of a partly filled block, hold NaN so that any read of them shows up.
+type), named by a tile code. Small pools get a distinct bank row per tile.
+Large pools use a 32768-row bank, which keeps generation fast, and give every
+tile a distinct code (bank row, sign mask): the tile is the bank row with the
+sign of its token row r flipped where bit r of the mask is set (fp8: the code
+bytes' sign bit; the row scales stay). A sign flip is exact in every storage
+format and keeps every element an N(0,1) draw, and no two tiles of a pool hold
+the same values, so a kernel that reads the wrong tile cannot land on equal
+contents. Unused blocks, and slots past the last token of a partly filled
+block, hold NaN so that any read of them shows up.
 """
 from __future__ import annotations
 
@@ -31,6 +36,32 @@ BF16_NAN = np.uint16(0x7FC0)
 E4M3_NAN = np.uint8(0x7F)
 F32_NAN_BYTES = np.array([np.nan], dtype=np.float32).view(np.uint8)
 MAX_BANK_ROWS = 32768
+
+
+MASK_BITS = 16  # token rows of a tile whose sign a tile code can flip
+
+
+def tile_parts(codes: np.ndarray, bank_rows: int, block_size: int):
+    """Split tile codes (>= 0) into bank rows and per-token-row sign flips:
+    code = mask * bank_rows + row; flips[..., r] = bit r of mask."""
+    codes = np.asarray(codes, dtype=np.int64)
+    rows = codes % bank_rows
+    mask = codes // bank_rows
+    flips = (mask[..., None] >> np.arange(block_size, dtype=np.int64)) & 1
+    return rows, flips.astype(bool)
+
+
+def _distinct_codes(rng, n: int, bank_rows: int, block_size: int) -> np.ndarray:
+    """n distinct tile codes: bank rows with sign masks, drawn uniformly."""
+    space = bank_rows << min(block_size, MASK_BITS)
+    codes = rng.integers(0, space, size=n)
+    while True:
+        uniq, first = np.unique(codes, return_index=True)
+        if len(uniq) == n:
+            return codes
+        dup = np.ones(n, dtype=bool)
+        dup[first] = False
+        codes[dup] = rng.integers(0, space, size=int(dup.sum()))
 
 
 def fp8_tile_bytes(block_size: int, head_dim: int) -> int:
@@ -69,7 +100,7 @@ class LayerInputs:
     query: np.ndarray       # uint16 [S, H, D]
     new_key: np.ndarray     # uint16 [S, H, D]
     new_value: np.ndarray   # uint16 [S, H, D]
-    tile_rows_k: np.ndarray  # int64 [NB, Hkv], row of ``base`` or -1 (NaN tile)
+    tile_rows_k: np.ndarray  # int64 [NB, Hkv], tile code (see tile_parts) or -1 (NaN tile)
     tile_rows_v: np.ndarray  # int64 [NB, Hkv]
 
 
@@ -200,7 +231,7 @@ def build_step(rng, name, *, num_blocks, block_size, num_heads, head_dim,
         if n_tiles <= rows:
             pick = rng.permutation(rows)[:n_tiles] if n_tiles else np.zeros(0, np.int64)
         else:
-            pick = rng.integers(0, rows, size=n_tiles)
+            pick = _distinct_codes(rng, n_tiles, rows, bs)
         pick = pick.astype(np.int64).reshape(2, len(filled), Hk) if n_tiles else \
             np.zeros((2, 0, Hk), np.int64)
         tk = np.full((num_blocks, Hk), -1, dtype=np.int64)
@@ -326,10 +357,12 @@ def host_pools(step: DecodeStep, layer: int = 0):
     if step.dtype == "fp8":
         return _host_pools_fp8(step, L)
     nan = nan_bits(step.dtype)
+    R = step.base.shape[0]
     pools = []
     for rows in (L.tile_rows_k, L.tile_rows_v):
-        p = step.base[np.maximum(rows, 0).reshape(-1)].reshape(
-            step.num_blocks, H, bs, D).copy()
+        bank_row, flips = tile_parts(np.maximum(rows, 0), R, bs)
+        p = step.base[bank_row.reshape(-1)].reshape(step.num_blocks, H, bs, D).copy()
+        p ^= np.where(flips, np.uint16(0x8000), np.uint16(0))[..., None]
         p[rows < 0] = nan
         mask = np.arange(bs)[None, :] >= step.valid_slots[:, None]
         p.transpose(0, 2, 1, 3)[mask] = nan
@@ -341,11 +374,14 @@ def _host_pools_fp8(step, L):
     bs, H, D = step.block_size, step.num_kv_heads, step.head_dim
     tb = fp8_tile_bytes(bs, D)
     dead = np.arange(bs)[None, :] >= step.valid_slots[:, None]          # [NB, bs]
+    R = step.base.shape[0]
     pools = []
     for rows in (L.tile_rows_k, L.tile_rows_v):
-        p = step.base[np.maximum(rows, 0).reshape(-1)].reshape(step.num_blocks, H, tb).copy()
-        p[rows < 0] = E4M3_NAN
+        bank_row, flips = tile_parts(np.maximum(rows, 0), R, bs)
+        p = step.base[bank_row.reshape(-1)].reshape(step.num_blocks, H, tb).copy()
         codes = p[:, :, : bs * D].reshape(step.num_blocks, H, bs, D)
+        codes ^= np.where(flips, np.uint8(0x80), np.uint8(0))[..., None]
+        p[rows < 0] = E4M3_NAN
         scales = p[:, :, bs * D:].reshape(step.num_blocks, H, bs, 4)
         codes.transpose(0, 2, 1, 3)[dead] = E4M3_NAN
         scales.transpose(0, 2, 1, 3)[dead] = F32_NAN_BYTES
