@@ -161,9 +161,9 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
 // One warp's share of a group: the G query rows of a (sequence, K/V head) as
 // the A operand, the output accumulator fragments and the online-softmax
 // state, and the math that consumes one staged chunk (the header comment
-// above describes it). T: __half, __nv_bfloat16 or E4M3; TWO: G > 8
-// (fragment rows 8-15 are live).
-template <typename T, int D, bool TWO> struct GroupWarp {
+// above describes it), for 8 < G <= 16: both fragment row halves are live
+// (G <= 8 takes GroupWarpT). T: __half, __nv_bfloat16 or E4M3.
+template <typename T, int D> struct GroupWarp {
     using Geo = GroupGeom<T, D>;
     static constexpr bool kFp8 = Geo::kFp8;
     static constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
@@ -244,9 +244,9 @@ template <typename T, int D, bool TWO> struct GroupWarp {
             const int c = kFp8 ? (16 * kk + 4 * q) / 2 : (16 * kk + q2) / 2;
             const int c2 = kFp8 ? c + 1 : c + 4;
             qa[kk][0] = g0 < G ? qp[r0 + c] : 0u;
-            qa[kk][1] = TWO && g1 < G ? qp[r1 + c] : 0u;
+            qa[kk][1] = g1 < G ? qp[r1 + c] : 0u;
             qa[kk][2] = g0 < G ? qp[r0 + c2] : 0u;
-            qa[kk][3] = TWO && g1 < G ? qp[r1 + c2] : 0u;
+            qa[kk][3] = g1 < G ? qp[r1 + c2] : 0u;
         }
     }
 
@@ -359,25 +359,18 @@ template <typename T, int D, bool TWO> struct GroupWarp {
                 pr[j][1] = exp2f(x[j][1] - mn0);
             }
             l0 = fmaf(l0, c0, (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
-            float c1 = 1.f;
-            if constexpr (TWO) {
-                float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
-                const float mn1 = fmaxf(m1, mx1);
-                c1 = exp2f(m1 - mn1);
-                m1 = mn1;
+            float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
+            const float mn1 = fmaxf(m1, mx1);
+            const float c1 = exp2f(m1 - mn1);
+            m1 = mn1;
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    pr[j][2] = exp2f(x[j][2] - mn1);
-                    pr[j][3] = exp2f(x[j][3] - mn1);
-                }
-                l1 = fmaf(l1, c1, (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]));
-            } else {
-#pragma unroll
-                for (int j = 0; j < 2; ++j)
-                    pr[j][2] = pr[j][3] = 0.f;
+            for (int j = 0; j < 2; ++j) {
+                pr[j][2] = exp2f(x[j][2] - mn1);
+                pr[j][3] = exp2f(x[j][3] - mn1);
             }
+            l1 = fmaf(l1, c1, (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]));
             float cr = 1.f; // fp8: R_old / R_new
             if constexpr (kFp8) {
                 // Fold the V scales into P relative to R (tokens past the
@@ -417,10 +410,8 @@ template <typename T, int D, bool TWO> struct GroupWarp {
                 for (int j = 0; j < 2 * KT; ++j) {
                     o[j][0] *= f0;
                     o[j][1] *= f0;
-                    if constexpr (TWO) {
-                        o[j][2] *= f1;
-                        o[j][3] *= f1;
-                    }
+                    o[j][2] *= f1;
+                    o[j][3] *= f1;
                 }
             }
 
@@ -495,13 +486,11 @@ template <typename T, int D, bool TWO> struct GroupWarp {
                 mw[g0 * MS + D + 1] = l0;
             }
         }
-        if constexpr (TWO) {
-            if (g1 < G) {
-                store_row(mw + g1 * MS, 2, oscale);
-                if ((lane & 3) == 0) {
-                    mw[g1 * MS + D] = m1;
-                    mw[g1 * MS + D + 1] = l1;
-                }
+        if (g1 < G) {
+            store_row(mw + g1 * MS, 2, oscale);
+            if ((lane & 3) == 0) {
+                mw[g1 * MS + D] = m1;
+                mw[g1 * MS + D + 1] = l1;
             }
         }
     }
@@ -873,7 +862,9 @@ template <typename T, int D, int BS> struct NewRow {
 };
 
 // decode_group_kernel: one CTA per (K/V head, sequence, partition) of a
-// fixed partition size; grid (num_kv_heads, num_seqs, num_parts).
+// fixed partition size; grid (num_kv_heads, num_seqs, num_parts). TWO: the
+// launch has G > 8 (heads as tile rows, GroupWarp); else the transposed
+// GroupWarpT.
 template <typename T, int D, int BS, int NW, int NS, bool TWO>
 __global__ void __launch_bounds__(NW * 32)
     decode_group_kernel(const __grid_constant__ GroupParams gp)
@@ -881,7 +872,7 @@ __global__ void __launch_bounds__(NW * 32)
     using Cfg = GroupCfg<T, D, BS, NW, NS>;
     static_assert(kGroupMaxHeads * D <= kMergeOutPerThread * NW * 32, "merge_if_last capacity");
     // G > 8: heads as tile rows; G <= 8: the transposed orientation.
-    using Wp = typename std::conditional<TWO, GroupWarp<T, D, true>, GroupWarpT<T, D>>::type;
+    using Wp = typename std::conditional<TWO, GroupWarp<T, D>, GroupWarpT<T, D>>::type;
     constexpr bool kFp8 = Cfg::kFp8;
     constexpr int CH = Cfg::kChunk, SEG = Cfg::kSeg, ROW = Cfg::kRow;
     constexpr int MS = Cfg::kMergeStride;
