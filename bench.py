@@ -337,6 +337,37 @@ def max_over_ranks(x, dist=None, device=None):
     return float(t.item())
 
 
+# The suite's other workloads, measured briefly after the default one's line
+# is timed (one GPU, default workload), each by this script in a child
+# process with its own warm-up, L2 flushes, CUDA-event timing and clocks.
+OTHER_CONFIGS = (("long_context", 30), ("prefix_cow", 100), ("full_step_bs16", 10))
+
+
+def other_config_runs(warmup):
+    """A compact record of each other workload's own JSON line."""
+    out = []
+    for name, steps in OTHER_CONFIGS:
+        cmd = [sys.executable, os.path.abspath(__file__), "--config", name, "--steps",
+               str(steps), "--warmup", str(max(3, warmup)), "--soak-seconds", "0.3",
+               "--no-e2e", "--no-cpu-baseline", "--no-other-configs"]
+        try:
+            res = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
+            d = json.loads(res.stdout.strip().splitlines()[-1])
+            r = d["roofline"]
+            out.append({"config": name, "workload": d["config"]["workload"],
+                        "value": d["value"], "unit": d["unit"], "steps": d["steps"],
+                        "ms_per_step": d["ms_per_step"], "decode_us": r["decode_us"],
+                        "roofline_frac": r["frac"], "frac_of_8tbs": r["frac_of_8tbs"],
+                        "traffic": r["traffic"], "partition_size": d["partition_size"],
+                        "clocks": d["clocks"]})
+            if name == "prefix_cow":
+                out[-1]["note"] = ("fractions count logical bytes: the shared prefix is read "
+                                   "once from HBM and then from L2, by design of the workload")
+        except Exception as e:  # reported in the line, never fatal to it
+            out.append({"config": name, "error": f"{type(e).__name__}: {e}"[:300]})
+    return out
+
+
 def job_throughput(world, seqs_per_rank, steps, max_ms):
     """Query tokens of all ranks per second of the slowest rank."""
     return world * seqs_per_rank * steps / (max_ms / 1e3)
@@ -681,6 +712,9 @@ def main():
                          "library's C++ one (default) or the Python allocator of workloads/")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the short runs of the other workloads that a default "
+                         "single-GPU run appends to its line")
     args = ap.parse_args()
     args.fused = not args.separate
     args.graph = not args.no_graph
@@ -907,6 +941,11 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, acc = cpu_baseline(step, timed_outs)
     bm_timing = block_manager_timing(step) if rank == 0 else None
+    others = None
+    if (rank == 0 and world == 1 and args.config == "llama7b_layer" and args.kv_dtype == "f16"
+            and not args.kv_heads and not args.seqs and not args.separate and args.graph
+            and not args.no_other_configs):
+        others = other_config_runs(args.warmup)
 
     if rank == 0:
         line = {
@@ -919,7 +958,7 @@ def main():
             "max_abs_err": acc["max_abs_err"] if acc else None, "accuracy": acc,
             "gpu_launches": launcher.launches_per_step * args.steps, "clocks": clocks,
             "host_paced_value": paced, "host_block_manager": bm_timing, "swap": swap_stats,
-            "partition_size": P, "split": split,
+            "partition_size": P, "split": split, "other_configs": others,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
