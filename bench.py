@@ -340,16 +340,24 @@ def max_over_ranks(x, dist=None, device=None):
 # The suite's other workloads, measured briefly after the default one's line
 # is timed (one GPU, default workload), each by this script in a child
 # process with its own warm-up, L2 flushes, CUDA-event timing and clocks.
-OTHER_CONFIGS = (("long_context", 30), ("prefix_cow", 100), ("full_step_bs16", 10))
+OTHER_CONFIGS = (
+    ("long_context", ["--config", "long_context"], 30),
+    ("prefix_cow", ["--config", "prefix_cow"], 100),
+    ("full_step_bs16", ["--config", "full_step_bs16"], 10),
+    ("llama7b_layer_fp8", ["--kv-dtype", "fp8"], 100),
+    ("llama7b_layer_kvh8", ["--kv-heads", "8"], 100),
+    ("llama7b_layer_kvh2", ["--kv-heads", "2"], 100),
+    ("llama7b_layer_fp8_kvh8", ["--kv-dtype", "fp8", "--kv-heads", "8"], 100),
+)
 
 
 def other_config_runs(warmup):
     """A compact record of each other workload's own JSON line."""
     out = []
-    for name, steps in OTHER_CONFIGS:
-        cmd = [sys.executable, os.path.abspath(__file__), "--config", name, "--steps",
-               str(steps), "--warmup", str(max(3, warmup)), "--soak-seconds", "0.3",
-               "--no-e2e", "--no-cpu-baseline", "--no-other-configs"]
+    for name, extra, steps in OTHER_CONFIGS:
+        cmd = [sys.executable, os.path.abspath(__file__), *extra, "--steps", str(steps),
+               "--warmup", str(max(3, warmup)), "--soak-seconds", "0.3", "--no-e2e",
+               "--no-cpu-baseline", "--no-other-configs"]
         try:
             res = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
             d = json.loads(res.stdout.strip().splitlines()[-1])
