@@ -359,7 +359,7 @@ def other_config_runs(warmup):
                "--warmup", str(max(3, warmup)), "--soak-seconds", "0.3", "--no-e2e",
                "--no-cpu-baseline", "--no-other-configs"]
         try:
-            res = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
+            res = subprocess.run(cmd, capture_output=True, text=True, timeout=300)
             d = json.loads(res.stdout.strip().splitlines()[-1])
             r = d["roofline"]
             out.append({"config": name, "workload": d["config"]["workload"],
