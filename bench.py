@@ -43,7 +43,7 @@ import workloads as wl  # noqa: E402
 
 METRIC = "paged-attn decode query-tokens/s; achieved KV-read HBM GB/s vs B200 peak"
 UNIT = "query-tokens/s"
-NORTH_STAR_PEAK_GBS = 8000.0
+NOMINAL_PEAK_GBS = 8000.0  # the B200's nominal ~8 TB/s HBM3e bandwidth
 FALLBACK_PEAK_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
@@ -891,7 +891,7 @@ def main():
                 "kv_bytes_per_launch": ab["kv"],
                 "decode_us": dec_avg_s * 1e6,
                 "kv_gbs": ab["kv"] / dec_avg_s / 1e9,
-                "frac_of_8tbs": achieved / NORTH_STAR_PEAK_GBS}
+                "frac_of_8tbs": achieved / NOMINAL_PEAK_GBS}
 
     swap_stats = None
     if swap is not None:
