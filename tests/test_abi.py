@@ -131,6 +131,9 @@ def test_workspace_and_partition_sizes(lib):
     assert lib.decode_partition_size(96, 32, desc(32), 2048, 0) == 2048  # single pass
     assert lib.decode_partition_size(8, 32, desc(32), 32768, 0) == 2048
     assert lib.decode_partition_size(1, 32, desc(32), 32768, 0) == 1024  # 32 x 32 CTAs
+    # 8 sequences x 32 heads, contexts up to ~600 tokens (the small-batch
+    # step): halved until the grid has 4 CTAs per SM (256 x 3 >= 4 x 148)
+    assert lib.decode_partition_size(8, 32, desc(32), 600, 0) == 256
     assert lib.decode_partition_size(96, 32, desc(32), 2048, 1024) == 1024
     assert lib.decode_partition_size(1, 1, desc(1), 30000, 0) == 128
     # Grouped heads (2 <= G <= 16) on a 16-bit cache, or on an fp8 cache with

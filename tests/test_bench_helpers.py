@@ -3,7 +3,6 @@ it divides by, and when an ncu traffic record is trusted. No GPU needed."""
 import json
 import os
 
-import numpy as np
 import pytest
 
 import bench
@@ -95,3 +94,14 @@ def test_committed_traffic_records_are_well_formed():
 def test_job_throughput_counts_every_rank():
     # 2 ranks x 96 sequences x 10 steps in 5 ms of the slowest rank
     assert bench.job_throughput(2, 96, 10, 5.0) == pytest.approx(2 * 96 * 10 / 5e-3)
+
+
+def test_other_configs_name_real_workloads():
+    """The short extra runs of a default bench line use workloads and flags
+    the script accepts."""
+    for name, extra, steps in bench.OTHER_CONFIGS:
+        assert steps > 0
+        if "--config" in extra:
+            assert extra[extra.index("--config") + 1] in bench.WORKLOADS, name
+        if "--kv-dtype" in extra:
+            assert extra[extra.index("--kv-dtype") + 1] in ("f16", "bf16", "fp8"), name
